@@ -1,0 +1,276 @@
+"""Checks that pin the float64 oracle to facts other than itself.
+
+Each pin_* function takes a loaded oracle library (so the mutation test can run the same
+checks against deliberately broken copies) and raises AssertionError on failure.  The
+facts come from the pages' printed figures (tests/golden/page_figures.json), closed forms,
+library routines for special cases (torch's scaled-dot-product attention, numpy matmul and
+complex exponentials) and invariants.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden", "page_figures.json")
+
+
+def _rs(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol, what=""):
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    scale = max(1.0, float(np.sqrt(np.mean(b * b))) if b.size else 1.0)
+    assert err <= tol * scale, f"{what}: max abs err {err:.3e} > {tol:.1e} * {scale:.3e}"
+
+
+def _sdpa(q, k, v, scale, causal=False):
+    """torch's attention on float64 CPU tensors: q [Lq, d], k [Lk, d], v [Lk, dv]."""
+    t = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float64))[None, None]
+    out = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), scale=scale, is_causal=causal)
+    return out[0, 0].numpy()
+
+
+# ------------------------------------------------------------------ page figures
+
+def pin_page_figures(lib):
+    g = json.load(open(GOLDEN))
+    m = g["mha_kv_bytes_per_token"]
+    b = oracle.mha_elems_per_token(m["heads"], m["d_head"], lib) * m["layers"] * m["bytes_per_elem"]
+    assert b == m["value_bytes"] == 512 * 1024, b
+    c = g["mha_100k_context"]
+    gb = b * c["tokens"] / 1e9
+    assert abs(gb - c["printed_gb"]) / c["printed_gb"] <= c["rel_tol"], gb
+    t = g["memory_table"]
+    mha = oracle.mha_elems_per_token(1, t["d_model"], lib)      # H * d_head = d_model
+    mla = oracle.mla_elems_per_token(t["d_c"], t["d_hR"], 1, lib)
+    assert mha == t["mha_values"] and mla == t["mla_values"], (mha, mla)
+    assert math.floor(mha / mla * 10) / 10 == t["printed_ratio"]   # the page truncates 17.78
+    mha_gb = mha * t["tokens"] * t["layers"] * t["bytes_per_elem"] / 1e9
+    mla_gb = mla * t["tokens"] * t["layers"] * t["bytes_per_elem"] / 1e9
+    assert abs(mha_gb - t["printed_mha_gb"]) / t["printed_mha_gb"] <= t["gb_rel_tol"], mha_gb
+    assert math.floor(mla_gb * 10) / 10 == t["printed_mla_gb"], mla_gb
+    q = g["gqa_equivalence"]
+    assert 2 * q["groups"] * q["d_head"] == oracle.mla_elems_per_token(q["d_c"], q["d_hR"], 1, lib)
+    v = g["v3_cache_example"]
+    e = oracle.mla_elems_per_token(v["kv_lora_rank"], v["qk_rope_head_dim"], v["num_hidden_layers"], lib)
+    assert e == v["elements_per_token"], e
+    assert e * v["bytes_per_elem"] * v["context"] / 2 ** 30 == v["gib"]
+
+
+# ------------------------------------------------------------------- rounding
+
+def pin_round_bf16(lib):
+    cases = {
+        1.0: 0x3F80, -2.5: 0xC020, 0.0: 0x0000,
+        1.0 + 2 ** -8: 0x3F80,               # exact tie -> even mantissa (0)
+        1.0 + 3 * 2 ** -8: 0x3F82,           # exact tie -> even mantissa (2)
+        1.0 + 2 ** -8 + 2 ** -30: 0x3F81,    # just above the tie: one rounding, not two
+        2.0 ** -130: 0x0008,                 # subnormal
+    }
+    for x, want in cases.items():
+        got = int(lib.oracle_round_bf16(x))
+        assert got == want, f"round_bf16({x!r}) = {got:#06x}, want {want:#06x}"
+    # values already in float32: torch's float32 -> bfloat16 cast (nearest-even) agrees
+    x = _rs(1).standard_normal(4096).astype(np.float32) * np.float32(7.0)
+    ref = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(oracle.round_bf16(x.astype(np.float64), lib), ref)
+
+
+# ------------------------------------------------------------------------ RoPE
+
+def pin_rope(lib):
+    r = _rs(2)
+    d = 16
+    x = r.standard_normal(d)
+    assert np.array_equal(oracle.rope(x, 0.0, 10000.0, lib), x)                 # position 0
+    # closed form per pair as a complex rotation z * e^{i pos theta^(-2i/d)}
+    for pos in (1.0, 7.0, 4096.0, 8192.0):
+        y = oracle.rope(x, pos, 10000.0, lib)
+        z = x[0::2] + 1j * x[1::2]
+        w = z * np.exp(1j * pos * 10000.0 ** (-2.0 * np.arange(d // 2) / d))
+        _close(y[0::2], w.real, 1e-12, "rope real")
+        _close(y[1::2], w.imag, 1e-12, "rope imag")
+        _close(np.hypot(y[0::2], y[1::2]), np.abs(z), 1e-12, "rope norm")
+    # sign convention on one pair: [1, 0] at angle pi/2 -> [0, 1]
+    _close(oracle.rope(np.array([1.0, 0.0]), math.pi / 2, 10000.0, lib), [0.0, 1.0], 1e-15, "rope sign")
+    # the score of two rotated vectors depends only on the position difference
+    q, k = r.standard_normal(d), r.standard_normal(d)
+    a = oracle.rope(q, 100.0, 10000.0, lib) @ oracle.rope(k, 37.0, 10000.0, lib)
+    b = oracle.rope(q, 163.0, 10000.0, lib) @ oracle.rope(k, 100.0, 10000.0, lib)
+    assert abs(a - b) <= 1e-10 * max(1.0, abs(a)), (a, b)
+
+
+# ---------------------------------------------------------- cache rows / query
+
+def pin_latent_rows(lib):
+    r = _rs(3)
+    n, d_model, d_c, d_hR = 5, 24, 12, 8
+    h = r.standard_normal((n, d_model))
+    W_DKV = r.standard_normal((d_c, d_model))
+    W_KR = r.standard_normal((d_hR, d_model))
+    pos = np.array([0, 1, 5, 100, 4097])
+    rows = oracle.latent_rows(h, W_DKV, W_KR, pos, 10000.0, lib)
+    assert rows.shape == (n, d_c + d_hR)
+    _close(rows[:, :d_c], h @ W_DKV.T, 1e-12, "latent c vs matmul")
+    # the rotary part, against the complex-exponential closed form of the rotation
+    kr = h @ W_KR.T
+    for i, p in enumerate(pos):
+        z = kr[i, 0::2] + 1j * kr[i, 1::2]
+        w = z * np.exp(1j * p * 10000.0 ** (-2.0 * np.arange(d_hR // 2) / d_hR))
+        _close(rows[i, d_c::2], w.real, 1e-12, "k_rope real")
+        _close(rows[i, d_c + 1::2], w.imag, 1e-12, "k_rope imag")
+    # a unit hidden state picks one column of each weight; at position 0 nothing rotates
+    e = np.zeros((1, d_model)); e[0, 3] = 1.0
+    row = oracle.latent_rows(e, W_DKV, W_KR, [0], 10000.0, lib)[0]
+    assert np.array_equal(row, np.concatenate([W_DKV[:, 3], W_KR[:, 3]]))
+
+
+def pin_query(lib):
+    r = _rs(4)
+    H, qk_nope, d_hR, d_model = 3, 4, 6, 10
+    W_Q = r.standard_normal((H * (qk_nope + d_hR), d_model))
+    e = np.zeros((1, d_model)); e[0, 7] = 1.0
+    qn, qr = oracle.query(e, W_Q, [0], H, qk_nope, d_hR, 10000.0, lib)
+    col = W_Q[:, 7].reshape(H, qk_nope + d_hR)        # head-major, content rows first
+    assert np.array_equal(qn[0], col[:, :qk_nope]) and np.array_equal(qr[0], col[:, qk_nope:])
+    h = r.standard_normal((2, d_model))
+    qn, qr = oracle.query(h, W_Q, [3, 11], H, qk_nope, d_hR, 10000.0, lib)
+    q = (h @ W_Q.T).reshape(2, H, qk_nope + d_hR)
+    _close(qn, q[:, :, :qk_nope], 1e-12, "q_nope vs matmul")
+    for i, p in enumerate((3, 11)):
+        z = q[i, :, qk_nope::2] + 1j * q[i, :, qk_nope + 1::2]
+        w = z * np.exp(1j * p * 10000.0 ** (-2.0 * np.arange(d_hR // 2) / d_hR))
+        _close(qr[i, :, 0::2], w.real, 1e-12, "q_rope real")
+        _close(qr[i, :, 1::2], w.imag, 1e-12, "q_rope imag")
+
+
+# ------------------------------------------------------------------- decode
+
+def _tiny(seed, T=23, d_c=16, d_hR=8, qk_nope=8, v_head=8):
+    r = _rs(seed)
+    return dict(q_nope=r.standard_normal(qk_nope), q_rope=r.standard_normal(d_hR),
+                rows=r.standard_normal((T, d_c + d_hR)), W_UK_h=r.standard_normal((qk_nope, d_c)) / 4,
+                W_UV_h=r.standard_normal((v_head, d_c)) / 4)
+
+
+def pin_decode_vs_library_attention(lib):
+    for seed, T in ((5, 1), (6, 23), (7, 64)):
+        a = _tiny(seed, T)
+        d_c = a["W_UK_h"].shape[1]
+        scale = 1 / math.sqrt(8 + 8)
+        o, p, lse = oracle.attend(**a, scale=scale, lib=lib)
+        c, kr = a["rows"][:, :d_c], a["rows"][:, d_c:]
+        K = np.concatenate([c @ a["W_UK_h"].T, kr], axis=1)
+        V = c @ a["W_UV_h"].T
+        q = np.concatenate([a["q_nope"], a["q_rope"]])[None]
+        _close(o, _sdpa(q, K, V, scale)[0], 1e-12, "decode vs torch sdpa")
+        s = scale * (K @ q[0])
+        assert abs(lse - float(torch.logsumexp(torch.from_numpy(s), 0))) <= 1e-12 * max(1, abs(lse))
+        assert abs(p.sum() - 1.0) <= 1e-12 and np.all(p > 0)
+
+
+def pin_decode_textbook_reduction(lib):
+    """qk_nope = v_head = d_c, W_UK = W_UV = I, q_rope = 0: single-KV-head attention on c."""
+    r = _rs(8)
+    T, d_c, d_hR = 31, 12, 4
+    rows = r.standard_normal((T, d_c + d_hR))
+    I = np.eye(d_c)
+    qn = r.standard_normal(d_c)
+    for absorbed in (False, True):
+        o, _, _ = oracle.attend(qn, np.zeros(d_hR), rows, I, I, 0.3, absorbed, lib)
+        _close(o, _sdpa(qn[None], rows[:, :d_c], rows[:, :d_c], 0.3)[0], 1e-12, "textbook mqa")
+
+
+def pin_decode_score_split(lib):
+    """score = content + positional: with q_nope = 0 only the rotary keys decide p."""
+    a = _tiny(9, 17)
+    d_c = a["W_UK_h"].shape[1]
+    a["q_nope"] = np.zeros_like(a["q_nope"])
+    o, _, _ = oracle.attend(**a, scale=0.25, lib=lib)
+    c, kr = a["rows"][:, :d_c], a["rows"][:, d_c:]
+    _close(o, _sdpa(a["q_rope"][None], kr, c @ a["W_UV_h"].T, 0.25)[0], 1e-12, "positional only")
+
+
+def pin_decode_special_cases(lib):
+    a = _tiny(10, 1)
+    d_c = a["W_UK_h"].shape[1]
+    o, p, _ = oracle.attend(**a, scale=0.5, lib=lib)                # one row: p = 1
+    _close(o, a["W_UV_h"] @ a["rows"][0, :d_c], 1e-13, "T=1")
+    a = _tiny(11, 9)
+    a["q_nope"][:] = 0; a["q_rope"][:] = 0                          # zero query: uniform p
+    o, p, _ = oracle.attend(**a, scale=0.5, lib=lib)
+    _close(p, np.full(9, 1 / 9), 1e-15, "uniform p")
+    _close(o, (a["rows"][:, :d_c] @ a["W_UV_h"].T).mean(0), 1e-13, "mean of v")
+    a = _tiny(12, 29)                                                # keys are a set
+    o1, _, _ = oracle.attend(**a, scale=0.5, lib=lib)
+    a["rows"] = a["rows"][_rs(13).permutation(29)]
+    o2, _, _ = oracle.attend(**a, scale=0.5, lib=lib)
+    _close(o1, o2, 1e-13, "permutation")
+
+
+def pin_naive_equals_absorbed(lib):
+    """Absorption is an exact re-association: naive and absorbed agree in float64."""
+    for seed, T, d_c, qk, v in ((14, 40, 16, 8, 8), (15, 3, 32, 12, 20), (16, 129, 64, 32, 32)):
+        a = _tiny(seed, T, d_c=d_c, d_hR=16 if d_c == 64 else 8, qk_nope=qk, v_head=v)
+        on, pn, ln = oracle.attend(**a, scale=0.2, absorbed=False, lib=lib)
+        oa, pa, la = oracle.attend(**a, scale=0.2, absorbed=True, lib=lib)
+        _close(on, oa, 1e-10, "naive vs absorbed o")
+        _close(pn, pa, 1e-10, "naive vs absorbed p")
+        assert abs(ln - la) <= 1e-10 * max(1, abs(ln))
+
+
+def pin_decode_batch_driver(lib):
+    r = _rs(17)
+    B, H, d_c, d_hR, qk, v = 3, 2, 16, 8, 8, 8
+    lens = [5, 0, 11]
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    rows = r.standard_normal((offs[-1], d_c + d_hR))
+    qn, qr = r.standard_normal((B, H, qk)), r.standard_normal((B, H, d_hR))
+    WUK, WUV = r.standard_normal((H, qk, d_c)), r.standard_normal((H, v, d_c))
+    o, lse = oracle.decode(qn, qr, rows, offs, WUK, WUV, 0.3, lib=lib)
+    for b in range(B):
+        for h in range(H):
+            rr = rows[offs[b]:offs[b + 1]]
+            if len(rr) == 0:
+                assert np.all(o[b, h] == 0) and lse[b, h] == -np.inf     # empty sequence
+                continue
+            d = rr[:, :d_c]
+            K = np.concatenate([d @ WUK[h].T, rr[:, d_c:]], 1)
+            ref = _sdpa(np.concatenate([qn[b, h], qr[b, h]])[None], K, d @ WUV[h].T, 0.3)[0]
+            _close(o[b, h], ref, 1e-12, f"batch b={b} h={h}")
+
+
+def pin_out_proj(lib):
+    r = _rs(18)
+    o = r.standard_normal((3, 4, 5))
+    W_O = r.standard_normal((7, 20))
+    _close(oracle.out_proj(o, W_O, lib), o.reshape(3, 20) @ W_O.T, 1e-12, "out proj")
+
+
+def pin_prefill(lib):
+    r = _rs(19)
+    S, d_c, d_hR, qk, v = 13, 16, 8, 8, 12
+    rows = r.standard_normal((S, d_c + d_hR))
+    qn, qr = r.standard_normal((S, qk)), r.standard_normal((S, d_hR))
+    WUK, WUV = r.standard_normal((qk, d_c)) / 4, r.standard_normal((v, d_c)) / 4
+    t = np.arange(S)
+    c = rows[:, :d_c]
+    K = np.concatenate([c @ WUK.T, rows[:, d_c:]], 1)
+    ref = _sdpa(np.concatenate([qn, qr], 1), K, c @ WUV.T, 0.3, causal=True)
+    for absorbed in (False, True):
+        o = oracle.prefill_head(qn, qr, rows, WUK, WUV, 0.3, t, absorbed, lib)
+        _close(o, ref, 1e-12, "prefill vs causal sdpa")
+
+
+ALL_PINS = [pin_page_figures, pin_round_bf16, pin_rope, pin_latent_rows, pin_query,
+            pin_decode_vs_library_attention, pin_decode_textbook_reduction, pin_decode_score_split,
+            pin_decode_special_cases, pin_naive_equals_absorbed, pin_decode_batch_driver,
+            pin_out_proj, pin_prefill]

@@ -1,0 +1,49 @@
+"""Plant plausible mistakes in a copy of the oracle's C source and check that the pins
+catch every one of them (CPU only).  The real oracle is never modified."""
+import os
+
+import pytest
+
+import oracle
+from oracle import build as obuild
+import pins
+
+MUTANTS = {
+    "rope_sign": ("out[2 * i] = x0 * c - x1 * s;", "out[2 * i] = x0 * c + x1 * s;"),
+    "rope_frequency": ("-2.0 * (double)i / (double)d", "-1.0 * (double)i / (double)d"),
+    "rope_pairing": ("double x0 = x[2 * i], x1 = x[2 * i + 1];",
+                     "double x0 = x[i], x1 = x[i + d / 2];"),
+    "drop_positional_term": ("s[t] = scale * (content + positional);", "s[t] = scale * (content);"),
+    "drop_scale": ("s[t] = scale * (content + positional);", "s[t] = (content + positional);"),
+    "no_softmax_normalisation": ("for (int t = 0; t < T; ++t) s[t] /= l;", ""),
+    "v_from_w_uk": ("acc += W_UV_h[(size_t)j * d_c + i] * c[i];", "acc += W_UK_h[(size_t)j * d_c + i] * c[i];"),
+    "absorbed_w_uk_transposed": ("for (int j = 0; j < qk_nope; ++j) acc += W_UK_h[(size_t)j * d_c + i] * q_nope[j];",
+                                 "for (int j = 0; j < qk_nope; ++j) acc += W_UK_h[(size_t)(i % qk_nope) * d_c + j] * q_nope[j];"),
+    "absorbed_o_lat_unweighted": ("o_lat[i] += s[t] * c[i];", "o_lat[i] += c[i] / T;"),
+    "query_layout": ("((size_t)hd * qh + j) * d_model", "((size_t)j * H + hd) * d_model"),
+    "query_no_rope": ("oracle_rope(d_hR, q + qk_nope, (double)pos[i], theta,", "oracle_rope(d_hR, q + qk_nope, 0.0, theta,"),
+    "latent_rope_position": ("oracle_rope(d_hR, kr, (double)pos[i], theta, row + d_c);",
+                             "oracle_rope(d_hR, kr, (double)(pos[i] + 1), theta, row + d_c);"),
+    "bf16_truncates": ("double r = rint(ldexp(m, 8));", "double r = floor(ldexp(m, 8));"),
+    "causal_excludes_self": ("oracle_attend_naive(t + 1, d_c", "oracle_attend_naive(t, d_c"),
+    "mla_row_without_rope": ("return (d_c + d_hR) * layers;", "return d_c * layers;"),
+    "out_proj_transposed": ("acc += W_O[(size_t)j * Hv + k] * o[(size_t)i * Hv + k];",
+                            "acc += W_O[(size_t)(k % d_model) * Hv + j % Hv] * o[(size_t)i * Hv + k];"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(obuild.SRC).read()
+    assert old in src, f"mutation site for {name} not found"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.load(obuild.build(str(path), str(tmp_path / "libmutant.so")))
+    failed = []
+    for pin in pins.ALL_PINS:
+        try:
+            pin(lib)
+        except AssertionError:
+            failed.append(pin.__name__)
+    assert failed, f"no pin detects the mutant {name}"
