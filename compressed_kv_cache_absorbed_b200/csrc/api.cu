@@ -1,0 +1,458 @@
+// The C ABI (include/mla.h): argument validation, workspace carving, kernel dispatch.
+#include <math.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "decode_tc.cuh"
+#include "mla.h"
+
+using mla::DevErr;
+using bf16 = __nv_bfloat16;
+
+// ------------------------------------------------------------------ error plumbing
+
+static __device__ int g_err_code;
+static __device__ long long g_err_detail;
+static char g_cuda_msg[256] = "no CUDA error";
+
+static mla_status cuda_fail(cudaError_t e, const char* where) {
+    snprintf(g_cuda_msg, sizeof g_cuda_msg, "%s: %s", where, cudaGetErrorString(e));
+    return MLA_ERR_CUDA;
+}
+#define MLA_CUDA(call)                                    \
+    do {                                                  \
+        cudaError_t e_ = (call);                          \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+    } while (0)
+
+static mla_status dev_err(DevErr* out) {
+    static std::mutex mu;
+    static DevErr cache[64];
+    static bool have[64];
+    int dev = 0;
+    MLA_CUDA(cudaGetDevice(&dev));
+    std::lock_guard<std::mutex> g(mu);
+    if (dev < 64 && have[dev]) {
+        *out = cache[dev];
+        return MLA_OK;
+    }
+    DevErr e;
+    MLA_CUDA(cudaGetSymbolAddress((void**)&e.code, g_err_code));
+    MLA_CUDA(cudaGetSymbolAddress((void**)&e.detail, g_err_detail));
+    if (dev < 64) {
+        cache[dev] = e;
+        have[dev] = true;
+    }
+    *out = e;
+    return MLA_OK;
+}
+
+// ---------------------------------------------------------------------- handle
+
+struct mla_weights_s {
+    mla_dims dims;
+    int device;
+    void* W_UK;    // [H, qk_nope, d_c]   copy, storage type
+    void* W_UKT;   // [H, d_c, qk_nope]   per-head transpose (K-major for the q absorption)
+    void* W_UV;    // [H, v_head, d_c]    copy
+    const void* W_Q;
+    const void* W_O;
+};
+
+// ------------------------------------------------------------------- validation
+
+static size_t esize(const mla_dims* d) { return d->dtype == MLA_BF16 ? 2 : 4; }
+static float scale_of(const mla_dims* d) {
+    return d->softmax_scale > 0.f ? d->softmax_scale : 1.0f / sqrtf((float)(d->qk_nope + d->d_hR));
+}
+static float theta_of(const mla_dims* d) { return d->rope_theta > 0.f ? d->rope_theta : 10000.f; }
+
+static bool dims_ok(const mla_dims* d) {
+    if (!d) return false;
+    if (d->H <= 0 || d->d_c <= 0 || d->d_hR <= 0 || d->qk_nope <= 0 || d->v_head <= 0) return false;
+    if (d->d_model < 0) return false;
+    if (d->dtype != MLA_F32 && d->dtype != MLA_BF16) return false;
+    return true;
+}
+// Shapes the kernels implement: rotary pairs must not straddle the content/rotary border.
+static mla_status dims_supported(const mla_dims* d) {
+    if (!dims_ok(d)) return MLA_ERR_INVALID_ARG;
+    if ((d->d_hR & 1) || (d->d_c & 1) || (d->qk_nope & 1)) return MLA_ERR_UNSUPPORTED;
+    if (d->d_c > 512 || d->v_head > 128 || d->qk_nope + d->d_hR > 256) return MLA_ERR_UNSUPPORTED;
+    return MLA_OK;
+}
+
+static int num_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+    return n;
+}
+
+// KV splits of the CUDA-core decode: about two waves of blocks.
+static int simt_splits(int B, int H) {
+    const int groups = (H + 7) / 8;
+    int ns = (2 * num_sms() + B * groups - 1) / (B * groups > 0 ? B * groups : 1);
+    return ns < 1 ? 1 : (ns > 32 ? 32 : ns);
+}
+
+// Bump allocator over the caller's workspace (256-byte aligned pieces).
+struct Carve {
+    char* base;
+    size_t used = 0;
+    explicit Carve(void* b) : base((char*)b) {}
+    void* take(size_t bytes) {
+        void* p = base ? base + used : nullptr;
+        used += (bytes + 255) & ~(size_t)255;
+        return p;
+    }
+};
+
+// ---------------------------------------------------------------- host helpers
+
+extern "C" const char* mla_status_string(mla_status s) {
+    switch (s) {
+        case MLA_OK: return "MLA_OK";
+        case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG: invalid pointer, size or dimension";
+        case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED: shape not implemented";
+        case MLA_ERR_WORKSPACE: return "MLA_ERR_WORKSPACE: workspace missing or too small";
+        case MLA_ERR_CUDA: return "MLA_ERR_CUDA: CUDA runtime call failed";
+        case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT: device-side wait gave up";
+        case MLA_ERR_OUT_OF_RANGE: return "MLA_ERR_OUT_OF_RANGE: slot or offset outside the cache";
+        case MLA_ERR_NO_MEMORY: return "MLA_ERR_NO_MEMORY: device allocation failed";
+    }
+    return "unknown mla_status";
+}
+
+extern "C" const char* mla_last_cuda_error(void) { return g_cuda_msg; }
+
+extern "C" int64_t mla_cache_row_elems(const mla_dims* d) {
+    if (!dims_ok(d)) return -1;
+    return (int64_t)d->d_c + d->d_hR;
+}
+
+extern "C" int64_t mla_cache_bytes_per_token(const mla_dims* d, int32_t layers) {
+    if (!dims_ok(d) || layers < 0) return -1;
+    return ((int64_t)d->d_c + d->d_hR) * layers * (int64_t)esize(d);
+}
+
+static bool tc_decode_ok(const mla_dims* d) {
+    return mla::tc::kEnabled && d->dtype == MLA_BF16 && d->H == mla::tc::kH &&
+           d->d_c == mla::tc::kDc && d->d_hR == mla::tc::kDr && d->qk_nope == 128 &&
+           d->v_head == 128;
+}
+
+extern "C" int32_t mla_decode_path(const mla_dims* d) {
+    if (dims_supported(d) != MLA_OK) return -1;
+    return tc_decode_ok(d) ? 1 : 0;
+}
+
+// ---------------------------------------------------------------------- weights
+
+extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, const void* W_UV,
+                                         const void* W_Q, const void* W_O, mla_weights* out,
+                                         mla_stream_t stream) {
+    if (!out) return MLA_ERR_INVALID_ARG;
+    *out = nullptr;
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!W_UK || !W_UV) return MLA_ERR_INVALID_ARG;
+    if ((W_Q || W_O) && d->d_model <= 0) return MLA_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t es = esize(d);
+    const size_t nk = (size_t)d->H * d->qk_nope * d->d_c, nv = (size_t)d->H * d->v_head * d->d_c;
+    int device = 0;
+    MLA_CUDA(cudaGetDevice(&device));
+    mla_weights w = new mla_weights_s();
+    w->dims = *d;
+    w->device = device;
+    w->W_Q = W_Q;
+    w->W_O = W_O;
+    if (cudaMalloc(&w->W_UK, nk * es) != cudaSuccess || cudaMalloc(&w->W_UKT, nk * es) != cudaSuccess ||
+        cudaMalloc(&w->W_UV, nv * es) != cudaSuccess) {
+        cudaFree(w->W_UK);
+        cudaFree(w->W_UKT);
+        cudaFree(w->W_UV);
+        delete w;
+        cudaGetLastError();
+        return MLA_ERR_NO_MEMORY;
+    }
+    cudaError_t e = cudaMemcpyAsync(w->W_UK, W_UK, nk * es, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(w->W_UV, W_UV, nv * es, cudaMemcpyDeviceToDevice, s);
+    if (e == cudaSuccess)
+        e = d->dtype == MLA_BF16
+                ? mla::launch_transpose_heads((const bf16*)W_UK, (bf16*)w->W_UKT, d->H, d->qk_nope, d->d_c, s)
+                : mla::launch_transpose_heads((const float*)W_UK, (float*)w->W_UKT, d->H, d->qk_nope, d->d_c, s);
+    if (e != cudaSuccess) {
+        cudaFree(w->W_UK);
+        cudaFree(w->W_UKT);
+        cudaFree(w->W_UV);
+        delete w;
+        return cuda_fail(e, "mla_absorb_weights");
+    }
+    *out = w;
+    return MLA_OK;
+}
+
+extern "C" mla_status mla_weights_destroy(mla_weights w) {
+    if (!w) return MLA_OK;
+    cudaDeviceSynchronize();
+    cudaFree(w->W_UK);
+    cudaFree(w->W_UKT);
+    cudaFree(w->W_UV);
+    delete w;
+    return MLA_OK;
+}
+
+// ------------------------------------------------------------------------ append
+
+template <typename T>
+static cudaError_t append_impl(const mla_dims* d, const void* h, const void* W_DKV, const void* W_KR,
+                               const int32_t* pos, int pos_mod, const int64_t* slot, int n,
+                               void* cache, long long capacity, DevErr err, cudaStream_t s) {
+    const int row = d->d_c + d->d_hR;
+    return mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)W_DKV, d->d_c,
+                                    (const T*)W_KR, row, row, d->d_c, d->d_hR, pos, pos_mod,
+                                    theta_of(d), slot, capacity, (T*)cache, row, err, s);
+}
+
+extern "C" mla_status mla_append_cache(const mla_dims* d, const void* h, const void* W_DKV,
+                                       const void* W_KR, const int32_t* pos, const int64_t* slot,
+                                       int32_t n, void* cache, int64_t capacity,
+                                       mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (n < 0 || capacity < 0 || d->d_model <= 0) return MLA_ERR_INVALID_ARG;
+    if (n == 0) return MLA_OK;
+    if (!h || !W_DKV || !W_KR || !pos || !slot || !cache) return MLA_ERR_INVALID_ARG;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = d->dtype == MLA_BF16
+                        ? append_impl<bf16>(d, h, W_DKV, W_KR, pos, 1, slot, n, cache, capacity, err, s)
+                        : append_impl<float>(d, h, W_DKV, W_KR, pos, 1, slot, n, cache, capacity, err, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_append_cache");
+}
+
+// ------------------------------------------------------------------------ decode
+
+struct DecodeWs {
+    void* q_buf;     // [B, H, qk_nope + d_hR] query projected from h (storage type)
+    float* q_lat;    // [B, H, d_c] fp32 (CUDA-core path)
+    float* part_o;   // [nsplit, B, H, d_c]
+    float* part_ml;  // [nsplit, B, H, 2]
+    float* o_lat;    // [B, H, d_c]
+    void* o_buf;     // [B, H, v_head] (storage type) when W_O follows
+    mla::tc::DecodeWs tc;  // tcgen05 path
+    size_t bytes;
+};
+
+static DecodeWs carve_decode(const mla_dims* d, int B, void* base, bool tc_path) {
+    Carve c(base);
+    DecodeWs w{};
+    const size_t es = esize(d), BH = (size_t)B * d->H;
+    w.q_buf = c.take(BH * (d->qk_nope + d->d_hR) * es);
+    w.o_buf = c.take(BH * d->v_head * es);
+    if (tc_path) {
+        w.tc = mla::tc::carve_decode_ws(c.base ? c.base + c.used : nullptr, B, num_sms());
+        c.used += mla::tc::decode_ws_bytes(B, num_sms());
+    } else {
+        const int ns = simt_splits(B, d->H);
+        w.q_lat = (float*)c.take(BH * d->d_c * 4);
+        w.part_o = (float*)c.take((size_t)ns * BH * d->d_c * 4);
+        w.part_ml = (float*)c.take((size_t)ns * BH * 2 * 4);
+        w.o_lat = (float*)c.take(BH * d->d_c * 4);
+    }
+    w.bytes = c.used;
+    return w;
+}
+
+extern "C" size_t mla_decode_workspace_size(const mla_dims* d, int32_t B) {
+    if (dims_supported(d) != MLA_OK || B < 0) return 0;
+    return carve_decode(d, B, nullptr, tc_decode_ok(d)).bytes;
+}
+
+template <typename T>
+static cudaError_t decode_simt(const mla_dims* d, mla_weights w, const T* qn, long long sQn_b,
+                               long long sQn_h, const T* qr, long long sQr_b, long long sQr_h,
+                               const T* cache, const int32_t* offsets, int B, T* o_dst,
+                               const DecodeWs& ws, DevErr err, cudaStream_t s) {
+    const int H = d->H, dc = d->d_c, qk = d->qk_nope, vh = d->v_head;
+    const int ns = simt_splits(B, H);
+    cudaError_t e;
+    // q_lat[b,h] = W_UK[h]^T q_nope[b,h]
+    e = mla::launch_gemm_nt<T, T, float>(H, B, dc, qk, qn, sQn_h, sQn_b, 1, (const T*)w->W_UKT,
+                                         (long long)dc * qk, qk, 1, ws.q_lat, dc, (long long)H * dc, 1, s);
+    if (e != cudaSuccess) return e;
+    e = mla::launch_decode_split_simt<T>(ws.q_lat, qr, sQr_b, sQr_h, cache, offsets, B, H, dc,
+                                         d->d_hR, scale_of(d), ns, ws.part_o, ws.part_ml, err, s);
+    if (e != cudaSuccess) return e;
+    e = mla::launch_combine(ws.part_o, ws.part_ml, ns, B, H, dc, ws.o_lat, s);
+    if (e != cudaSuccess) return e;
+    // o[b,h] = W_UV[h] o_lat[b,h]
+    return mla::launch_gemm_nt<float, T, T>(H, B, vh, dc, ws.o_lat, dc, (long long)H * dc, 1,
+                                            (const T*)w->W_UV, (long long)vh * dc, dc, 1, o_dst, vh,
+                                            (long long)H * vh, 1, s);
+}
+
+template <typename T>
+static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_nope,
+                               const void* q_rope, const void* h, const int32_t* q_pos,
+                               const void* cache, const int32_t* offsets, int B, void* out,
+                               const DecodeWs& ws, bool tc_path, DevErr err, cudaStream_t s) {
+    const int H = d->H, qk = d->qk_nope, dR = d->d_hR, vh = d->v_head;
+    const T* qn = (const T*)q_nope;
+    const T* qr = (const T*)q_rope;
+    long long sQn_b = (long long)H * qk, sQn_h = qk, sQr_b = (long long)H * dR, sQr_h = dR;
+    cudaError_t e;
+    if (!q_nope) {
+        // q = W_Q h with RoPE on each head's rotary part [L1 "Multi-head attention estandar"]
+        const int qh = qk + dR;
+        e = mla::launch_proj_rope<T>((const T*)h, B, d->d_model, (const T*)w->W_Q, H * qh, nullptr,
+                                     H * qh, qh, qk, dR, q_pos, 1, theta_of(d), nullptr, 0,
+                                     (T*)ws.q_buf, (long long)H * qh, err, s);
+        if (e != cudaSuccess) return e;
+        qn = (const T*)ws.q_buf;
+        qr = (const T*)ws.q_buf + qk;
+        sQn_b = sQr_b = (long long)H * qh;
+        sQn_h = sQr_h = qh;
+    }
+    T* o_dst = w->W_O ? (T*)ws.o_buf : (T*)out;
+    if (tc_path) {
+        e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
+                                        (const bf16*)w->W_UKT, (const bf16*)w->W_UV,
+                                        (const bf16*)cache, offsets, B, scale_of(d), (bf16*)o_dst,
+                                        ws.tc, num_sms(), err.code, err.detail, s);
+    } else {
+        e = decode_simt<T>(d, w, qn, sQn_b, sQn_h, qr, sQr_b, sQr_h, (const T*)cache, offsets, B,
+                           o_dst, ws, err, s);
+    }
+    if (e != cudaSuccess) return e;
+    if (w->W_O) {
+        // out[b] = W_O concat_h o[b,h] [L2 "Informacion tecnica": output projection]
+        const int Hv = H * vh;
+        e = mla::launch_gemm_nt<T, T, T>(1, B, d->d_model, Hv, (const T*)ws.o_buf, 0, Hv, 1,
+                                         (const T*)w->W_O, 0, Hv, 1, (T*)out, 0, d->d_model, 1, s);
+    }
+    return e;
+}
+
+extern "C" mla_status mla_decode_absorbed(const mla_dims* d, mla_weights w, const void* q_nope,
+                                          const void* q_rope, const void* h, const int32_t* q_pos,
+                                          const void* cache, const int32_t* offsets, int32_t B,
+                                          void* out, void* workspace, size_t ws_bytes,
+                                          mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if (B == 0) return MLA_OK;
+    if (!cache || !offsets || !out) return MLA_ERR_INVALID_ARG;
+    const bool from_q = q_nope || q_rope;
+    if (from_q && (!q_nope || !q_rope)) return MLA_ERR_INVALID_ARG;
+    if (!from_q && (!h || !q_pos || !w->W_Q)) return MLA_ERR_INVALID_ARG;
+    const bool tc_path = tc_decode_ok(d);
+    DecodeWs ws = carve_decode(d, B, workspace, tc_path);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = d->dtype == MLA_BF16
+                        ? decode_impl<bf16>(d, w, q_nope, q_rope, h, q_pos, cache, offsets, B, out, ws, tc_path, err, s)
+                        : decode_impl<float>(d, w, q_nope, q_rope, h, q_pos, cache, offsets, B, out, ws, false, err, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed");
+}
+
+// ----------------------------------------------------------------------- prefill
+
+struct PrefillWs {
+    void* q_buf;   // [B*S, H, qk_nope + d_hR]
+    void* k_buf;   // [B*S, H, qk_nope]
+    void* v_buf;   // [B*S, H, v_head]
+    size_t bytes;
+};
+
+static PrefillWs carve_prefill(const mla_dims* d, int B, int S, void* base) {
+    Carve c(base);
+    PrefillWs w{};
+    const size_t es = esize(d), nH = (size_t)B * S * d->H;
+    w.q_buf = c.take(nH * (d->qk_nope + d->d_hR) * es);
+    w.k_buf = c.take(nH * d->qk_nope * es);
+    w.v_buf = c.take(nH * d->v_head * es);
+    w.bytes = c.used;
+    return w;
+}
+
+extern "C" size_t mla_prefill_workspace_size(const mla_dims* d, int32_t B, int32_t S) {
+    if (dims_supported(d) != MLA_OK || B < 0 || S < 0) return 0;
+    return carve_prefill(d, B, S, nullptr).bytes;
+}
+
+template <typename T>
+static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h, const void* W_DKV,
+                                const void* W_KR, void* cache, void* out, int B, int S,
+                                const PrefillWs& ws, DevErr err, cudaStream_t s) {
+    const int H = d->H, dc = d->d_c, dR = d->d_hR, qk = d->qk_nope, vh = d->v_head;
+    const int n = B * S, row = dc + dR, qh = qk + dR;
+    cudaError_t e;
+    // 1. cache rows for every token, position t = i % S, row b*S + t
+    e = append_impl<T>(d, h, W_DKV, W_KR, nullptr, S, nullptr, n, cache, n, err, s);
+    if (e != cudaSuccess) return e;
+    // 2. queries with RoPE at t
+    e = mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)w->W_Q, H * qh, nullptr, H * qh,
+                                 qh, qk, dR, nullptr, S, theta_of(d), nullptr, 0, (T*)ws.q_buf,
+                                 (long long)H * qh, err, s);
+    if (e != cudaSuccess) return e;
+    // 3. K_nope = W_UK[h] c and V = W_UV[h] c, materialised [L1 "La compresion de MLA"]
+    e = mla::launch_gemm_nt<T, T, T>(H, n, qk, dc, (const T*)cache, 0, row, 1, (const T*)w->W_UK,
+                                     (long long)qk * dc, dc, 1, (T*)ws.k_buf, qk, (long long)H * qk, 1, s);
+    if (e != cudaSuccess) return e;
+    e = mla::launch_gemm_nt<T, T, T>(H, n, vh, dc, (const T*)cache, 0, row, 1, (const T*)w->W_UV,
+                                     (long long)vh * dc, dc, 1, (T*)ws.v_buf, vh, (long long)H * vh, 1, s);
+    if (e != cudaSuccess) return e;
+    // 4. causal attention
+    return mla::launch_prefill_attn_simt<T>((const T*)ws.q_buf, (const T*)ws.k_buf, (const T*)cache,
+                                            (const T*)ws.v_buf, B, S, H, qk, dR, dc, vh, scale_of(d),
+                                            (T*)out, s);
+}
+
+extern "C" mla_status mla_prefill_causal(const mla_dims* d, mla_weights w, const void* h,
+                                         const void* W_DKV, const void* W_KR, void* cache, void* out,
+                                         int32_t B, int32_t S, void* workspace, size_t ws_bytes,
+                                         mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0 || S < 0 || d->d_model <= 0) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if ((long long)B * S > (1LL << 31) - 1) return MLA_ERR_UNSUPPORTED;
+    if (B == 0 || S == 0) return MLA_OK;
+    if (!h || !W_DKV || !W_KR || !cache || !out || !w->W_Q) return MLA_ERR_INVALID_ARG;
+    PrefillWs ws = carve_prefill(d, B, S, workspace);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e = d->dtype == MLA_BF16
+                        ? prefill_impl<bf16>(d, w, h, W_DKV, W_KR, cache, out, B, S, ws, err, s)
+                        : prefill_impl<float>(d, w, h, W_DKV, W_KR, cache, out, B, S, ws, err, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_prefill_causal");
+}
+
+// ------------------------------------------------------------------- diagnostics
+
+extern "C" mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail) {
+    MLA_CUDA(cudaStreamSynchronize((cudaStream_t)stream));
+    int code = 0;
+    long long det = 0;
+    MLA_CUDA(cudaMemcpyFromSymbol(&code, g_err_code, sizeof code));
+    MLA_CUDA(cudaMemcpyFromSymbol(&det, g_err_detail, sizeof det));
+    const int zero = 0;
+    const long long zero64 = 0;
+    MLA_CUDA(cudaMemcpyToSymbol(g_err_code, &zero, sizeof zero));
+    MLA_CUDA(cudaMemcpyToSymbol(g_err_detail, &zero64, sizeof zero64));
+    if (detail) *detail = det;
+    return (mla_status)code;
+}

@@ -1,0 +1,186 @@
+/*
+ * mla.h -- C ABI of the B200 (sm_100a) Multi-head Latent Attention library.
+ *
+ * The library computes decode-time attention over the compressed MLA cache (each token
+ * stores only its latent c_kv and a small decoupled RoPE key), with W_UK absorbed into
+ * the query and W_UV applied after the softmax-weighted sum, so per-head K and V are never
+ * formed; plus the cache append and a materialised-K/V causal prefill.
+ *
+ * Sources, by page title and section:
+ *   [L1] "02 - Multi-Latent Attention (MLA)" (lynx-cortex, phase 36): "La compresion de
+ *        MLA" (c_t = W_DKV h_t; k_t = W_UK c_t; v_t = W_UV c_t), "Truco de codificacion
+ *        posicional" (decoupled rotary key k^rope, width d_hR, cached as is), "Coste de
+ *        computo" (re-associating the matmuls so attention runs on c directly).
+ *   [L2] "Multi-head latent attention" (aiunderstanding.org), "Informacion tecnica":
+ *        the up-projections are absorbed into the query and output projections.
+ *   [L4] "Multi-head Latent Attention (MLA) si arhitectura DeepSeekMoE" (dexblog.ro),
+ *        opening section: (d_c + d_hR) cached elements per token per layer.
+ *   [L5] "DeepSeek MLA" (llm-engineer cards): score = content + positional; decode reads
+ *        the whole cache every step.
+ *
+ * Conventions shared by every call
+ *   - Every tensor pointer is a DEVICE pointer unless stated; tensors are dense row-major.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - Argument errors are detected on the host and returned before anything is launched;
+ *     outputs are then untouched.  Errors found on the device (a slot outside the cache,
+ *     decreasing offsets) skip the offending work and latch a device error word that
+ *     mla_get_device_error() reads.  No call traps, aborts or throws.
+ *   - The caller owns every tensor (cache, inputs, outputs, workspace).  The only
+ *     library-owned object is an mla_weights handle (device memory it allocates once).
+ *   - Storage type: all float tensors of one call share `dims->dtype` (fp32 or bf16);
+ *     accumulation is always fp32.  Index arrays are int32 (offsets, positions) or
+ *     int64 (slots); row arithmetic is done in 64 bits.
+ *   - Cache layout [L4]: row r of the cache is (d_c + d_hR) elements, the latent c in
+ *     columns [0, d_c) and the rotated key k_rope in [d_c, d_c + d_hR).
+ *   - RoPE: pairs (2i, 2i+1) rotated by pos * theta^(-2i/d_hR); one rotary key per token,
+ *     shared by all heads.
+ */
+#ifndef MLA_B200_H
+#define MLA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* mla_stream_t; /* cudaStream_t */
+
+typedef enum {
+    MLA_OK = 0,
+    MLA_ERR_INVALID_ARG = 1,    /* a pointer, size or dimension is invalid */
+    MLA_ERR_UNSUPPORTED = 2,    /* valid but not implemented (e.g. odd d_hR) */
+    MLA_ERR_WORKSPACE = 3,      /* workspace missing or smaller than *_workspace_size() */
+    MLA_ERR_CUDA = 4,           /* a CUDA runtime call failed (message: mla_last_cuda_error) */
+    MLA_ERR_DEVICE_TIMEOUT = 5, /* a device-side wait gave up (reported by mla_get_device_error) */
+    MLA_ERR_OUT_OF_RANGE = 6,   /* device-side: a slot/offset outside the cache */
+    MLA_ERR_NO_MEMORY = 7       /* allocation of an mla_weights handle failed */
+} mla_status;
+
+typedef enum { MLA_F32 = 0, MLA_BF16 = 1 } mla_dtype;
+
+/* Layer dimensions.  softmax_scale <= 0 selects 1/sqrt(qk_nope + d_hR); rope_theta <= 0
+ * selects 10000.  d_model may be 0 for calls that never touch the hidden size. */
+typedef struct {
+    int32_t H;          /* attention heads */
+    int32_t d_model;    /* hidden size */
+    int32_t d_c;        /* latent width (kv_lora_rank) */
+    int32_t d_hR;       /* decoupled RoPE key width (even) */
+    int32_t qk_nope;    /* per-head content query/key width */
+    int32_t v_head;     /* per-head value width */
+    float softmax_scale;
+    float rope_theta;
+    int32_t dtype;      /* mla_dtype */
+} mla_dims;
+
+typedef struct mla_weights_s* mla_weights;
+
+/* ---------------------------------------------------------------- host-only helpers */
+
+/* Human-readable name of a status code (static string). */
+const char* mla_status_string(mla_status s);
+
+/* Message of the last failed CUDA runtime call in this process (static buffer). */
+const char* mla_last_cuda_error(void);
+
+/* Elements one token adds to the cache per layer: d_c + d_hR [L4].  -1 if dims invalid. */
+int64_t mla_cache_row_elems(const mla_dims* dims);
+
+/* Bytes one token adds to the cache over `layers` layers: (d_c + d_hR) * layers * elem. */
+int64_t mla_cache_bytes_per_token(const mla_dims* dims, int32_t layers);
+
+/* Which decode kernel family a call with these dims would use: 1 = tcgen05/TMEM
+ * split-KV kernel (bf16, H = 128, d_c = 512, d_hR = 64), 0 = CUDA-core kernel,
+ * -1 = invalid dims.  Host-only; used by tests to assert the fast path is taken. */
+int32_t mla_decode_path(const mla_dims* dims);
+
+/* ------------------------------------------------------------------------- weights */
+
+/* Pack the per-head up-projections for the kernels [L1 "Coste de computo"; L2].
+ *   W_UK [H, qk_nope, d_c]   (k_nope = W_UK[h] c)          -- copied and re-laid out
+ *   W_UV [H, v_head, d_c]    (v = W_UV[h] c)               -- copied
+ *   W_Q  [H*(qk_nope+d_hR), d_model] or NULL               -- borrowed (not copied)
+ *   W_O  [d_model, H*v_head] or NULL                       -- borrowed (not copied)
+ * W_Q rows are head-major, the qk_nope content rows of a head before its d_hR rotary rows.
+ * Borrowed tensors must stay valid until mla_weights_destroy.  The handle owns device
+ * memory allocated here (the only allocation the library makes).  Stream-ordered: the
+ * packing kernels run on `stream`. */
+mla_status mla_absorb_weights(const mla_dims* dims, const void* W_UK, const void* W_UV,
+                              const void* W_Q, const void* W_O, mla_weights* out,
+                              mla_stream_t stream);
+
+/* Free a handle (synchronises the device first).  NULL is accepted. */
+mla_status mla_weights_destroy(mla_weights w);
+
+/* ------------------------------------------------------------------- cache append */
+
+/* KV down-projection, RoPE and cache write [L1 "La compresion de MLA", "Truco de
+ * codificacion posicional"; L4]: for token i < n,
+ *     c = W_DKV h_i,   k_r = RoPE(W_KR h_i, pos[i]),   cache[slot[i]] = [c | k_r]
+ * (fp32 accumulation, one rounding to the storage type).
+ *   h [n, d_model]; W_DKV [d_c, d_model]; W_KR [d_hR, d_model]; pos int32 [n];
+ *   slot int64 [n]; cache [capacity, d_c + d_hR].
+ * Only the rows slot[i] are written.  A slot outside [0, capacity) is skipped and latches
+ * MLA_ERR_OUT_OF_RANGE in the device error word.  Duplicate slots race (last writer wins).
+ * n = 0 is a no-op. */
+mla_status mla_append_cache(const mla_dims* dims, const void* h, const void* W_DKV,
+                            const void* W_KR, const int32_t* pos, const int64_t* slot,
+                            int32_t n, void* cache, int64_t capacity, mla_stream_t stream);
+
+/* --------------------------------------------------------------- absorbed decode */
+
+/* Bytes of workspace mla_decode_absorbed needs for B sequences on the current device. */
+size_t mla_decode_workspace_size(const mla_dims* dims, int32_t B);
+
+/* Absorbed decode attention over the latent cache, one query token per sequence
+ * [L1 "Coste de computo"; L2; L5]:
+ *     q_lat[b,h]  = W_UK[h]^T q_nope[b,h]                         (d_c)
+ *     s[b,h,t]    = scale * (q_lat[b,h] . c_t + q_rope[b,h] . k_r,t)
+ *     o_lat[b,h]  = sum_t softmax_t(s[b,h,:]) c_t                 (d_c, fp32)
+ *     o[b,h]      = W_UV[h] o_lat[b,h]                            (v_head)
+ *     out[b]      = W_O concat_h o[b,h]        (only when the handle holds W_O)
+ * Sequence b attends over cache rows [offsets[b], offsets[b+1]) (int32 [B+1], ragged).
+ * An empty sequence gives o = 0.  The query comes either from (q_nope [B,H,qk_nope],
+ * q_rope [B,H,d_hR], q_rope already rotated) or, when both are NULL, from the hidden
+ * state h [B, d_model] through the handle's W_Q with RoPE at q_pos int32 [B].
+ * out is [B, H, v_head], or [B, d_model] when the handle holds W_O.
+ * workspace: device, >= mla_decode_workspace_size(dims, B) bytes, 256-byte aligned;
+ * its contents on entry do not matter.  Decreasing offsets latch MLA_ERR_OUT_OF_RANGE. */
+mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* q_nope,
+                               const void* q_rope, const void* h, const int32_t* q_pos,
+                               const void* cache, const int32_t* offsets, int32_t B,
+                               void* out, void* workspace, size_t ws_bytes,
+                               mla_stream_t stream);
+
+/* ---------------------------------------------------------------- causal prefill */
+
+/* Bytes of workspace mla_prefill_causal needs for B sequences of S tokens. */
+size_t mla_prefill_workspace_size(const mla_dims* dims, int32_t B, int32_t S);
+
+/* Causal prefill with K and V materialised from the latent [L1 "La compresion de MLA"]:
+ * appends every token (as mla_append_cache, position t, cache row b*S + t), then per head
+ *     K_t = [W_UK[h] c_t | k_r,t],   V_t = W_UV[h] c_t,
+ *     q = W_Q h_t (rotary part rotated at t),
+ *     out[b,t,h] = sum_{tau <= t} softmax(scale * q . K_tau) V_tau.
+ *   h [B, S, d_model]; W_DKV [d_c, d_model]; W_KR [d_hR, d_model];
+ *   cache [B*S, d_c + d_hR] (written); out [B, S, H, v_head].
+ * The handle must hold W_Q.  workspace >= mla_prefill_workspace_size(dims, B, S). */
+mla_status mla_prefill_causal(const mla_dims* dims, mla_weights w, const void* h,
+                              const void* W_DKV, const void* W_KR, void* cache, void* out,
+                              int32_t B, int32_t S, void* workspace, size_t ws_bytes,
+                              mla_stream_t stream);
+
+/* ------------------------------------------------------------------- diagnostics */
+
+/* Synchronise `stream`, then read and clear the device error word of the current device.
+ * Returns MLA_OK if no device-side error was latched since the last call, else the
+ * latched code (MLA_ERR_OUT_OF_RANGE, MLA_ERR_DEVICE_TIMEOUT); *detail (nullable)
+ * receives a kernel-specific detail value. */
+mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_B200_H */

@@ -1,0 +1,330 @@
+"""Parity of the CUDA path (through the C ABI) with the float64 oracle, on the same seeded
+inputs: reduced sizes that span several tiles and a ragged tail, the full workload sizes on
+sampled outputs, and the edge cases (empty, single-row and ragged sequences, B = 0, n = 0,
+slots outside the cache, decreasing offsets)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads
+from helpers import CACHE_ABS_RMS, CACHE_EXACT_FRAC, assert_close, bf16_bits, bf16_ulp_diff, np64, rms, to_dev
+
+pytestmark = pytest.mark.gpu
+
+mla = pytest.importorskip("compressed_kv_cache_absorbed_b200")
+
+DEV = "cuda"
+
+
+def dims_of(w: workloads.Workload):
+    return mla.make_dims(w.H, w.d_model, w.d_c, w.d_hR, w.qk_nope, w.v_head, w.dtype)
+
+
+def storage_round(rows64: np.ndarray, dtype: str) -> np.ndarray:
+    """The oracle's cache rows rounded once to the storage type (nearest-even)."""
+    if dtype == "f32":
+        return rows64.astype(np.float32).astype(np.float64)
+    return oracle.bf16_value(oracle.round_bf16(rows64))
+
+
+def sample_units(B, H, n, seed, must_b=(), must_h=(0,)):
+    r = np.random.default_rng(seed)
+    units = {(int(b), int(h)) for b in must_b for h in must_h}
+    units |= {(0, 0), (0, H - 1)}
+    while len(units) < n:
+        units.add((int(r.integers(B)), int(r.integers(H))))
+    return sorted(units)
+
+
+# ----------------------------------------------------------------------- append
+
+def check_rows(gpu_rows: torch.Tensor, want64: np.ndarray, dtype: str, what: str):
+    if dtype == "f32":
+        assert_close(gpu_rows, want64, "f32", what)
+        return 1.0
+    got = bf16_bits(gpu_rows)
+    ref = oracle.round_bf16(want64)
+    ulp = bf16_ulp_diff(got, ref)
+    # beyond one ulp only where the value is so small that fp32 accumulation error over the
+    # d_model-long dot product (~sqrt(K) * 2^-24 * RMS) exceeds a bf16 ulp of it
+    err = np.abs(oracle.bf16_value(got) - want64)
+    far = (ulp > 1) & (err > CACHE_ABS_RMS * rms(want64))
+    assert not far.any(), f"{what}: {int(far.sum())} elements off by more than 1 ulp and the fp32 bound"
+    frac = float((ulp == 0).mean())
+    assert frac >= CACHE_EXACT_FRAC, f"{what}: only {frac:.4f} of values bit-exact"
+    return frac
+
+
+@pytest.mark.parametrize("name,n", [("tiny_fp32_layer", 37), ("v3_layer_b128_ctx8192", 128),
+                                    ("v2_prefill_b4_s4096", 200)])
+def test_append_rows_and_layout(name, n):
+    w = workloads.WORKLOADS[name]
+    d = workloads.make_weights(w)
+    dims = dims_of(w)
+    tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    h = torch.from_numpy(np.random.default_rng(1).standard_normal((n, w.d_model))).to(tdt)
+    cap = 3 * n + 5
+    rng = np.random.default_rng(2)
+    slots = np.sort(rng.choice(cap, n, replace=False))[::-1].copy()   # scattered, descending
+    pos = rng.integers(0, 40000, n).astype(np.int32)
+    pos[0] = 0
+    sentinel = torch.full((cap, w.row), -7.25, dtype=tdt)
+    cache = sentinel.clone().to(DEV)
+    mla.mla_append_cache(dims, h.to(DEV), d["W_DKV"].to(DEV), d["W_KR"].to(DEV),
+                         torch.from_numpy(pos).to(DEV), torch.from_numpy(slots).to(DEV), cache)
+    assert mla.mla_get_device_error() == (0, 0)
+    cache = cache.cpu()
+    want = oracle.latent_rows(h, d["W_DKV"], d["W_KR"], pos, w.rope_theta)
+    frac = check_rows(cache[torch.from_numpy(slots)], want, w.dtype, f"{name} rows")
+    assert frac >= CACHE_EXACT_FRAC
+    untouched = np.setdiff1d(np.arange(cap), slots)
+    assert torch.equal(cache[torch.from_numpy(untouched)], sentinel[torch.from_numpy(untouched)])
+
+
+def test_append_slot_out_of_range_latches_and_skips():
+    w = workloads.WORKLOADS["tiny_fp32_layer"]
+    d = workloads.make_weights(w)
+    dims = dims_of(w)
+    h = torch.randn(4, w.d_model)
+    cache = torch.zeros(4, w.row, device=DEV)
+    slot = torch.tensor([0, 9, 2, -1], dtype=torch.int64, device=DEV)
+    pos = torch.zeros(4, dtype=torch.int32, device=DEV)
+    mla.mla_append_cache(dims, h.to(DEV), d["W_DKV"].to(DEV), d["W_KR"].to(DEV), pos, slot, cache)
+    st, _ = mla.mla_get_device_error()
+    assert st == mla.MLA_ERR_OUT_OF_RANGE
+    c = cache.cpu()
+    assert torch.all(c[1] == 0) and torch.all(c[3] == 0) and not torch.all(c[0] == 0)
+    assert mla.mla_get_device_error() == (0, 0)      # reading clears the word
+
+
+def test_append_zero_tokens_is_a_noop():
+    w = workloads.WORKLOADS["tiny_fp32_layer"]
+    cache = torch.zeros(2, w.row, device=DEV)
+    e = torch.empty(0, device=DEV)
+    mla.mla_append_cache(dims_of(w), e.view(0, w.d_model), e, e, e.int(), e.long(), cache)
+    assert torch.all(cache == 0)
+
+
+# ----------------------------------------------------------------------- decode
+
+def run_decode_attn(w, inp, B=None):
+    dims = dims_of(w)
+    g = to_dev({k: inp[k] for k in ("cache", "offsets", "q_nope", "q_rope", "W_UK", "W_UV")})
+    B = g["offsets"].numel() - 1
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    out = torch.empty(B, w.H, w.v_head, dtype=g["cache"].dtype, device=DEV)
+    ws = mla.workspace(mla.mla_decode_workspace_size(dims, B))
+    mla.mla_decode_absorbed(dims, weights, g["cache"], g["offsets"], out, ws, q_nope=g["q_nope"],
+                            q_rope=g["q_rope"])
+    assert mla.mla_get_device_error() == (0, 0)
+    return out.cpu()
+
+
+def oracle_decode_units(w, inp, units, absorbed=True, seqs=None):
+    """Oracle o for (b, h) units, reading only the rows of the sequences involved."""
+    offs = inp["offsets"].numpy().astype(np.int64)
+    bs = sorted({b for b, _ in units})
+    rows, new_offs, remap = [], [0], {}
+    for i, b in enumerate(bs):
+        remap[b] = i
+        rows.append(np64(inp["cache"][offs[b]:offs[b + 1]]))
+        new_offs.append(new_offs[-1] + offs[b + 1] - offs[b])
+    rows = np.concatenate(rows) if rows else np.zeros((0, w.row))
+    qn = np64(inp["q_nope"][bs])
+    qr = np64(inp["q_rope"][bs])
+    o, _ = oracle.decode(qn, qr, rows, new_offs, inp["W_UK"], inp["W_UV"], w.scale,
+                         units=[(remap[b], h) for b, h in units], absorbed=absorbed)
+    return o
+
+
+def reduced_attn_inputs(lengths, seed=11):
+    w = workloads.WORKLOADS["v3_decode_b32_ctx4096"]
+    w = workloads.shrink(w, B=len(lengths), seed=seed)
+    d = workloads.make_weights(w)
+    r = np.random.default_rng(seed)
+    offs = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int32)
+    tot = int(offs[-1])
+    d["offsets"] = torch.from_numpy(offs)
+    d["cache"] = (torch.from_numpy(r.standard_normal((tot, w.row))) * 0.5).to(torch.bfloat16)
+    d["q_nope"] = torch.from_numpy(r.standard_normal((w.B, w.H, w.qk_nope))).to(torch.bfloat16)
+    d["q_rope"] = torch.from_numpy(r.standard_normal((w.B, w.H, w.d_hR))).to(torch.bfloat16)
+    return w, d
+
+
+@pytest.mark.parametrize("lengths", [[300, 1, 77, 513, 64], [0, 1000, 2], [4096, 129]])
+def test_decode_attn_reduced_all_units(lengths):
+    w, inp = reduced_attn_inputs(lengths)
+    out = run_decode_attn(w, inp)
+    units = [(b, h) for b in range(w.B) for h in range(w.H)]
+    want = oracle_decode_units(w, inp, units).reshape(w.B, w.H, w.v_head)
+    for b, L in enumerate(lengths):
+        if L == 0:
+            assert torch.all(out[b] == 0), "an empty sequence decodes to zeros"
+    nz = [b for b, L in enumerate(lengths) if L > 0]
+    assert_close(out[nz], want[nz], "bf16", f"decode {lengths}")
+    # a few units through the naive (materialised K/V) form as well
+    few = [(nz[0], 0), (nz[-1], w.H - 1), (nz[0], 77)]
+    naive = oracle_decode_units(w, inp, few, absorbed=False)
+    assert_close(torch.stack([out[b, h] for b, h in few]), naive, "bf16", "decode vs naive")
+
+
+@pytest.mark.parametrize("name", ["v3_decode_b32_ctx4096", "v3_ragged_b64"])
+def test_decode_attn_full_size_sampled(name):
+    w = workloads.WORKLOADS[name]
+    inp = workloads.make_inputs(w)
+    out = run_decode_attn(w, inp)
+    L = workloads.lengths(w)
+    must = (int(np.argmax(L)), int(np.argmin(L)), w.B - 1)
+    units = sample_units(w.B, w.H, 64, 5, must_b=must, must_h=(0, w.H - 1))
+    want = oracle_decode_units(w, inp, units)
+    got = torch.stack([out[b, h] for b, h in units])
+    assert_close(got, want, "bf16", name)
+    naive = oracle_decode_units(w, inp, units[:2], absorbed=False)
+    assert_close(got[:2], naive, "bf16", name + " naive")
+
+
+# --------------------------------------------------------------- decode layer
+
+def run_decode_layer(w, inp):
+    dims = dims_of(w)
+    g = to_dev(inp)
+    B = w.B
+    offs = inp["offsets"].numpy().astype(np.int64)
+    L = workloads.lengths(w)
+    if w.history == "hidden":
+        cache = torch.zeros(int(offs[-1]), w.row, dtype=g["h_new"].dtype, device=DEV)
+        pos = np.tile(np.arange(w.ctx), B).astype(np.int32)
+        slot = (offs[:-1, None] + np.arange(w.ctx)[None]).reshape(-1)
+        mla.mla_append_cache(dims, g["h_hist"].reshape(-1, w.d_model), g["W_DKV"], g["W_KR"],
+                             torch.from_numpy(pos).to(DEV), torch.from_numpy(slot).to(DEV), cache)
+    else:
+        cache = g["cache"]
+    # the token being decoded: appended at position L, then attends over L + 1 rows
+    q_pos = torch.from_numpy(L.astype(np.int32)).to(DEV)
+    slot = torch.from_numpy(offs[:-1] + L).to(DEV)
+    mla.mla_append_cache(dims, g["h_new"], g["W_DKV"], g["W_KR"], q_pos, slot, cache)
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"])
+    out = torch.empty(B, w.d_model, dtype=g["h_new"].dtype, device=DEV)
+    ws = mla.workspace(mla.mla_decode_workspace_size(dims, B))
+    mla.mla_decode_absorbed(dims, weights, cache, g["offsets"], out, ws, h=g["h_new"], q_pos=q_pos)
+    assert mla.mla_get_device_error() == (0, 0)
+    return out.cpu(), cache
+
+
+def oracle_decode_layer(w, inp, bs, absorbed):
+    """Oracle out[b] for the sequences bs, computing every row it needs itself."""
+    L = workloads.lengths(w)
+    offs = inp["offsets"].numpy().astype(np.int64)
+    rows_all, o_offs = [], [0]
+    for b in bs:
+        if w.history == "hidden":
+            hist = oracle.latent_rows(inp["h_hist"][b], inp["W_DKV"], inp["W_KR"], np.arange(w.ctx), w.rope_theta)
+            hist = storage_round(hist, w.dtype)
+        else:
+            hist = np64(inp["cache"][offs[b]:offs[b] + L[b]])
+        new = oracle.latent_rows(inp["h_new"][b:b + 1], inp["W_DKV"], inp["W_KR"], [L[b]], w.rope_theta)
+        rows_all.append(np.concatenate([hist, storage_round(new, w.dtype)]))
+        o_offs.append(o_offs[-1] + L[b] + 1)
+    qn, qr = oracle.query(inp["h_new"][bs], inp["W_Q"], L[bs], w.H, w.qk_nope, w.d_hR, w.rope_theta)
+    o, _ = oracle.decode(qn, qr, np.concatenate(rows_all), o_offs, inp["W_UK"], inp["W_UV"], w.scale,
+                         absorbed=absorbed)
+    return oracle.out_proj(o, inp["W_O"]), np.concatenate([r[-1:] for r in rows_all])
+
+
+def test_decode_layer_tiny_fp32_end_to_end():
+    w = workloads.WORKLOADS["tiny_fp32_layer"]
+    inp = workloads.make_inputs(w)
+    out, cache = run_decode_layer(w, inp)
+    want, _ = oracle_decode_layer(w, inp, list(range(w.B)), absorbed=False)
+    assert_close(out, want, "f32", "tiny fp32 layer (naive oracle)")
+    # every cache row the GPU wrote (history and new token) against the oracle's rows
+    offs = inp["offsets"].numpy()
+    for b in range(w.B):
+        rows = oracle.latent_rows(np.concatenate([np64(inp["h_hist"][b]), np64(inp["h_new"][b:b + 1])]),
+                                  inp["W_DKV"], inp["W_KR"], np.arange(w.ctx + 1), w.rope_theta)
+        assert_close(cache[offs[b]:offs[b + 1]].cpu(), rows, "f32", f"tiny cache b={b}")
+
+
+def test_decode_layer_v3_full_size_sampled():
+    w = workloads.WORKLOADS["v3_layer_b128_ctx8192"]
+    inp = workloads.make_inputs(w)
+    out, cache = run_decode_layer(w, inp)
+    bs = [0, 57, w.B - 1]
+    want, new_rows = oracle_decode_layer(w, inp, bs, absorbed=True)
+    assert_close(out[bs], want, "bf16", "v3 layer out")
+    offs = inp["offsets"].numpy().astype(np.int64)
+    L = workloads.lengths(w)
+    # the appended rows of all 128 sequences, and the untouched history around them
+    allnew = oracle.latent_rows(inp["h_new"], inp["W_DKV"], inp["W_KR"], L, w.rope_theta)
+    got = cache[torch.from_numpy(offs[:-1] + L).to(DEV)].cpu()
+    frac = check_rows(got, allnew, "bf16", "v3 appended rows")
+    assert frac >= CACHE_EXACT_FRAC
+    assert torch.equal(cache[:8192].cpu(), inp["cache"][:8192])
+
+
+# ---------------------------------------------------------------------- prefill
+
+def run_prefill(w, inp):
+    dims = dims_of(w)
+    g = to_dev(inp)
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"])
+    cache = torch.zeros(w.B * w.ctx, w.row, dtype=g["h"].dtype, device=DEV)
+    out = torch.empty(w.B, w.ctx, w.H, w.v_head, dtype=g["h"].dtype, device=DEV)
+    ws = mla.workspace(mla.mla_prefill_workspace_size(dims, w.B, w.ctx))
+    mla.mla_prefill_causal(dims, weights, g["h"], g["W_DKV"], g["W_KR"], cache, out, ws)
+    assert mla.mla_get_device_error() == (0, 0)
+    return out.cpu(), cache.cpu()
+
+
+def oracle_prefill(w, inp, b, t_list, heads, absorbed=True):
+    S_needed = max(t_list) + 1
+    rows = oracle.latent_rows(inp["h"][b, :S_needed], inp["W_DKV"], inp["W_KR"], np.arange(S_needed),
+                              w.rope_theta)
+    rows_s = storage_round(rows, w.dtype)
+    qn, qr = oracle.query(inp["h"][b, t_list], inp["W_Q"], t_list, w.H, w.qk_nope, w.d_hR, w.rope_theta)
+    # scatter the sampled queries into position-indexed arrays for the per-head routine
+    QN = np.zeros((S_needed, w.qk_nope))
+    QR = np.zeros((S_needed, w.d_hR))
+    res = {}
+    for h in heads:
+        QN[t_list] = qn[:, h]
+        QR[t_list] = qr[:, h]
+        res[h] = oracle.prefill_head(QN, QR, rows_s, inp["W_UK"][h], inp["W_UV"][h], w.scale, t_list,
+                                     absorbed)
+    return res, rows
+
+
+@pytest.mark.parametrize("B,S", [(2, 200)])
+def test_prefill_reduced(B, S):
+    w = workloads.shrink(workloads.WORKLOADS["v2_prefill_b4_s4096"], B=B, ctx=S, seed=77)
+    inp = workloads.make_inputs(w)
+    out, cache = run_prefill(w, inp)
+    t_list = [0, 1, 63, 64, 65, 127, 128, 150, 191, 192, 199]
+    heads = [0, 5, 127]
+    for b in range(B):
+        res, rows = oracle_prefill(w, inp, b, t_list, heads)
+        for h in heads:
+            assert_close(out[b, t_list, h], res[h], "bf16", f"prefill b={b} h={h}")
+        assert len(rows) == S
+        check_rows(cache[b * S:(b + 1) * S], rows, "bf16", "prefill cache")
+    res, _ = oracle_prefill(w, inp, 1, [0, 150], [3], absorbed=False)
+    assert_close(out[1, [0, 150], 3], res[3], "bf16", "prefill naive")
+
+
+def test_prefill_full_size_sampled():
+    w = workloads.WORKLOADS["v2_prefill_b4_s4096"]
+    inp = workloads.make_inputs(w)
+    out, cache = run_prefill(w, inp)
+    b = 2
+    t_list = [0, 1, 2, 127, 128, 2047, 4094, 4095]
+    heads = [0, 64, 127]
+    res, rows = oracle_prefill(w, inp, b, t_list, heads)
+    for h in heads:
+        assert_close(out[b, t_list, h], res[h], "bf16", f"prefill full h={h}")
+    frac = check_rows(cache[b * w.ctx:(b + 1) * w.ctx], rows, "bf16", "prefill cache rows")
+    assert frac >= CACHE_EXACT_FRAC
