@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the absorbed MLA decode on B200.
+
+One step = one mla_decode_absorbed call (query absorption, split-KV attention over the
+latent cache, log-sum-exp merge, W_UV) for the DeepSeek-V3-shaped workload: 32 sequences
+of 4096 cached tokens, 128 heads, d_c = 512, d_hR = 64, bf16 storage, fp32 accumulation.
+Inputs are resident in HBM when the timed region starts; L2 is flushed (256 MiB write)
+between steps, outside the per-step events.
+
+Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle instead.
+Multi-GPU (torchrun): every rank decodes its own batch (weak scaling, no collective on the
+data path); times are the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "MLA decode tokens/s + latent-cache GB/s, % roofline (H=128,d_c=512,ctx 4k)"
+WORKLOAD = "v3_decode_b32_ctx4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+FLUSH_BYTES = 256 << 20
+
+
+# ------------------------------------------------------------------ arithmetic
+
+def alg_step(w: workloads.Workload) -> dict:
+    """Bytes the method must move and flops it must do for one decode step."""
+    L = workloads.lengths(w)
+    tokens = int(L.sum())
+    e = 2  # bf16
+    cache = tokens * w.row * e
+    weights = 2 * w.H * w.qk_nope * w.d_c * e            # W_UK and W_UV (qk_nope = v_head)
+    q = w.B * w.H * (w.qk_nope + w.d_hR) * e
+    out = w.B * w.H * w.v_head * e
+    flops_attn = tokens * w.H * (2 * w.row + 2 * w.d_c)    # scores over 576 + P.c over 512
+    flops_proj = 2 * w.B * w.H * w.qk_nope * w.d_c * 2     # absorption and W_UV
+    return {"bytes": cache + weights + q + out, "cache_bytes": cache, "flops": flops_attn + flops_proj,
+            "attn_flops": flops_attn, "tokens": tokens}
+
+
+def alg_kernel_bytes(name: str, w: workloads.Workload) -> int:
+    """Algorithmic bytes of one launch of the kernel that dominates the step: the cache rows
+    it attends over (1152 B per token) plus the queries it reads."""
+    L = workloads.lengths(w)
+    cache = int(L.sum()) * w.row * 2
+    if name.startswith("tc_"):
+        return cache + w.B * w.H * w.row * 2
+    return cache + w.B * w.H * (w.d_c * 4 + w.d_hR * 2)
+
+
+def peaks() -> tuple:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"]))}, "measured"
+    return dict(FALLBACK_PEAKS, bf16_tflops_sustained=1400.0), "fallback"
+
+
+def traffic_for(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source has not
+    changed since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    src = os.path.join(ROOT, d["source"])
+    if not os.path.exists(src) or hashlib.sha256(open(src, "rb").read()).hexdigest() != d["sha256"]:
+        return None
+    return d["bytes_per_launch"]
+
+
+# ---------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.samples = []
+        self.proc = None
+        self.gpu = gpu_index
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                self.samples.append((time.time(), parts))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float) -> dict:
+        inside = [p for t, p in self.samples if t0 <= t <= t1]
+        used = inside or [p for _, p in self.samples]
+        if not used:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for p in used for n, v in zip(names, p[5:9]) if v.lower() == "active"})
+        sm = [float(p[1]) for p in used if p[1].replace(".", "").isdigit()]
+        mx = [float(p[2]) for p in used if p[2].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(used), "samples_in_timed_region": len(inside)}
+
+
+# ----------------------------------------------------------------- distributed
+
+def dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float) -> float:
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def rank_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
+    """Each rank decodes its own batch of the same shape (its own seed)."""
+    return w if rank == 0 else workloads.shrink(w, seed=w.seed + 1000 * rank)
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def time_oracle_units(w: workloads.Workload, inp: dict, budget_s: float, min_units: int = 2,
+                      max_units: int = 10 ** 6, tokens: int = 0):
+    """Run the float64 naive oracle on (b, h) units until `budget_s` is spent.  With
+    tokens > 0 each unit attends over only its first `tokens` rows; the naive cost is
+    linear in the rows attended, so the step time scales by (rows of the unit / tokens)."""
+    import oracle
+    offs = inp["offsets"].numpy().astype(np.int64)
+    rng = np.random.default_rng(0)
+    lib = oracle.load()
+    done, t_spent, scale_sum = 0, 0.0, 0.0
+    while done < max_units and (done < min_units or t_spent < budget_s):
+        b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
+        T = int(offs[b + 1] - offs[b])
+        n = T if tokens <= 0 else max(1, min(T, tokens))
+        rows = inp["cache"][offs[b]:offs[b] + n]
+        t = time.perf_counter()
+        oracle.attend(inp["q_nope"][b, h], inp["q_rope"][b, h], rows, inp["W_UK"][h], inp["W_UV"][h],
+                      w.scale, absorbed=False, lib=lib)
+        dt = time.perf_counter() - t
+        t_spent += dt
+        scale_sum += dt * T / n
+        done += 1
+    per_unit = scale_sum / done
+    step_s = per_unit * w.B * w.H
+    what = "all rows" if tokens <= 0 else f"its first {tokens} rows (time scaled to all rows)"
+    return {"value": w.B / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"{done} (sequence, head) units of {w.name}, each over {what}, through the naive "
+                      f"float64 oracle (K and V materialised), {t_spent:.1f} s single-threaded; the full "
+                      f"step ({w.B * w.H} units) extrapolated as {per_unit * 1e3:.1f} ms x {w.B * w.H}",
+            "step_s_extrapolated": step_s}
+
+
+# ------------------------------------------------------------------------ arms
+
+def run_reference(args, w):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    inp = workloads.make_inputs(w)
+    import oracle
+    oracle.load()
+    # calibrate: rows per second of the naive oracle, then size each step's sample so the
+    # whole run (warm-up + timed) takes about args.reference_seconds
+    cal = time_oracle_units(w, inp, 0.0, min_units=2, max_units=2, tokens=256)
+    rows_per_s = 256.0 / (cal["step_s_extrapolated"] / (w.B * w.H) * 256.0 / w.ctx) if w.ctx else 1e5
+    per_step = args.reference_seconds / (args.steps + args.warmup)
+    tokens = int(max(16, min(w.ctx or 10 ** 9, per_step * rows_per_s)))
+    time_oracle_units(w, inp, 0.0, min_units=args.warmup, max_units=args.warmup, tokens=tokens)
+    r = time_oracle_units(w, inp, 0.0, min_units=args.steps, max_units=args.steps, tokens=tokens)
+    line = {"impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": r["step_s_extrapolated"] * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, world),
+            "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, world):
+    return {"workload": w.name, "B_per_gpu": w.B, "ctx": w.ctx, "H": w.H, "d_c": w.d_c, "d_hR": w.d_hR,
+            "qk_nope": w.qk_nope, "v_head": w.v_head, "global_batch": w.B * world,
+            "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write, outside the step events)"}
+
+
+def run_ours(args, w0):
+    world, rank, local = dist_init()
+    import compressed_kv_cache_absorbed_b200 as mla
+    w = rank_workload(w0, rank)
+    inp = workloads.make_inputs(w)
+    dev = torch.device("cuda", local)
+    g = {k: v.to(dev) for k, v in inp.items()}
+    dims = mla.make_dims(w.H, w.d_model, w.d_c, w.d_hR, w.qk_nope, w.v_head, w.dtype)
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    out = torch.empty(w.B, w.H, w.v_head, dtype=torch.bfloat16, device=dev)
+    ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        mla.mla_decode_absorbed(dims, weights, g["cache"], g["offsets"], out, ws, q_nope=g["q_nope"],
+                                q_rope=g["q_rope"])
+
+    # warm-up
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    st, det = mla.mla_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} ({det}) during warm-up")
+
+    clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    time.sleep(0.3 if clocks else 0)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # timed region: per-step events (the L2 flush sits between them); per-kernel events on
+    # the library's launches give the dominant kernel's live launch duration
+    mla.mla_profile_report(reset=True)
+    mla.mla_profile_enable(True)
+    barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    barrier()
+    mla.mla_profile_enable(False)
+    prof = mla.mla_profile_report(reset=True)
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    ms = max_over_ranks(float(np.mean(step_ms)))
+
+    # the same timed loop without per-kernel events (their cost on the step)
+    ev2 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.zero_()
+        ev2[i][0].record(stream)
+        step()
+        ev2[i][1].record(stream)
+    torch.cuda.synchronize()
+    ms_noprof = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev2])))
+    clk = clocks.summary(t0, t1) if clocks else None
+    if clocks:
+        clocks.stop()
+
+    # end to end through the same call with host buffers: H2D of the queries, D2H of o
+    qn_h = inp["q_nope"].pin_memory()
+    qr_h = inp["q_rope"].pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps + args.warmup):
+        flush.zero_()
+        j = i - args.warmup
+        if j >= 0:
+            ev3[j][0].record(stream)
+        g["q_nope"].copy_(qn_h, non_blocking=True)
+        g["q_rope"].copy_(qr_h, non_blocking=True)
+        step()
+        out_h.copy_(out, non_blocking=True)
+        if j >= 0:
+            ev3[j][1].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev3])))
+    st, det = mla.mla_get_device_error()
+    if st != 0:
+        raise RuntimeError(f"device error {st} ({det})")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = time_oracle_units(w, inp, args.cpu_seconds)
+        cpu.pop("step_s_extrapolated", None)
+
+    if rank == 0:
+        a = alg_step(w)
+        pk, pk_kind = peaks()
+        dom = max(prof, key=lambda k: prof[k][1])
+        n_launch, dom_ms = prof[dom]
+        launch_s = dom_ms / n_launch * 1e-3
+        kbytes = alg_kernel_bytes(dom, w)
+        achieved = kbytes / launch_s / 1e9
+        launches_per_step = sum(v[0] for v in prof.values()) / args.steps
+        step_s = ms * 1e-3
+        roof_s = max(a["bytes"] / (pk["hbm_gbs"] * 1e9), a["flops"] / (pk["bf16_tflops"] * 1e12))
+        line = {
+            "metric": METRIC, "value": world * w.B / step_s, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, world),
+            "latent_cache_GBps": a["cache_bytes"] / step_s / 1e9,
+            "step_roofline": {"alg_bytes": a["bytes"], "alg_flops": a["flops"], "roofline_us": roof_s * 1e6,
+                              "frac": roof_s / step_s, "tflops": a["flops"] / step_s / 1e12,
+                              "peaks": f"{pk_kind}: hbm {pk['hbm_gbs']} GB/s, bf16 {pk['bf16_tflops']} TFLOP/s"},
+            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom),
+                         "alg_bytes_per_launch": kbytes, "launch_us": launch_s * 1e6,
+                         "peak_source": f"{pk_kind} hbm_gbs"},
+            "kernels": {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in prof.items()},
+            "ms_per_step_without_kernel_events": ms_noprof,
+            "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": int(inp["q_nope"].numel() * 2 + inp["q_rope"].numel() * 2),
+                    "d2h_bytes_per_step": int(out.numel() * 2), "ms_per_step": e2e_ms,
+                    "note": "latent cache and weights stay resident in HBM (decode state)"},
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": clk,
+            "cpu_baseline": cpu,
+            "decode_path": "tcgen05" if mla.mla_decode_path(dims) == 1 else "cuda-core",
+        }
+        print(json.dumps(line), flush=True)
+    weights.close()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=WORKLOAD, choices=sorted(workloads.WORKLOADS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--reference-seconds", type=float, default=90.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    w = workloads.WORKLOADS[args.workload]
+    if w.kind != "decode_attn":
+        ap.error("the benchmark step is the absorbed decode of a decode_attn workload")
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -52,6 +52,8 @@ SIGNATURES = {
     "mla_prefill_causal": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
                                 ctypes.c_size_t, _P]),
     "mla_get_device_error": (_S, [_P, ctypes.POINTER(ctypes.c_int64)]),
+    "mla_profile_enable": (None, [ctypes.c_int32]),
+    "mla_profile_report": (ctypes.c_int32, [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_int32]),
 }
 for _name, (_res, _args) in SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -178,6 +180,21 @@ def mla_get_device_error(stream=None):
     d = ctypes.c_int64(0)
     st = _lib.mla_get_device_error(_stream(stream), ctypes.byref(d))
     return int(st), int(d.value)
+
+
+def mla_profile_enable(on: bool = True) -> None:
+    _lib.mla_profile_enable(1 if on else 0)
+
+
+def mla_profile_report(reset: bool = True) -> dict:
+    """{kernel_name: (launches, total_ms)} of the library's own launches since the last reset."""
+    buf = ctypes.create_string_buffer(1 << 16)
+    _lib.mla_profile_report(buf, len(buf), 1 if reset else 0)
+    out = {}
+    for line in buf.value.decode().splitlines():
+        name, n, ms = line.split()
+        out[name] = (int(n), float(ms))
+    return out
 
 
 def lib():

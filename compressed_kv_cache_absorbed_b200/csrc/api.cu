@@ -214,6 +214,7 @@ static cudaError_t append_impl(const mla_dims* d, const void* h, const void* W_D
                                const int32_t* pos, int pos_mod, const int64_t* slot, int n,
                                void* cache, long long capacity, DevErr err, cudaStream_t s) {
     const int row = d->d_c + d->d_hR;
+    mla::ProfScope ps(s, "simt_append_proj_rope");
     return mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)W_DKV, d->d_c,
                                     (const T*)W_KR, row, row, d->d_c, d->d_hR, pos, pos_mod,
                                     theta_of(d), slot, capacity, (T*)cache, row, err, s);
@@ -284,15 +285,19 @@ static cudaError_t decode_simt(const mla_dims* d, mla_weights w, const T* qn, lo
     const int ns = simt_splits(B, H);
     cudaError_t e;
     // q_lat[b,h] = W_UK[h]^T q_nope[b,h]
+    { mla::ProfScope ps(s, "simt_q_absorb");
     e = mla::launch_gemm_nt<T, T, float>(H, B, dc, qk, qn, sQn_h, sQn_b, 1, (const T*)w->W_UKT,
-                                         (long long)dc * qk, qk, 1, ws.q_lat, dc, (long long)H * dc, 1, s);
+                                         (long long)dc * qk, qk, 1, ws.q_lat, dc, (long long)H * dc, 1, s); }
     if (e != cudaSuccess) return e;
+    { mla::ProfScope ps(s, "simt_decode_split");
     e = mla::launch_decode_split_simt<T>(ws.q_lat, qr, sQr_b, sQr_h, cache, offsets, B, H, dc,
-                                         d->d_hR, scale_of(d), ns, ws.part_o, ws.part_ml, err, s);
+                                         d->d_hR, scale_of(d), ns, ws.part_o, ws.part_ml, err, s); }
     if (e != cudaSuccess) return e;
-    e = mla::launch_combine(ws.part_o, ws.part_ml, ns, B, H, dc, ws.o_lat, s);
+    { mla::ProfScope ps(s, "simt_combine");
+    e = mla::launch_combine(ws.part_o, ws.part_ml, ns, B, H, dc, ws.o_lat, s); }
     if (e != cudaSuccess) return e;
     // o[b,h] = W_UV[h] o_lat[b,h]
+    mla::ProfScope ps(s, "simt_w_uv");
     return mla::launch_gemm_nt<float, T, T>(H, B, vh, dc, ws.o_lat, dc, (long long)H * dc, 1,
                                             (const T*)w->W_UV, (long long)vh * dc, dc, 1, o_dst, vh,
                                             (long long)H * vh, 1, s);
@@ -311,6 +316,7 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (!q_nope) {
         // q = W_Q h with RoPE on each head's rotary part [L1 "Multi-head attention estandar"]
         const int qh = qk + dR;
+        mla::ProfScope ps(s, "simt_q_proj_rope");
         e = mla::launch_proj_rope<T>((const T*)h, B, d->d_model, (const T*)w->W_Q, H * qh, nullptr,
                                      H * qh, qh, qk, dR, q_pos, 1, theta_of(d), nullptr, 0,
                                      (T*)ws.q_buf, (long long)H * qh, err, s);
@@ -334,6 +340,7 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (w->W_O) {
         // out[b] = W_O concat_h o[b,h] [L2 "Informacion tecnica": output projection]
         const int Hv = H * vh;
+        mla::ProfScope ps(s, "simt_w_o");
         e = mla::launch_gemm_nt<T, T, T>(1, B, d->d_model, Hv, (const T*)ws.o_buf, 0, Hv, 1,
                                          (const T*)w->W_O, 0, Hv, 1, (T*)out, 0, d->d_model, 1, s);
     }
@@ -402,18 +409,22 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
     e = append_impl<T>(d, h, W_DKV, W_KR, nullptr, S, nullptr, n, cache, n, err, s);
     if (e != cudaSuccess) return e;
     // 2. queries with RoPE at t
+    { mla::ProfScope ps(s, "simt_q_proj_rope");
     e = mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)w->W_Q, H * qh, nullptr, H * qh,
                                  qh, qk, dR, nullptr, S, theta_of(d), nullptr, 0, (T*)ws.q_buf,
-                                 (long long)H * qh, err, s);
+                                 (long long)H * qh, err, s); }
     if (e != cudaSuccess) return e;
     // 3. K_nope = W_UK[h] c and V = W_UV[h] c, materialised [L1 "La compresion de MLA"]
+    { mla::ProfScope ps(s, "simt_k_materialise");
     e = mla::launch_gemm_nt<T, T, T>(H, n, qk, dc, (const T*)cache, 0, row, 1, (const T*)w->W_UK,
-                                     (long long)qk * dc, dc, 1, (T*)ws.k_buf, qk, (long long)H * qk, 1, s);
+                                     (long long)qk * dc, dc, 1, (T*)ws.k_buf, qk, (long long)H * qk, 1, s); }
     if (e != cudaSuccess) return e;
+    { mla::ProfScope ps(s, "simt_v_materialise");
     e = mla::launch_gemm_nt<T, T, T>(H, n, vh, dc, (const T*)cache, 0, row, 1, (const T*)w->W_UV,
-                                     (long long)vh * dc, dc, 1, (T*)ws.v_buf, vh, (long long)H * vh, 1, s);
+                                     (long long)vh * dc, dc, 1, (T*)ws.v_buf, vh, (long long)H * vh, 1, s); }
     if (e != cudaSuccess) return e;
     // 4. causal attention
+    mla::ProfScope ps(s, "simt_prefill_attn");
     return mla::launch_prefill_attn_simt<T>((const T*)ws.q_buf, (const T*)ws.k_buf, (const T*)cache,
                                             (const T*)ws.v_buf, B, S, H, qk, dR, dc, vh, scale_of(d),
                                             (T*)out, s);

@@ -37,6 +37,15 @@ constexpr int kErrTimeout = 5;
 
 // ---------------------------------------------------------------- launch helpers
 
+// per-kernel event timing (profile.cu); no-ops unless mla_profile_enable(1)
+void prof_begin(cudaStream_t s, const char* name);
+void prof_end(cudaStream_t s);
+struct ProfScope {
+    cudaStream_t s;
+    ProfScope(cudaStream_t st, const char* name) : s(st) { prof_begin(st, name); }
+    ~ProfScope() { prof_end(s); }
+};
+
 template <typename T> struct Dt;
 template <> struct Dt<float> { static constexpr int id = 0; };
 template <> struct Dt<__nv_bfloat16> { static constexpr int id = 1; };

@@ -179,6 +179,15 @@ mla_status mla_prefill_causal(const mla_dims* dims, mla_weights w, const void* h
  * receives a kernel-specific detail value. */
 mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail);
 
+/* Per-kernel device timing of this library's own launches (a diagnostic, off by default).
+ * While enabled, each launch is bracketed by two CUDA events recorded on its stream. */
+void mla_profile_enable(int32_t on);
+
+/* Writes one line "kernel_name launches total_ms" per kernel timed since the last reset
+ * into buf (nullable; truncated to cap), waiting for the recorded events.  Returns the
+ * number of kernels; reset != 0 clears the totals. */
+int32_t mla_profile_report(char* buf, size_t cap, int32_t reset);
+
 #ifdef __cplusplus
 }
 #endif
