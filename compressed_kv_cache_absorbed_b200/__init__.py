@@ -52,6 +52,7 @@ SIGNATURES = {
     "mla_prefill_causal": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
                                 ctypes.c_size_t, _P]),
     "mla_get_device_error": (_S, [_P, ctypes.POINTER(ctypes.c_int64)]),
+    "mla_decode_absorbed_noalloc": (_S, [_D, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
     "mla_profile_report": (ctypes.c_int32, [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_int32]),
 }
@@ -166,6 +167,16 @@ def mla_decode_absorbed(dims, weights: MLAWeights, cache, offsets, out, ws, q_no
                                     _ptr(h), _ptr(q_pos), _ptr(cache), _ptr(offsets), B, _ptr(out),
                                     _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "mla_decode_absorbed")
+
+
+def mla_decode_absorbed_noalloc(dims, weights: MLAWeights, cache, offsets, out, q_nope=None,
+                                q_rope=None, h=None, q_pos=None, stream=None) -> None:
+    """mla_decode_absorbed with the library's fixed device scratch instead of a workspace,
+    for callers that cannot allocate device memory."""
+    B = offsets.numel() - 1
+    _check(_lib.mla_decode_absorbed_noalloc(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
+                                            _ptr(h), _ptr(q_pos), _ptr(cache), _ptr(offsets), B, _ptr(out),
+                                            _stream(stream)), "mla_decode_absorbed_noalloc")
 
 
 def mla_prefill_causal(dims, weights: MLAWeights, h, W_DKV, W_KR, cache, out, ws, stream=None) -> None:

@@ -153,6 +153,31 @@ mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* 
                                void* out, void* workspace, size_t ws_bytes,
                                mla_stream_t stream);
 
+/* Size of the fixed device scratch used by mla_decode_absorbed_noalloc (64 MiB). */
+#define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
+
+/* mla_decode_absorbed without a workspace argument, for callers that cannot allocate
+ * device memory (an engine that gives all GPU memory to its own pool at start-up, code
+ * in a region where allocation is forbidden, a plugin host without an allocation hook).
+ * The source pages have no counterpart to this call; it exists for those callers.
+ * Arguments, layouts and results are those of mla_decode_absorbed.  The scratch comes
+ * from one fixed device array of MLA_NOALLOC_SCRATCH_BYTES inside the library, which
+ * every GPU that loads the library holds until the process exits; this call itself
+ * allocates nothing (no cudaMalloc, no cudaFree).
+ *   - A call whose scratch need (mla_decode_workspace_size(dims, B)) exceeds
+ *     MLA_NOALLOC_SCRATCH_BYTES returns MLA_ERR_WORKSPACE before launching anything
+ *     (compare the two to know in advance whether a batch fits).
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     with that device current; make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the previous call's contents (nothing
+ *     in it needs to start at zero).  Calls that overlap on the GPU (other streams,
+ *     other host threads, without ordering between them) race on it and give wrong
+ *     results; order them on one stream or with events. */
+mla_status mla_decode_absorbed_noalloc(const mla_dims* dims, mla_weights w, const void* q_nope,
+                                       const void* q_rope, const void* h, const int32_t* q_pos,
+                                       const void* cache, const int32_t* offsets, int32_t B,
+                                       void* out, mla_stream_t stream);
+
 /* ---------------------------------------------------------------- causal prefill */
 
 /* Bytes of workspace mla_prefill_causal needs for B sequences of S tokens. */
