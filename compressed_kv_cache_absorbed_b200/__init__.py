@@ -46,13 +46,14 @@ SIGNATURES = {
     "mla_weights_destroy": (_S, [_P]),
     "mla_append_cache": (_S, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64, _P]),
     "mla_decode_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32]),
-    "mla_decode_absorbed": (_S, [_D, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P,
+    "mla_decode_absorbed": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
                                  ctypes.c_size_t, _P]),
     "mla_prefill_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32]),
     "mla_prefill_causal": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int32, ctypes.c_int32, _P,
                                 ctypes.c_size_t, _P]),
     "mla_get_device_error": (_S, [_P, ctypes.POINTER(ctypes.c_int64)]),
-    "mla_decode_absorbed_noalloc": (_S, [_D, _P, _P, _P, _P, _P, _P, _P, ctypes.c_int32, _P, _P]),
+    "mla_decode_absorbed_noalloc": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P,
+                                         _P]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
     "mla_profile_report": (ctypes.c_int32, [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_int32]),
 }
@@ -164,8 +165,8 @@ def mla_decode_absorbed(dims, weights: MLAWeights, cache, offsets, out, ws, q_no
                         h=None, q_pos=None, stream=None) -> None:
     B = offsets.numel() - 1
     _check(_lib.mla_decode_absorbed(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
-                                    _ptr(h), _ptr(q_pos), _ptr(cache), _ptr(offsets), B, _ptr(out),
-                                    _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
+                                    _ptr(h), _ptr(q_pos), _ptr(cache), cache.shape[0], _ptr(offsets), B,
+                                    _ptr(out), _ptr(ws), ws.numel() if ws is not None else 0, _stream(stream)),
            "mla_decode_absorbed")
 
 
@@ -175,8 +176,8 @@ def mla_decode_absorbed_noalloc(dims, weights: MLAWeights, cache, offsets, out, 
     for callers that cannot allocate device memory."""
     B = offsets.numel() - 1
     _check(_lib.mla_decode_absorbed_noalloc(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
-                                            _ptr(h), _ptr(q_pos), _ptr(cache), _ptr(offsets), B, _ptr(out),
-                                            _stream(stream)), "mla_decode_absorbed_noalloc")
+                                            _ptr(h), _ptr(q_pos), _ptr(cache), cache.shape[0], _ptr(offsets), B,
+                                            _ptr(out), _stream(stream)), "mla_decode_absorbed_noalloc")
 
 
 def mla_prefill_causal(dims, weights: MLAWeights, h, W_DKV, W_KR, cache, out, ws, stream=None) -> None:

@@ -279,7 +279,7 @@ extern "C" size_t mla_decode_workspace_size(const mla_dims* d, int32_t B) {
 template <typename T>
 static cudaError_t decode_simt(const mla_dims* d, mla_weights w, const T* qn, long long sQn_b,
                                long long sQn_h, const T* qr, long long sQr_b, long long sQr_h,
-                               const T* cache, const int32_t* offsets, int B, T* o_dst,
+                               const T* cache, long long cache_rows, const int32_t* offsets, int B, T* o_dst,
                                const DecodeWs& ws, DevErr err, cudaStream_t s) {
     const int H = d->H, dc = d->d_c, qk = d->qk_nope, vh = d->v_head;
     const int ns = simt_splits(B, H);
@@ -290,7 +290,7 @@ static cudaError_t decode_simt(const mla_dims* d, mla_weights w, const T* qn, lo
                                          (long long)dc * qk, qk, 1, ws.q_lat, dc, (long long)H * dc, 1, s); }
     if (e != cudaSuccess) return e;
     { mla::ProfScope ps(s, "simt_decode_split");
-    e = mla::launch_decode_split_simt<T>(ws.q_lat, qr, sQr_b, sQr_h, cache, offsets, B, H, dc,
+    e = mla::launch_decode_split_simt<T>(ws.q_lat, qr, sQr_b, sQr_h, cache, cache_rows, offsets, B, H, dc,
                                          d->d_hR, scale_of(d), ns, ws.part_o, ws.part_ml, err, s); }
     if (e != cudaSuccess) return e;
     { mla::ProfScope ps(s, "simt_combine");
@@ -306,7 +306,7 @@ static cudaError_t decode_simt(const mla_dims* d, mla_weights w, const T* qn, lo
 template <typename T>
 static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_nope,
                                const void* q_rope, const void* h, const int32_t* q_pos,
-                               const void* cache, const int32_t* offsets, int B, void* out,
+                               const void* cache, long long cache_rows, const int32_t* offsets, int B, void* out,
                                const DecodeWs& ws, bool tc_path, DevErr err, cudaStream_t s) {
     const int H = d->H, qk = d->qk_nope, dR = d->d_hR, vh = d->v_head;
     const T* qn = (const T*)q_nope;
@@ -330,10 +330,10 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (tc_path) {
         e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
                                         (const bf16*)w->W_UKT, (const bf16*)w->W_UV,
-                                        (const bf16*)cache, offsets, B, scale_of(d), (bf16*)o_dst,
+                                        (const bf16*)cache, cache_rows, offsets, B, scale_of(d), (bf16*)o_dst,
                                         ws.tc, num_sms(), err.code, err.detail, s);
     } else {
-        e = decode_simt<T>(d, w, qn, sQn_b, sQn_h, qr, sQr_b, sQr_h, (const T*)cache, offsets, B,
+        e = decode_simt<T>(d, w, qn, sQn_b, sQn_h, qr, sQr_b, sQr_h, (const T*)cache, cache_rows, offsets, B,
                            o_dst, ws, err, s);
     }
     if (e != cudaSuccess) return e;
@@ -349,15 +349,15 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
 
 extern "C" mla_status mla_decode_absorbed(const mla_dims* d, mla_weights w, const void* q_nope,
                                           const void* q_rope, const void* h, const int32_t* q_pos,
-                                          const void* cache, const int32_t* offsets, int32_t B,
-                                          void* out, void* workspace, size_t ws_bytes,
+                                          const void* cache, int64_t cache_rows, const int32_t* offsets,
+                                          int32_t B, void* out, void* workspace, size_t ws_bytes,
                                           mla_stream_t stream) {
     mla_status st = dims_supported(d);
     if (st != MLA_OK) return st;
     if (!w || B < 0) return MLA_ERR_INVALID_ARG;
     if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
     if (B == 0) return MLA_OK;
-    if (!cache || !offsets || !out) return MLA_ERR_INVALID_ARG;
+    if (!cache || !offsets || !out || cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return MLA_ERR_INVALID_ARG;
     const bool from_q = q_nope || q_rope;
     if (from_q && (!q_nope || !q_rope)) return MLA_ERR_INVALID_ARG;
     if (!from_q && (!h || !q_pos || !w->W_Q)) return MLA_ERR_INVALID_ARG;
@@ -368,8 +368,8 @@ extern "C" mla_status mla_decode_absorbed(const mla_dims* d, mla_weights w, cons
     if ((st = dev_err(&err)) != MLA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e = d->dtype == MLA_BF16
-                        ? decode_impl<bf16>(d, w, q_nope, q_rope, h, q_pos, cache, offsets, B, out, ws, tc_path, err, s)
-                        : decode_impl<float>(d, w, q_nope, q_rope, h, q_pos, cache, offsets, B, out, ws, false, err, s);
+                        ? decode_impl<bf16>(d, w, q_nope, q_rope, h, q_pos, cache, cache_rows, offsets, B, out, ws, tc_path, err, s)
+                        : decode_impl<float>(d, w, q_nope, q_rope, h, q_pos, cache, cache_rows, offsets, B, out, ws, false, err, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed");
 }
 

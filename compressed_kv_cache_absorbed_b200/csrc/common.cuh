@@ -73,9 +73,10 @@ cudaError_t launch_gemm_nt(int Z, int M, int N, int K, const TA* A, long long sA
 // split-KV decode on CUDA cores; q_lat fp32 [B,H,d_c]; q_rope rows at q_rope + b*sQb + h*sQh
 template <typename T>
 cudaError_t launch_decode_split_simt(const float* q_lat, const T* q_rope, long long sQb,
-                                     long long sQh, const T* cache, const int32_t* offsets,
-                                     int B, int H, int d_c, int d_hR, float scale, int nsplit,
-                                     float* part_o, float* part_ml, DevErr err, cudaStream_t s);
+                                     long long sQh, const T* cache, long long cache_rows,
+                                     const int32_t* offsets, int B, int H, int d_c, int d_hR,
+                                     float scale, int nsplit, float* part_o, float* part_ml,
+                                     DevErr err, cudaStream_t s);
 
 // merge nsplit partials (O unnormalised, m, l) -> o_lat fp32 [B,H,d_c]
 cudaError_t launch_combine(const float* part_o, const float* part_ml, int nsplit, int B, int H,

@@ -1,16 +1,610 @@
+// Absorbed MLA decode on the tcgen05 tensor cores, for H = 128 heads, d_c = 512, d_hR = 64.
+//
+// Problem (per sequence b, head h, cached token t; scale = 1/sqrt(192)):
+//     s[h,t] = scale * ([q_lat | q_rope][h] . [c_t | k_r,t])      (576-long dot product)
+//     o_lat[h] = sum_t softmax_t(s[h,:]) c_t                       (512 wide)
+// With 128 heads sharing every cache row this is a dense contraction: per 64-token tile,
+// S = Q[128 x 576] . tile^T and O += P[128 x 64] . tile[:, :512].
+//
+// Why two CTAs per tile.  O for 128 heads x 512 latent columns in fp32 is 512 TMEM columns,
+// all of an SM's TMEM.  So a cluster of two CTAs (two SMs) splits the latent columns: CTA r
+// owns c columns [256r, 256r + 256) and rotary columns [32r, 32r + 32), loads only those
+// (no duplicate HBM/L2 traffic, no multicast), and accumulates O_r = 128 x 256.  The
+// softmax needs the full 576-long scores, so each CTA computes a partial S_r over its 288
+// columns and the pair exchanges halves through distributed shared memory: CTA r finishes
+// the softmax for heads [64r, 64r + 64) and returns those P rows (bf16) to its peer.
+//
+// TMEM of one CTA (512 columns x 128 lanes; lane = head):
+//     [0, 144)   Q_r as the MMA A operand (288 bf16, two per column)
+//     [160, 224) S_r partial scores, fp32, 64 tokens
+//     [224, 256) P probabilities as the A operand (64 bf16)
+//     [256, 512) O_r accumulator, fp32
+// Both MMAs read A from TMEM and only the tile from shared memory, which keeps shared
+// memory bandwidth at 64 B/clk (a 128x64 MMA with both operands in shared memory needs
+// 192 B/clk, more than the SM supplies).
+//
+// Warp roles (192 threads): warp 0 issues TMA loads of 64-token tiles (4 latent chunks of
+// 64 columns + the 64 rotary columns, 128-byte swizzle) into a 4-stage ring; warp 1 owns
+// TMEM and issues the MMAs; warps 2-5 (thread = head = TMEM lane) load Q, exchange partial
+// scores, run the online softmax (base-2, lazy rescale: the running max moves only when a
+// tile exceeds it by more than 8, so p <= 256), write P, and read O back at the end.
+//
+// Work split: the tiles of all sequences, in order, are cut into equal ranges, one per
+// cluster; a range may hold pieces of several sequences.  Each piece writes an
+// un-normalised partial (O, running max, row sum) that a merge kernel combines.
+// Every wait is bounded; a timeout latches an error and the kernel drains and exits.
+#include <math.h>
+
+#include "common.cuh"
 #include "decode_tc.cuh"
+#include "gemm_tc.cuh"
+#include "tc_common.cuh"
 
 namespace mla {
 namespace tc {
 
-size_t decode_ws_bytes(int, int) { return 0; }
-DecodeWs carve_decode_ws(char*, int, int) { return DecodeWs{}; }
+namespace {
 
-cudaError_t decode_absorbed_tc(const __nv_bfloat16*, long long, long long, const __nv_bfloat16*,
-                               long long, long long, const __nv_bfloat16*, const __nv_bfloat16*,
-                               const __nv_bfloat16*, const int32_t*, int, float, __nv_bfloat16*,
-                               const DecodeWs&, int, int*, long long*, cudaStream_t) {
-    return cudaErrorNotSupported;
+constexpr int kT = 64;                        // tokens per tile
+constexpr int kStages = 4;
+constexpr int kChunkBytes = kT * 128;         // one 64-column box of a tile
+constexpr int kTileBytes = 5 * kChunkBytes;   // 4 latent chunks + the rotary chunk
+constexpr int kXStride = kT + 4;              // floats per exchanged score row (bank spread)
+constexpr int kXBytes = 64 * kXStride * 4;
+constexpr int kPRow = 144;                    // bytes per exchanged P row: 128 B + alpha
+constexpr int kPBytes = 64 * kPRow;
+constexpr int kBarBytes = 256;
+constexpr int kSmem = kStages * kTileBytes + 2 * kXBytes + 2 * kPBytes + kBarBytes + 1024;
+constexpr uint32_t kColQ = 0, kColS = 160, kColP = 224, kColO = 256, kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;     // log2 units
+
+// plan layout (int32): [0] total tiles, [1] tiles per cluster, [2] clusters,
+// [4, 4+B+1) first tile of each sequence, [4+B+1, 4+2B+2) first partial slot of each sequence
+__device__ __forceinline__ const int32_t* plan_tstart(const int32_t* w) { return w + 4; }
+__device__ __forceinline__ const int32_t* plan_sbase(const int32_t* w, int B) { return w + 4 + B + 1; }
+
+__global__ void plan_kernel(const int32_t* __restrict__ offsets, int B, int P, int32_t* __restrict__ work,
+                            int* err_code, long long* err_detail) {
+    if (threadIdx.x != 0) return;
+    int32_t* ts = work + 4;
+    int32_t* sb = work + 4 + B + 1;
+    long long t = 0;
+    for (int b = 0; b < B; ++b) {
+        long long L = (long long)offsets[b + 1] - offsets[b];
+        if (L < 0) {
+            latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
+            L = 0;
+        }
+        ts[b] = (int32_t)t;
+        t += (L + kT - 1) / kT;
+    }
+    ts[B] = (int32_t)t;
+    const int per = (int)((t + P - 1) / P) > 0 ? (int)((t + P - 1) / P) : 1;
+    int s = 0;
+    for (int b = 0; b < B; ++b) {
+        sb[b] = s;
+        const int nt = ts[b + 1] - ts[b];
+        if (nt > 0) s += (ts[b] + nt - 1) / per - ts[b] / per + 1;
+    }
+    sb[B] = s;
+    work[0] = (int32_t)t;
+    work[1] = per;
+    work[2] = P;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id_x() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+struct Seg {
+    int b, j0, j1, L, slot;
+    long long row0;
+};
+
+// Iterates over the pieces of sequences in this cluster's tile range (same order in both CTAs).
+struct SegIter {
+    const int32_t* ts;
+    const int32_t* sb;
+    const int32_t* offsets;
+    int B, lo, hi, per, cluster, b;
+    __device__ bool next(Seg& s) {
+        for (; b < B && ts[b] < hi; ++b) {
+            const int t0 = ts[b], t1 = ts[b + 1];
+            if (t1 <= lo || t1 == t0) continue;
+            s.b = b;
+            s.j0 = (lo > t0 ? lo : t0) - t0;
+            s.j1 = (hi < t1 ? hi : t1) - t0;
+            s.row0 = offsets[b];
+            s.L = offsets[b + 1] - offsets[b];
+            s.slot = sb[b] + cluster - t0 / per;
+            ++b;
+            return true;
+        }
+        return false;
+    }
+};
+
+__device__ __forceinline__ void fail(int* code, long long* detail, volatile int* abort_flag, int where) {
+    latch(DevErr{code, detail}, kErrTimeout, (long long)where * 1000000 + blockIdx.x);
+    *abort_flag = 1;
+}
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat16* __restrict__ q_lat,
+                 const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
+                 const int32_t* __restrict__ offsets, int B, long long cache_rows,
+                 const int32_t* __restrict__ work, float scale_log2,
+                 float* __restrict__ part_o, float* __restrict__ part_ml, int* err_code, long long* err_detail) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* tiles = smem;
+    float* xbuf = (float*)(smem + kStages * kTileBytes);
+    uint8_t* pbuf = (uint8_t*)xbuf + 2 * kXBytes;
+    uint64_t* bars = (uint64_t*)(pbuf + 2 * kPBytes);
+    uint64_t* tile_full = bars;
+    uint64_t* tile_empty = bars + kStages;
+    uint64_t* s_full = bars + 2 * kStages;
+    uint64_t* s_free = s_full + 1;
+    uint64_t* p_ready = s_full + 2;
+    uint64_t* o_done = s_full + 3;
+    uint64_t* q_ready = s_full + 4;
+    uint64_t* x_full = s_full + 5;   // [2] peer's partial scores arrived
+    uint64_t* x_empty = s_full + 7;  // [2] peer consumed the scores this CTA sent
+    uint64_t* p_full = s_full + 9;   // [2] peer's P rows arrived
+    uint64_t* p_empty = s_full + 11; // [2] peer consumed the P rows this CTA sent
+    uint64_t* drain = s_full + 13;   // all MMAs issued by this CTA have completed
+    uint32_t* tmem_slot = (uint32_t*)(s_full + 14);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+    const uint32_t rank = cluster_rank(), peer = rank ^ 1;
+    const int cluster = (int)cluster_id_x();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) {
+            ptx::mbar_init(&tile_full[s], 1);
+            ptx::mbar_init(&tile_empty[s], 1);
+        }
+        ptx::mbar_init(s_full, 1);
+        ptx::mbar_init(s_free, 128);
+        ptx::mbar_init(p_ready, 128);
+        ptx::mbar_init(o_done, 1);
+        ptx::mbar_init(q_ready, 128);
+        ptx::mbar_init(drain, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&x_full[i], 64);
+            ptx::mbar_init(&x_empty[i], 64);
+            ptx::mbar_init(&p_full[i], 64);
+            ptx::mbar_init(&p_empty[i], 64);
+        }
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, kTmemCols);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    cluster_sync_all();  // the peer's barriers exist before anyone arrives on them remotely
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    const int per = work[1];
+    const int total = work[0];
+    SegIter it{plan_tstart(work), plan_sbase(work, B), offsets, B, cluster * per,
+               min(total, cluster * per + per), per, cluster, 0};
+    Seg sg;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ TMA producer
+        if (lane == 0) {
+            ptx::tma_prefetch(&tm_cache);
+            uint32_t g = 0;
+            while (!*abort_flag && it.next(sg)) {
+                if (sg.row0 + (long long)sg.L > cache_rows) {   // sequence beyond the cache
+                    latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
+                    *abort_flag = 1;
+                    break;
+                }
+                for (int j = sg.j0; j < sg.j1; ++j, ++g) {
+                    const int s = g % kStages;
+                    const uint32_t n = g / kStages;
+                    if (g >= (uint32_t)kStages && !ptx::mbar_wait(&tile_empty[s], (n - 1) & 1, abort_flag)) {
+                        fail(err_code, err_detail, abort_flag, 1);
+                        break;
+                    }
+                    uint8_t* dst = tiles + s * kTileBytes;
+                    const int row = (int)(sg.row0 + (long long)j * kT);
+                    ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        ptx::tma_load_2d(dst + i * kChunkBytes, &tm_cache, &tile_full[s], 256 * (int)rank + 64 * i, row);
+                    ptx::tma_load_2d(dst + 4 * kChunkBytes, &tm_cache, &tile_full[s], 512, row);
+                }
+            }
+            // loads still in flight after an abort complete before the CTA leaves
+            for (uint32_t k = 0; k < (uint32_t)kStages && k < g; ++k) {
+                const uint32_t gg = g - 1 - k;
+                ptx::mbar_wait(&tile_full[gg % kStages], (gg / kStages) & 1, nullptr);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, kT, 0, 0);
+            constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 256, 0, 1);
+            uint32_t g = 0, sidx = 0;
+            bool ok = true;
+            auto issue_o = [&](uint32_t gt, bool first) -> bool {
+                if (!ptx::mbar_wait(p_ready, gt & 1, abort_flag)) return false;
+                ptx::tc_fence_after();
+                const uint32_t v = ptx::smem_u32(tiles + (gt % kStages) * kTileBytes);
+#pragma unroll
+                for (int k = 0; k < kT / 16; ++k)
+                    ptx::mma_ts(tmem + kColO, tmem + kColP + 8 * k, ptx::desc_mnmajor_sw128(v + 2048 * k, kChunkBytes),
+                                idesc_o, !(first && k == 0));
+                ptx::mma_commit(o_done);
+                ptx::mma_commit(&tile_empty[gt % kStages]);
+                return true;
+            };
+            while (ok && !*abort_flag && it.next(sg)) {
+                if (!ptx::mbar_wait(q_ready, sidx & 1, abort_flag)) { ok = false; break; }
+                for (int j = sg.j0; j < sg.j1; ++j, ++g) {
+                    const int s = g % kStages;
+                    if (!ptx::mbar_wait(&tile_full[s], (g / kStages) & 1, abort_flag)) { ok = false; break; }
+                    if (g > 0 && !ptx::mbar_wait(s_free, (g - 1) & 1, abort_flag)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    const uint32_t t = ptx::smem_u32(tiles + s * kTileBytes);
+#pragma unroll
+                    for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
+                        ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
+                                    ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
+                                    ks != 0);
+#pragma unroll
+                    for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
+                        ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
+                                    ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
+                    ptx::mma_commit(s_full);
+                    if (j > sg.j0 && !issue_o(g - 1, j - 1 == sg.j0)) { ok = false; break; }
+                }
+                if (!ok) break;
+                if (!issue_o(g - 1, sg.j1 - 1 == sg.j0)) { ok = false; break; }
+                ++sidx;
+            }
+            if (!ok) fail(err_code, err_detail, abort_flag, 2);
+            // drain: wait (bounded) for every MMA issued above before TMEM is released
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait(drain, 0, nullptr)) fail(err_code, err_detail, abort_flag, 4);
+        }
+    } else {
+        // ------------------------------------------------ softmax / exchange / epilogue
+        const int sub = warp & 3;
+        const int h = sub * 32 + lane;
+        const bool owner = (uint32_t)(sub >> 1) == rank;
+        const int hl = h & 63;
+        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+        const uint32_t xrow_local = ptx::smem_u32(xbuf) + (uint32_t)(hl * kXStride * 4);
+        const uint32_t prow_local = ptx::smem_u32(pbuf) + (uint32_t)(hl * kPRow);
+        uint32_t g = 0, sidx = 0;
+        bool ok = true;
+        // waits are made warp-uniform so the warp-collective TMEM instructions never diverge
+        auto uwait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag));
+        };
+        auto uwait_cluster = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, ptx::mbar_wait_cluster(bar, parity, abort_flag));
+        };
+        while (ok && !__any_sync(0xffffffffu, *abort_flag != 0) && it.next(sg)) {
+            // Q_r -> TMEM: 256 latent columns + 32 rotary columns of this head
+            {
+                const uint4* ql = (const uint4*)(q_lat + ((long long)sg.b * 128 + h) * 512 + 256 * rank);
+                const uint4* qr = (const uint4*)(q_rope + sg.b * sQr_b + h * sQr_h + 32 * rank);
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t r[32];
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const uint4 x = ql[c * 8 + v];
+                        r[4 * v] = x.x; r[4 * v + 1] = x.y; r[4 * v + 2] = x.z; r[4 * v + 3] = x.w;
+                    }
+                    ptx::tmem_st32(lane_addr + kColQ + 32 * c, r);
+                }
+                uint32_t r16[16];
+#pragma unroll
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 x = qr[v];
+                    r16[4 * v] = x.x; r16[4 * v + 1] = x.y; r16[4 * v + 2] = x.z; r16[4 * v + 3] = x.w;
+                }
+                ptx::tmem_st16(lane_addr + kColQ + 128, r16);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(q_ready);
+            }
+            float m_run = -INFINITY, l_run = 0.f;
+            for (int j = sg.j0; j < sg.j1; ++j, ++g) {
+                const uint32_t par = g & 1, use = g >> 1;
+                float s[kT];
+                if (!uwait(s_full, g & 1)) { ok = false; break; }
+                ptx::tc_fence_after();
+                {
+                    uint32_t r[32];
+                    ptx::tmem_ld32(lane_addr + kColS, r);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(r[i]);
+                    ptx::tmem_ld32(lane_addr + kColS + 32, r);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) s[32 + i] = __uint_as_float(r[i]);
+                }
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(s_free);
+                uint32_t pw[32];
+                float alpha;
+                if (!owner) {
+                    // send this partial score row to the CTA that owns the head
+                    if (g >= 2 && !uwait_cluster(&x_empty[par], (use - 1) & 1)) { ok = false; break; }
+                    const uint32_t dst = mapa(xrow_local + par * kXBytes, peer);
+#pragma unroll
+                    for (int i = 0; i < kT; i += 4)
+                        st_cluster_v4(dst + 4 * i, __float_as_uint(s[i]), __float_as_uint(s[i + 1]),
+                                      __float_as_uint(s[i + 2]), __float_as_uint(s[i + 3]));
+                    ptx::mbar_arrive_cluster(&x_full[par], peer);
+                    // receive its probabilities
+                    if (!uwait_cluster(&p_full[par], use & 1)) { ok = false; break; }
+                    const uint4* src = (const uint4*)(pbuf + par * kPBytes + hl * kPRow);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) {
+                        const uint4 x = src[v];
+                        pw[4 * v] = x.x; pw[4 * v + 1] = x.y; pw[4 * v + 2] = x.z; pw[4 * v + 3] = x.w;
+                    }
+                    alpha = __uint_as_float(src[8].x);
+                    ptx::mbar_arrive_cluster(&p_empty[par], peer);
+                } else {
+                    if (!uwait_cluster(&x_full[par], use & 1)) { ok = false; break; }
+                    const float4* src = (const float4*)(xbuf + par * (kXBytes / 4) + hl * kXStride);
+#pragma unroll
+                    for (int i = 0; i < kT / 4; ++i) {
+                        const float4 x = src[i];
+                        s[4 * i] += x.x; s[4 * i + 1] += x.y; s[4 * i + 2] += x.z; s[4 * i + 3] += x.w;
+                    }
+                    ptx::mbar_arrive_cluster(&x_empty[par], peer);
+                    // online softmax in base 2 over this tile's valid tokens
+                    const int valid = min(kT, sg.L - j * kT);
+                    float mt = -INFINITY;
+#pragma unroll
+                    for (int i = 0; i < kT; ++i) {
+                        s[i] = i < valid ? s[i] * scale_log2 : -INFINITY;
+                        mt = fmaxf(mt, s[i]);
+                    }
+                    alpha = 1.f;
+                    if (mt > m_run + kRescaleThreshold) {
+                        alpha = exp2f(m_run - mt);
+                        m_run = mt;
+                    }
+                    float sum = 0.f;
+#pragma unroll
+                    for (int i = 0; i < kT; i += 2) {
+                        const float p0 = exp2f(s[i] - m_run), p1 = exp2f(s[i + 1] - m_run);
+                        sum += p0 + p1;
+                        pw[i / 2] = ptx::pack_bf16(p0, p1);
+                    }
+                    l_run = l_run * alpha + sum;
+                    // send P and alpha to the peer, which holds the other half of O for this head
+                    if (g >= 2 && !uwait_cluster(&p_empty[par], (use - 1) & 1)) { ok = false; break; }
+                    const uint32_t dst = mapa(prow_local + par * kPBytes, peer);
+#pragma unroll
+                    for (int v = 0; v < 8; ++v) st_cluster_v4(dst + 16 * v, pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
+                    st_cluster_v4(dst + 128, __float_as_uint(alpha), 0u, 0u, 0u);
+                    ptx::mbar_arrive_cluster(&p_full[par], peer);
+                }
+                // P (TMEM) and O are free once the previous tile's O MMA has completed
+                if (g > 0 && !uwait(o_done, (g - 1) & 1)) { ok = false; break; }
+                ptx::tc_fence_after();
+                if (__any_sync(0xffffffffu, j > sg.j0 && alpha != 1.f)) {
+                    const float a = j > sg.j0 ? alpha : 1.f;
+#pragma unroll 1
+                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(lane_addr + kColO + c0, r);
+                        ptx::tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * a);
+                        ptx::tmem_st32(lane_addr + kColO + c0, r);
+                    }
+                }
+                ptx::tmem_st32(lane_addr + kColP, pw);
+                ptx::tmem_wait_st();
+                ptx::tc_fence_before();
+                ptx::mbar_arrive(p_ready);
+            }
+            if (!ok) break;
+            // piece epilogue: un-normalised O_r -> part_o[slot][c][h], (m, l) by the owner
+            if (!uwait(o_done, (g - 1) & 1)) { ok = false; break; }
+            ptx::tc_fence_after();
+            float* po = part_o + (long long)sg.slot * 512 * 128 + (long long)(256 * rank) * 128 + h;
+#pragma unroll 1
+            for (int c0 = 0; c0 < 256; c0 += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(lane_addr + kColO + c0, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) po[(long long)(c0 + i) * 128] = __uint_as_float(r[i]);
+            }
+            if (owner) {
+                part_ml[((long long)sg.slot * 128 + h) * 2] = m_run;
+                part_ml[((long long)sg.slot * 128 + h) * 2 + 1] = l_run;
+            }
+            ptx::tc_fence_before();
+            ++sidx;
+        }
+        if (!ok) fail(err_code, err_detail, abort_flag, 3);
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, kTmemCols);
+    cluster_sync_all();  // neither CTA leaves while its peer may still touch its shared memory
+}
+
+// ------------------------------------------------------------------- merge
+// o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[c,h] / sum_p 2^(m_p - M) l_p  over the pieces p of b.
+__global__ void __launch_bounds__(256)
+combine_tc_kernel(const int32_t* __restrict__ work, int B, const float* __restrict__ part_o,
+                  const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o_lat) {
+    const int b = blockIdx.x, cb = blockIdx.y;   // 64 latent columns per block
+    const int h = threadIdx.x & 127, half = threadIdx.x >> 7;
+    const int32_t* ts = plan_tstart(work);
+    const int32_t* sb = plan_sbase(work, B);
+    const int per = work[1];
+    const int t0 = ts[b], t1 = ts[b + 1];
+    __nv_bfloat16* dst = o_lat + ((long long)b * 128 + h) * 512 + cb * 64 + half * 32;
+    if (t1 == t0) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) dst[i] = __float2bfloat16_rn(0.f);
+        return;
+    }
+    const int np = (t1 - 1) / per - t0 / per + 1;
+    const int base = sb[b];
+    float M = -INFINITY;
+    for (int p = 0; p < np; ++p) M = fmaxf(M, part_ml[((long long)(base + p) * 128 + h) * 2]);
+    float L = 0.f;
+    for (int p = 0; p < np; ++p) {
+        const long long q = ((long long)(base + p) * 128 + h) * 2;
+        L += exp2f(part_ml[q] - M) * part_ml[q + 1];
+    }
+    float acc[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
+    for (int p = 0; p < np; ++p) {
+        const float w = exp2f(part_ml[((long long)(base + p) * 128 + h) * 2] - M) / L;
+        const float* src = part_o + (long long)(base + p) * 512 * 128 + (long long)(cb * 64 + half * 32) * 128 + h;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, src[(long long)i * 128], acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        __nv_bfloat162 v = __floats2bfloat162_rn(acc[i], acc[i + 1]);
+        *reinterpret_cast<__nv_bfloat162*>(dst + i) = v;
+    }
+}
+
+int g_clusters_cached = 0;
+
+int max_clusters(int num_sms) {
+    if (g_clusters_cached > 0) return g_clusters_cached;
+    cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
+    cfg.blockDim = dim3(192, 1, 1);
+    cfg.dynamicSmemBytes = kSmem;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+        cudaGetLastError();
+        n = num_sms / 2;
+    }
+    g_clusters_cached = n;
+    return n;
+}
+
+}  // namespace
+
+size_t decode_ws_bytes(int B, int num_sms) {
+    const size_t P = (size_t)(num_sms / 2);
+    const size_t slots = (size_t)B + P + 1;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    return up((size_t)B * 128 * 512 * 2) + up((4 + 2 * ((size_t)B + 1)) * 4) + up(slots * 512 * 128 * 4) +
+           up(slots * 128 * 2 * 4) + up((size_t)B * 128 * 512 * 2);
+}
+
+DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
+    const size_t P = (size_t)(num_sms / 2);
+    const size_t slots = (size_t)B + P + 1;
+    auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+    DecodeWs w{};
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> char* {
+        char* p = base ? base + off : nullptr;
+        off += up(bytes);
+        return p;
+    };
+    w.q_lat = (__nv_bfloat16*)take((size_t)B * 128 * 512 * 2);
+    w.work = (int32_t*)take((4 + 2 * ((size_t)B + 1)) * 4);
+    w.part_o = (float*)take(slots * 512 * 128 * 4);
+    w.part_ml = (float*)take(slots * 128 * 2 * 4);
+    w.o_lat = (__nv_bfloat16*)take((size_t)B * 128 * 512 * 2);
+    w.q_cat = nullptr;
+    w.max_parts = (int)slots;
+    return w;
+}
+
+cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h, const __nv_bfloat16* qr,
+                               long long sQr_b, long long sQr_h, const __nv_bfloat16* W_UKT,
+                               const __nv_bfloat16* W_UV, const __nv_bfloat16* cache, long long cache_rows,
+                               const int32_t* offsets, int B, float scale, __nv_bfloat16* o, const DecodeWs& ws,
+                               int num_sms,
+                               int* err_code, long long* err_detail, cudaStream_t s) {
+    if (B <= 0) return cudaSuccess;
+    cudaError_t e;
+    if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    const int P = max_clusters(num_sms);
+    {
+        ProfScope ps(s, "tc_plan");
+        plan_kernel<<<1, 32, 0, s>>>(offsets, B, P, ws.work, err_code, err_detail);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]  (per head: [512 x 128] x [128 x B])
+        ProfScope ps(s, "tc_q_absorb");
+        GemmOut out{ws.q_lat, 512, 1, 128LL * 512, 0};
+        e = gemm_bf16_tc(128, 512, B, 128, W_UKT, 512LL * 128, 128, qn, sQn_h, sQn_b, out, err_code, err_detail, s);
+        if (e != cudaSuccess) return e;
+    }
+    {
+        ProfScope ps(s, "tc_flash_decode");
+        CUtensorMap m;
+        const uint64_t dims[2] = {576, (uint64_t)cache_rows};
+        const uint64_t strides[1] = {576 * 2};
+        const uint32_t box[2] = {64, (uint32_t)kT};
+        if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        decode_tc_kernel<<<2 * P, 192, kSmem, s>>>(m, ws.q_lat, qr, sQr_b, sQr_h, offsets, B, cache_rows, ws.work,
+                                                    scale * 1.4426950408889634f, ws.part_o, ws.part_ml, err_code,
+                                                    err_detail);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        ProfScope ps(s, "tc_combine");
+        combine_tc_kernel<<<dim3(B, 8), 256, 0, s>>>(ws.work, B, ws.part_o, ws.part_ml, ws.o_lat);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    {
+        // o[b,h,:] = W_UV[h] o_lat[b,h,:]  (per head: [128 x 512] x [512 x B])
+        ProfScope ps(s, "tc_w_uv");
+        GemmOut out{o, 128, 1, 128LL * 128, 0};
+        e = gemm_bf16_tc(128, 128, B, 512, W_UV, 128LL * 512, 512, ws.o_lat, 512, 128LL * 512, out, err_code,
+                         err_detail, s);
+    }
+    return e;
 }
 
 }  // namespace tc

@@ -14,15 +14,15 @@ constexpr int kH = 128;
 constexpr int kDc = 512;
 constexpr int kDr = 64;
 constexpr int kRow = kDc + kDr;  // 576 cache elements per token
-constexpr bool kEnabled = false;
+constexpr bool kEnabled = true;
 
 // Workspace pieces of the tensor-core decode (all device memory, carved by the caller).
 struct DecodeWs {
     __nv_bfloat16* q_lat;   // [B, H, d_c] absorbed query, bf16
-    __nv_bfloat16* q_cat;   // [B, H, 576] = [q_lat | q_rope] (the MMA A operand)
-    float* part_o;          // [max_parts, H, d_c] un-normalised partial o_lat
+    __nv_bfloat16* q_cat;   // unused
+    float* part_o;          // [max_parts, d_c, H] un-normalised partial o_lat
     float* part_ml;         // [max_parts, H, 2] running max (log2 domain) and sum
-    int32_t* work;          // split plan: [n_ctas + 1] ranges and per-part metadata
+    int32_t* work;          // split plan: totals, first tile and first partial slot per sequence
     __nv_bfloat16* o_lat;   // [B, H, d_c] merged, normalised o_lat (bf16, W_UV operand)
     int max_parts;
 };
@@ -35,8 +35,8 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms);
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
                                const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV,
-                               const __nv_bfloat16* cache, const int32_t* offsets, int B,
-                               float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
+                               const __nv_bfloat16* cache, long long cache_rows, const int32_t* offsets,
+                               int B, float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s);
 
 }  // namespace tc

@@ -42,15 +42,16 @@ mla_status scratch_address(void** out) {
 extern "C" mla_status mla_decode_absorbed_noalloc(const mla_dims* dims, mla_weights w,
                                                   const void* q_nope, const void* q_rope,
                                                   const void* h, const int32_t* q_pos,
-                                                  const void* cache, const int32_t* offsets,
-                                                  int32_t B, void* out, mla_stream_t stream) {
+                                                  const void* cache, int64_t cache_rows,
+                                                  const int32_t* offsets, int32_t B, void* out,
+                                                  mla_stream_t stream) {
     const size_t need = mla_decode_workspace_size(dims, B);
     if (need == 0 && B != 0) return mla_decode_absorbed(dims, w, q_nope, q_rope, h, q_pos, cache,
-                                                        offsets, B, out, nullptr, 0, stream);
+                                                        cache_rows, offsets, B, out, nullptr, 0, stream);
     if (need > (size_t)MLA_NOALLOC_SCRATCH_BYTES) return MLA_ERR_WORKSPACE;
     void* scratch = nullptr;
     mla_status st = scratch_address(&scratch);
     if (st != MLA_OK) return st;
-    return mla_decode_absorbed(dims, w, q_nope, q_rope, h, q_pos, cache, offsets, B, out, scratch,
+    return mla_decode_absorbed(dims, w, q_nope, q_rope, h, q_pos, cache, cache_rows, offsets, B, out, scratch,
                                (size_t)MLA_NOALLOC_SCRATCH_BYTES, stream);
 }

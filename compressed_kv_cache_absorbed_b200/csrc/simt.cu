@@ -166,8 +166,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 decode_split_simt_kernel(const float* __restrict__ q_lat, const T* __restrict__ q_rope,
                          long long sQb, long long sQh, const T* __restrict__ cache,
-                         const int32_t* __restrict__ offsets, int B, int H, int d_c, int d_hR,
-                         float scale, int nsplit, float* __restrict__ part_o,
+                         long long cache_rows, const int32_t* __restrict__ offsets, int B, int H,
+                         int d_c, int d_hR, float scale, int nsplit, float* __restrict__ part_o,
                          float* __restrict__ part_ml, DevErr err) {
     extern __shared__ float sm[];
     const int row = d_c + d_hR, rs = row + 1;
@@ -177,9 +177,9 @@ decode_split_simt_kernel(const float* __restrict__ q_lat, const T* __restrict__ 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     const int h = hg * kDecHPB + warp;
     long long r0 = offsets[b], r1 = offsets[b + 1];
-    if (r1 < r0) {
+    if (r1 < r0 || r0 < 0 || r1 > cache_rows) {
         if (threadIdx.x == 0 && split == 0 && hg == 0) latch(err, kErrOutOfRange, b);
-        r1 = r0;
+        r0 = r1 = 0;
     }
     const long long Tn = r1 - r0;
     const long long chunk = (Tn + nsplit - 1) / nsplit;
@@ -432,9 +432,10 @@ cudaError_t launch_gemm_nt(int Z, int M, int N, int K, const TA* A, long long sA
 
 template <typename T>
 cudaError_t launch_decode_split_simt(const float* q_lat, const T* q_rope, long long sQb,
-                                     long long sQh, const T* cache, const int32_t* offsets,
-                                     int B, int H, int d_c, int d_hR, float scale, int nsplit,
-                                     float* part_o, float* part_ml, DevErr err, cudaStream_t s) {
+                                     long long sQh, const T* cache, long long cache_rows,
+                                     const int32_t* offsets, int B, int H, int d_c, int d_hR,
+                                     float scale, int nsplit, float* part_o, float* part_ml,
+                                     DevErr err, cudaStream_t s) {
     if (B == 0) return cudaSuccess;
     const int row = d_c + d_hR;
     const size_t smem = sizeof(float) * ((size_t)kDecTT * (row + 1) + (size_t)kDecHPB * row);
@@ -442,7 +443,7 @@ cudaError_t launch_decode_split_simt(const float* q_lat, const T* q_rope, long l
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     dim3 grid(nsplit, B, ceil_div(H, kDecHPB));
-    decode_split_simt_kernel<T><<<grid, 256, smem, s>>>(q_lat, q_rope, sQb, sQh, cache, offsets, B,
+    decode_split_simt_kernel<T><<<grid, 256, smem, s>>>(q_lat, q_rope, sQb, sQh, cache, cache_rows, offsets, B,
                                                         H, d_c, d_hR, scale, nsplit, part_o,
                                                         part_ml, err);
     return cudaGetLastError();
@@ -487,9 +488,9 @@ using bf16 = __nv_bfloat16;
                                              const int64_t*, long long, T*, long long, DevErr,  \
                                              cudaStream_t);                                     \
     template cudaError_t launch_decode_split_simt<T>(const float*, const T*, long long,         \
-                                                     long long, const T*, const int32_t*, int,  \
-                                                     int, int, int, float, int, float*, float*, \
-                                                     DevErr, cudaStream_t);                     \
+                                                     long long, const T*, long long,            \
+                                                     const int32_t*, int, int, int, int, float, \
+                                                     int, float*, float*, DevErr, cudaStream_t);\
     template cudaError_t launch_prefill_attn_simt<T>(const T*, const T*, const T*, const T*,    \
                                                      int, int, int, int, int, int, int, float,  \
                                                      T*, cudaStream_t);                         \

@@ -140,7 +140,9 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t B);
  *     o_lat[b,h]  = sum_t softmax_t(s[b,h,:]) c_t                 (d_c, fp32)
  *     o[b,h]      = W_UV[h] o_lat[b,h]                            (v_head)
  *     out[b]      = W_O concat_h o[b,h]        (only when the handle holds W_O)
- * Sequence b attends over cache rows [offsets[b], offsets[b+1]) (int32 [B+1], ragged).
+ * Sequence b attends over cache rows [offsets[b], offsets[b+1]) (int32 [B+1], ragged) of a
+ * cache of cache_rows rows (1 <= cache_rows < 2^31); a sequence reaching past cache_rows
+ * latches MLA_ERR_OUT_OF_RANGE.
  * An empty sequence gives o = 0.  The query comes either from (q_nope [B,H,qk_nope],
  * q_rope [B,H,d_hR], q_rope already rotated) or, when both are NULL, from the hidden
  * state h [B, d_model] through the handle's W_Q with RoPE at q_pos int32 [B].
@@ -149,8 +151,8 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t B);
  * its contents on entry do not matter.  Decreasing offsets latch MLA_ERR_OUT_OF_RANGE. */
 mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* q_nope,
                                const void* q_rope, const void* h, const int32_t* q_pos,
-                               const void* cache, const int32_t* offsets, int32_t B,
-                               void* out, void* workspace, size_t ws_bytes,
+                               const void* cache, int64_t cache_rows, const int32_t* offsets,
+                               int32_t B, void* out, void* workspace, size_t ws_bytes,
                                mla_stream_t stream);
 
 /* Size of the fixed device scratch used by mla_decode_absorbed_noalloc (64 MiB). */
@@ -175,8 +177,9 @@ mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* 
  *     results; order them on one stream or with events. */
 mla_status mla_decode_absorbed_noalloc(const mla_dims* dims, mla_weights w, const void* q_nope,
                                        const void* q_rope, const void* h, const int32_t* q_pos,
-                                       const void* cache, const int32_t* offsets, int32_t B,
-                                       void* out, mla_stream_t stream);
+                                       const void* cache, int64_t cache_rows,
+                                       const int32_t* offsets, int32_t B, void* out,
+                                       mla_stream_t stream);
 
 /* ---------------------------------------------------------------- causal prefill */
 

@@ -51,6 +51,7 @@ def test_cache_row_matches_the_oracle_and_the_pages():
 
 
 def test_decode_path_selection():
+    assert mla.mla_decode_path(v3()) == 1                     # bf16 V2/V3 head shape: tcgen05
     assert mla.mla_decode_path(v3(dtype="f32")) == 0
     assert mla.mla_decode_path(v3(d_hR=63)) == -1              # odd rotary width
     assert mla.mla_decode_path(v3(d_c=1024)) == -1             # wider than the kernels
@@ -84,6 +85,6 @@ def test_argument_errors_return_before_any_launch():
     assert lib.mla_append_cache(ctypes.byref(bad), None, None, None, None, None, 1, None, 1, None) == mla.MLA_ERR_UNSUPPORTED
     h = ctypes.c_void_p()
     assert lib.mla_absorb_weights(ctypes.byref(d), None, None, None, None, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
-    assert lib.mla_decode_absorbed(ctypes.byref(d), None, None, None, None, None, None, None, 1, None, None, 0, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_absorbed(ctypes.byref(d), None, None, None, None, None, None, 0, None, 1, None, None, 0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_prefill_causal(ctypes.byref(d), None, None, None, None, None, None, 1, 1, None, 0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_weights_destroy(None) == mla.MLA_OK
