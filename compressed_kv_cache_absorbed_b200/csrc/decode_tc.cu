@@ -11,8 +11,9 @@
 // owns c columns [256r, 256r + 256) and rotary columns [32r, 32r + 32), loads only those
 // (no duplicate HBM/L2 traffic, no multicast), and accumulates O_r = 128 x 256.  The
 // softmax needs the full 576-long scores, so each CTA computes a partial S_r over its 288
-// columns and the pair exchanges halves through distributed shared memory: CTA r finishes
-// the softmax for heads [64r, 64r + 64) and returns those P rows (bf16) to its peer.
+// columns and the pair swaps them through distributed shared memory (one 16 KB bulk copy
+// per tile, bf16 partials); both CTAs then run the same softmax for all 128 heads,
+// which costs 64 exponentials per thread per tile and saves a second exchange hop.
 //
 // TMEM of one CTA (512 columns x 128 lanes; lane = head):
 //     [0, 144)   Q_r as the MMA A operand (288 bf16, two per column)
@@ -24,8 +25,8 @@
 // 192 B/clk, more than the SM supplies).
 //
 // Warp roles (192 threads): warp 0 issues TMA loads of 64-token tiles (4 latent chunks of
-// 64 columns + the 64 rotary columns, 128-byte swizzle) into a 4-stage ring; warp 1 owns
-// TMEM and issues the MMAs; warps 2-5 (thread = head = TMEM lane) load Q, exchange partial
+// 64 columns + the 64 rotary columns, 128-byte swizzle) into a 3-stage ring; warp 1 owns
+// TMEM and issues the MMAs; warps 2-5 (thread = head = TMEM lane) load Q, swap partial
 // scores, run the online softmax (base-2, lazy rescale: the running max moves only when a
 // tile exceeds it by more than 8, so p <= 256), write P, and read O back at the end.
 //
@@ -49,47 +50,99 @@ constexpr int kT = 64;                        // tokens per tile
 constexpr int kStages = 4;
 constexpr int kChunkBytes = kT * 128;         // one 64-column box of a tile
 constexpr int kTileBytes = 5 * kChunkBytes;   // 4 latent chunks + the rotary chunk
-constexpr int kXStride = kT + 4;              // floats per exchanged score row (bank spread)
-constexpr int kXBytes = 64 * kXStride * 4;
-constexpr int kPRow = 144;                    // bytes per exchanged P row: 128 B + alpha
-constexpr int kPBytes = 64 * kPRow;
+constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
+constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
 constexpr int kBarBytes = 256;
-constexpr int kSmem = kStages * kTileBytes + 2 * kXBytes + 2 * kPBytes + kBarBytes + 1024;
+// tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer)
+constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kBarBytes + 1024;
 constexpr uint32_t kColQ = 0, kColS = 160, kColP = 224, kColO = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
+constexpr int kThreads = 320;                 // producer, MMA, 4 sender and 4 softmax warps
 
 // plan layout (int32): [0] total tiles, [1] tiles per cluster, [2] clusters,
 // [4, 4+B+1) first tile of each sequence, [4+B+1, 4+2B+2) first partial slot of each sequence
 __device__ __forceinline__ const int32_t* plan_tstart(const int32_t* w) { return w + 4; }
 __device__ __forceinline__ const int32_t* plan_sbase(const int32_t* w, int B) { return w + 4 + B + 1; }
 
-__global__ void plan_kernel(const int32_t* __restrict__ offsets, int B, int P, int32_t* __restrict__ work,
-                            int* err_code, long long* err_detail) {
-    if (threadIdx.x != 0) return;
-    int32_t* ts = work + 4;
-    int32_t* sb = work + 4 + B + 1;
-    long long t = 0;
-    for (int b = 0; b < B; ++b) {
+// Block-wide exclusive scan of one value per thread (256 threads) with warp shuffles.
+template <typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    T incl = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const T n = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_tot[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+        T t = lane < 8 ? warp_tot[lane] : T(0);
+        T ti = t;
+#pragma unroll
+        for (int o = 1; o < 8; o <<= 1) {
+            const T n = __shfl_up_sync(0xffffffffu, ti, o);
+            if (lane >= o) ti += n;
+        }
+        if (lane < 8) warp_tot[lane] = ti - t;
+        if (lane == 7) *total = ti;
+    }
+    __syncthreads();
+    return warp_tot[w] + incl - v;
+}
+
+// One block of 256 threads: each thread takes a contiguous run of sequences; two block
+// scans give every sequence its first tile and its first partial slot.
+__global__ void __launch_bounds__(256)
+plan_kernel(const int32_t* __restrict__ offsets, int B, int P, int32_t* __restrict__ work, int* err_code,
+            long long* err_detail) {
+    __shared__ long long s_wt[8];
+    __shared__ long long s_tot;
+    __shared__ int s_wp[8];
+    __shared__ int s_ptot;
+    const int t = threadIdx.x;
+    const int per_thread = (B + 255) / 256;
+    const int b0 = min(B, t * per_thread), b1 = min(B, b0 + per_thread);
+    auto tiles_of = [&](int b) -> long long {
         long long L = (long long)offsets[b + 1] - offsets[b];
         if (L < 0) {
             latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
             L = 0;
         }
-        ts[b] = (int32_t)t;
-        t += (L + kT - 1) / kT;
+        return (L + kT - 1) / kT;
+    };
+    long long mine = 0;
+    for (int b = b0; b < b1; ++b) mine += tiles_of(b);
+    const long long t_first = block_exclusive_scan<long long>(mine, s_wt, &s_tot);
+    const long long total = s_tot;
+    const long long per_l = (total + P - 1) / P;
+    const int per = per_l > 0 ? (int)per_l : 1;
+    int32_t* ts = work + 4;
+    long long tcur = t_first;
+    int pieces = 0;
+    for (int b = b0; b < b1; ++b) {
+        const long long nt = tiles_of(b);
+        ts[b] = (int32_t)tcur;
+        if (nt > 0) pieces += (int)((tcur + nt - 1) / per - tcur / per + 1);
+        tcur += nt;
     }
-    ts[B] = (int32_t)t;
-    const int per = (int)((t + P - 1) / P) > 0 ? (int)((t + P - 1) / P) : 1;
-    int s = 0;
-    for (int b = 0; b < B; ++b) {
-        sb[b] = s;
-        const int nt = ts[b + 1] - ts[b];
-        if (nt > 0) s += (ts[b] + nt - 1) / per - ts[b] / per + 1;
+    const int p_first = block_exclusive_scan<int>(pieces, s_wp, &s_ptot);
+    int32_t* sb = work + 4 + B + 1;
+    tcur = t_first;
+    int scur = p_first;
+    for (int b = b0; b < b1; ++b) {
+        sb[b] = scur;
+        const long long nt = tiles_of(b);
+        if (nt > 0) scur += (int)((tcur + nt - 1) / per - tcur / per + 1);
+        tcur += nt;
     }
-    sb[B] = s;
-    work[0] = (int32_t)t;
-    work[1] = per;
-    work[2] = P;
+    if (t == 0) {
+        work[0] = (int32_t)total;
+        work[1] = per;
+        work[2] = P;
+        work[4 + B] = (int32_t)total;
+        work[4 + B + 1 + B] = s_ptot;
+    }
 }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -110,9 +163,21 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
     return r;
 }
-__device__ __forceinline__ void st_cluster_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared::cluster.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d)
-                 : "memory");
+
+// Two floats rounded to bf16 (nearest even) with integer operations and packed into one
+// word (first value in the low half).  Both CTAs of a pair round their own partial scores
+// with this, so the sums they form are identical.
+__device__ __forceinline__ uint32_t bf16_pair_rne(float a, float b) {
+    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
+    const uint32_t ra = ua + 0x7FFFu + ((ua >> 16) & 1u);
+    const uint32_t rb = ub + 0x7FFFu + ((ub >> 16) & 1u);
+    return __byte_perm(ra, rb, 0x7632);
+}
+// 2^x with the hardware approximation (inputs here are <= 8; results below 2^-126 flush to 0)
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
 struct Seg {
@@ -148,7 +213,7 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
     *abort_flag = 1;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(192, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
@@ -157,9 +222,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint8_t* tiles = smem;
-    float* xbuf = (float*)(smem + kStages * kTileBytes);
-    uint8_t* pbuf = (uint8_t*)xbuf + 2 * kXBytes;
-    uint64_t* bars = (uint64_t*)(pbuf + 2 * kPBytes);
+    uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
+    uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
+    uint64_t* bars = (uint64_t*)(xstage + 2 * kXBytes);
     uint64_t* tile_full = bars;
     uint64_t* tile_empty = bars + kStages;
     uint64_t* s_full = bars + 2 * kStages;
@@ -167,11 +232,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     uint64_t* p_ready = s_full + 2;
     uint64_t* o_done = s_full + 3;
     uint64_t* q_ready = s_full + 4;
-    uint64_t* x_full = s_full + 5;   // [2] peer's partial scores arrived
-    uint64_t* x_empty = s_full + 7;  // [2] peer consumed the scores this CTA sent
-    uint64_t* p_full = s_full + 9;   // [2] peer's P rows arrived
-    uint64_t* p_empty = s_full + 11; // [2] peer consumed the P rows this CTA sent
-    uint64_t* drain = s_full + 13;   // all MMAs issued by this CTA have completed
+    // [2] the peer's partial scores for tile g landed in xbuf[g & 1]: armed locally with the
+    // byte count, completed by the peer's bulk copy
+    uint64_t* x_full = s_full + 5;
+    // [2] the peer has read what this CTA sent into its xbuf[g & 1]; that copy therefore also
+    // finished reading this CTA's xstage[g & 1] (one arrive per peer warp)
+    uint64_t* x_empty = s_full + 7;
+    uint64_t* drain = s_full + 9;    // all MMAs issued by this CTA have completed
+    uint64_t* xs_ready = s_full + 10;  // [2] all 128 rows of xstage[g & 1] written
+    uint64_t* xs_free = s_full + 12;   // [2] the local softmax has read xstage[g & 1]
     uint32_t* tmem_slot = (uint32_t*)(s_full + 14);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -191,10 +260,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         ptx::mbar_init(q_ready, 128);
         ptx::mbar_init(drain, 1);
         for (int i = 0; i < 2; ++i) {
-            ptx::mbar_init(&x_full[i], 64);
-            ptx::mbar_init(&x_empty[i], 64);
-            ptx::mbar_init(&p_full[i], 64);
-            ptx::mbar_init(&p_empty[i], 64);
+            ptx::mbar_init(&x_full[i], 1);
+            ptx::mbar_init(&x_empty[i], 4);
+            ptx::mbar_init(&xs_ready[i], 128);
+            ptx::mbar_init(&xs_free[i], 128);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -267,29 +336,50 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 ptx::mma_commit(&tile_empty[gt % kStages]);
                 return true;
             };
-            while (ok && !*abort_flag && it.next(sg)) {
-                if (!ptx::mbar_wait(q_ready, sidx & 1, abort_flag)) { ok = false; break; }
-                for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int s = g % kStages;
-                    if (!ptx::mbar_wait(&tile_full[s], (g / kStages) & 1, abort_flag)) { ok = false; break; }
-                    if (g > 0 && !ptx::mbar_wait(s_free, (g - 1) & 1, abort_flag)) { ok = false; break; }
-                    ptx::tc_fence_after();
-                    const uint32_t t = ptx::smem_u32(tiles + s * kTileBytes);
+            // S runs two tiles ahead of O: S of tile t+2 needs only that the softmax warps
+            // have read S of tile t+1 (they do so while finishing tile t), while O of tile t
+            // needs P of tile t.  The tile order is one flat pass over all pieces.
+            SegIter its = it;   // second iterator: tiles whose S is issued next
+            Seg ss;
+            bool s_have = !*abort_flag && its.next(ss);
+            int s_j = s_have ? ss.j0 : 0;
+            uint32_t s_g = 0;
+            auto issue_s = [&]() -> bool {   // S of tile s_g (= s_j of piece ss), then advance
+                if (s_j == ss.j0 && !ptx::mbar_wait(q_ready, (sidx++) & 1, abort_flag)) return false;
+                const int st = s_g % kStages;
+                if (!ptx::mbar_wait(&tile_full[st], (s_g / kStages) & 1, abort_flag)) return false;
+                if (s_g > 0 && !ptx::mbar_wait(s_free, (s_g - 1) & 1, abort_flag)) return false;
+                ptx::tc_fence_after();
+                const uint32_t t = ptx::smem_u32(tiles + st * kTileBytes);
 #pragma unroll
-                    for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
-                        ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
-                                    ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
-                                    ks != 0);
+                for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
+                    ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
+                                ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
+                                ks != 0);
 #pragma unroll
-                    for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
-                        ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
-                                    ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
-                    ptx::mma_commit(s_full);
-                    if (j > sg.j0 && !issue_o(g - 1, j - 1 == sg.j0)) { ok = false; break; }
+                for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
+                    ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
+                                ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
+                ptx::mma_commit(s_full);
+                ++s_g;
+                if (++s_j == ss.j1) {
+                    s_have = !*abort_flag && its.next(ss);
+                    s_j = s_have ? ss.j0 : 0;
                 }
-                if (!ok) break;
-                if (!issue_o(g - 1, sg.j1 - 1 == sg.j0)) { ok = false; break; }
-                ++sidx;
+                return true;
+            };
+            // O follows the same flat order with the primary iterator
+            bool have = !*abort_flag && it.next(sg);
+            int j = have ? sg.j0 : 0;
+            for (int k = 0; k < 2 && ok && s_have; ++k) ok = issue_s();
+            while (ok && have) {
+                if (s_have && !issue_s()) { ok = false; break; }
+                if (!issue_o(g, j == sg.j0)) { ok = false; break; }
+                ++g;
+                if (++j == sg.j1) {
+                    have = !*abort_flag && it.next(sg);
+                    j = have ? sg.j0 : 0;
+                }
             }
             if (!ok) fail(err_code, err_detail, abort_flag, 2);
             // drain: wait (bounded) for every MMA issued above before TMEM is released
@@ -297,15 +387,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             if (!ptx::mbar_wait(drain, 0, nullptr)) fail(err_code, err_detail, abort_flag, 4);
         }
     } else {
-        // ------------------------------------------------ softmax / exchange / epilogue
+        // warps 2-5 send partial scores, warps 6-9 run the softmax; warp w works on TMEM
+        // lanes 32 * (w % 4) .. +31, so thread h of either role owns head h
         const int sub = warp & 3;
         const int h = sub * 32 + lane;
-        const bool owner = (uint32_t)(sub >> 1) == rank;
-        const int hl = h & 63;
         const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
-        const uint32_t xrow_local = ptx::smem_u32(xbuf) + (uint32_t)(hl * kXStride * 4);
-        const uint32_t prow_local = ptx::smem_u32(pbuf) + (uint32_t)(hl * kPRow);
-        uint32_t g = 0, sidx = 0;
+        const bool sender = warp < 6;
         bool ok = true;
         // waits are made warp-uniform so the warp-collective TMEM instructions never diverge
         auto uwait = [&](uint64_t* bar, uint32_t parity) {
@@ -314,11 +401,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         auto uwait_cluster = [&](uint64_t* bar, uint32_t parity) {
             return __all_sync(0xffffffffu, ptx::mbar_wait_cluster(bar, parity, abort_flag));
         };
-        while (ok && !__any_sync(0xffffffffu, *abort_flag != 0) && it.next(sg)) {
-            // Q_r -> TMEM: 256 latent columns + 32 rotary columns of this head
-            {
-                const uint4* ql = (const uint4*)(q_lat + ((long long)sg.b * 128 + h) * 512 + 256 * rank);
-                const uint4* qr = (const uint4*)(q_rope + sg.b * sQr_b + h * sQr_h + 32 * rank);
+        // exchange rows are 128 B (64 bf16); 16-byte chunk v of row h sits at chunk
+        // v ^ (h & 7), so a warp's row accesses hit all 32 banks
+        Seg cur;
+        bool have = it.next(cur);
+        int j = have ? cur.j0 : 0;
+        uint32_t g = 0;
+        if (sender) {
+            // ------------------------------------------------------- score senders
+            // Q_r of sequence b -> TMEM: 256 latent columns + 32 rotary columns of this head
+            auto load_q = [&](int b) {
+                const uint4* ql = (const uint4*)(q_lat + ((long long)b * 128 + h) * 512 + 256 * rank);
+                const uint4* qr = (const uint4*)(q_rope + b * sQr_b + h * sQr_h + 32 * rank);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
@@ -339,90 +433,116 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(q_ready);
-            }
-            float m_run = -INFINITY, l_run = 0.f;
-            for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                const uint32_t par = g & 1, use = g >> 1;
-                float s[kT];
+            };
+            if (have) load_q(cur.b);
+            while (have) {
+                const uint32_t b = g & 1, u = g >> 1;
+                // partial scores: TMEM -> registers (log2 units, bf16 pairs)
                 if (!uwait(s_full, g & 1)) { ok = false; break; }
                 ptx::tc_fence_after();
+                uint32_t own[32];
                 {
                     uint32_t r[32];
+                    float sc[kT];
                     ptx::tmem_ld32(lane_addr + kColS, r);
-                    ptx::tmem_wait_ld();
+                    ptx::tmem_ld32x2_second(lane_addr + kColS + 32, sc, r);
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(s_free);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) s[i] = __uint_as_float(r[i]);
-                    ptx::tmem_ld32(lane_addr + kColS + 32, r);
-                    ptx::tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) s[32 + i] = __uint_as_float(r[i]);
+                    for (int i = 0; i < kT; i += 2) own[i / 2] = bf16_pair_rne(sc[i] * scale_log2, sc[i + 1] * scale_log2);
                 }
-                ptx::tc_fence_before();
-                ptx::mbar_arrive(s_free);
-                uint32_t pw[32];
-                float alpha;
-                if (!owner) {
-                    // send this partial score row to the CTA that owns the head
-                    if (g >= 2 && !uwait_cluster(&x_empty[par], (use - 1) & 1)) { ok = false; break; }
-                    const uint32_t dst = mapa(xrow_local + par * kXBytes, peer);
+                // staging buffer b is free once the local softmax read it (tile g-2) and the
+                // peer read the copy made from it
+                if (g >= 2 && !(uwait(&xs_free[b], (u - 1) & 1) && uwait_cluster(&x_empty[b], (u - 1) & 1))) {
+                    ok = false;
+                    break;
+                }
+                uint4* row = (uint4*)(xstage + b * kXBytes + h * kXRowBytes);
 #pragma unroll
-                    for (int i = 0; i < kT; i += 4)
-                        st_cluster_v4(dst + 4 * i, __float_as_uint(s[i]), __float_as_uint(s[i + 1]),
-                                      __float_as_uint(s[i + 2]), __float_as_uint(s[i + 3]));
-                    ptx::mbar_arrive_cluster(&x_full[par], peer);
-                    // receive its probabilities
-                    if (!uwait_cluster(&p_full[par], use & 1)) { ok = false; break; }
-                    const uint4* src = (const uint4*)(pbuf + par * kPBytes + hl * kPRow);
+                for (int v = 0; v < 8; ++v)
+                    row[v ^ (h & 7)] = make_uint4(own[4 * v], own[4 * v + 1], own[4 * v + 2], own[4 * v + 3]);
+                ptx::fence_proxy_async_smem();   // the copy engine reads what this thread wrote
+                ptx::mbar_arrive(&xs_ready[b]);
+                if (h == 0) {
+                    if (!ptx::mbar_wait(&xs_ready[b], u & 1, abort_flag)) {
+                        fail(err_code, err_detail, abort_flag, 5);
+                    } else {
+                        ptx::bulk_copy_to_peer(mapa(ptx::smem_u32(xbuf + b * kXBytes), peer), xstage + b * kXBytes,
+                                               kXBytes, mapa(ptx::smem_u32(&x_full[b]), peer));
+                    }
+                }
+                ++g;
+                if (++j == cur.j1) {
+                    have = it.next(cur);
+                    if (have) {
+                        j = cur.j0;
+                        load_q(cur.b);   // the S of this piece's last tile is already read
+                    }
+                }
+            }
+        } else {
+            // ----------------------------------------------------- softmax / epilogue
+            float m_run = -INFINITY, l_run = 0.f;
+            while (have) {
+                const uint32_t b = g & 1, u = g >> 1;
+                if (h == 0) ptx::mbar_expect_tx(&x_full[b], kXBytes);
+                if (!uwait(&xs_ready[b], u & 1)) { ok = false; break; }
+                if (!uwait_cluster(&x_full[b], u & 1)) { ok = false; break; }
+                // full scores = own + peer partial, both bf16-valued (identical in both CTAs)
+                float s[kT];
+                {
+                    const uint4* mine = (const uint4*)(xstage + b * kXBytes + h * kXRowBytes);
+                    const uint4* theirs = (const uint4*)(xbuf + b * kXBytes + h * kXRowBytes);
 #pragma unroll
                     for (int v = 0; v < 8; ++v) {
-                        const uint4 x = src[v];
-                        pw[4 * v] = x.x; pw[4 * v + 1] = x.y; pw[4 * v + 2] = x.z; pw[4 * v + 3] = x.w;
-                    }
-                    alpha = __uint_as_float(src[8].x);
-                    ptx::mbar_arrive_cluster(&p_empty[par], peer);
-                } else {
-                    if (!uwait_cluster(&x_full[par], use & 1)) { ok = false; break; }
-                    const float4* src = (const float4*)(xbuf + par * (kXBytes / 4) + hl * kXStride);
+                        const uint4 x = mine[v ^ (h & 7)], y = theirs[v ^ (h & 7)];
+                        const uint32_t a4[4] = {x.x, x.y, x.z, x.w};
+                        const uint32_t b4[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
-                    for (int i = 0; i < kT / 4; ++i) {
-                        const float4 x = src[i];
-                        s[4 * i] += x.x; s[4 * i + 1] += x.y; s[4 * i + 2] += x.z; s[4 * i + 3] += x.w;
+                        for (int q = 0; q < 4; ++q) {
+                            s[8 * v + 2 * q] = __uint_as_float(a4[q] << 16) + __uint_as_float(b4[q] << 16);
+                            s[8 * v + 2 * q + 1] =
+                                __uint_as_float(a4[q] & 0xFFFF0000u) + __uint_as_float(b4[q] & 0xFFFF0000u);
+                        }
                     }
-                    ptx::mbar_arrive_cluster(&x_empty[par], peer);
-                    // online softmax in base 2 over this tile's valid tokens
-                    const int valid = min(kT, sg.L - j * kT);
-                    float mt = -INFINITY;
-#pragma unroll
-                    for (int i = 0; i < kT; ++i) {
-                        s[i] = i < valid ? s[i] * scale_log2 : -INFINITY;
-                        mt = fmaxf(mt, s[i]);
-                    }
-                    alpha = 1.f;
-                    if (mt > m_run + kRescaleThreshold) {
-                        alpha = exp2f(m_run - mt);
-                        m_run = mt;
-                    }
-                    float sum = 0.f;
-#pragma unroll
-                    for (int i = 0; i < kT; i += 2) {
-                        const float p0 = exp2f(s[i] - m_run), p1 = exp2f(s[i + 1] - m_run);
-                        sum += p0 + p1;
-                        pw[i / 2] = ptx::pack_bf16(p0, p1);
-                    }
-                    l_run = l_run * alpha + sum;
-                    // send P and alpha to the peer, which holds the other half of O for this head
-                    if (g >= 2 && !uwait_cluster(&p_empty[par], (use - 1) & 1)) { ok = false; break; }
-                    const uint32_t dst = mapa(prow_local + par * kPBytes, peer);
-#pragma unroll
-                    for (int v = 0; v < 8; ++v) st_cluster_v4(dst + 16 * v, pw[4 * v], pw[4 * v + 1], pw[4 * v + 2], pw[4 * v + 3]);
-                    st_cluster_v4(dst + 128, __float_as_uint(alpha), 0u, 0u, 0u);
-                    ptx::mbar_arrive_cluster(&p_full[par], peer);
+                    // both buffers are consumed: the staging one may be refilled (after the
+                    // copy finished), the peer may copy its next tile into ours
+                    ptx::mbar_arrive(&xs_free[b]);
+                    __syncwarp();
+                    if (lane == 31) ptx::mbar_arrive_cluster_relaxed(&x_empty[b], peer);
                 }
+                // online softmax in base 2 over this tile's valid tokens
+                const bool first = (j == cur.j0);
+                if (first) {
+                    m_run = -INFINITY;
+                    l_run = 0.f;
+                }
+                const int valid = min(kT, cur.L - j * kT);
+                float mt = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < kT; ++i) {
+                    s[i] = i < valid ? s[i] : -INFINITY;
+                    mt = fmaxf(mt, s[i]);
+                }
+                float alpha = 1.f;
+                if (mt > m_run + kRescaleThreshold) {
+                    alpha = ex2_ftz(m_run - mt);
+                    m_run = mt;
+                }
+                uint32_t pw[32];
+                float sum = 0.f;
+#pragma unroll
+                for (int i = 0; i < kT; i += 2) {
+                    const float p0 = ex2_ftz(s[i] - m_run), p1 = ex2_ftz(s[i + 1] - m_run);
+                    sum += p0 + p1;
+                    pw[i / 2] = ptx::pack_bf16(p0, p1);
+                }
+                l_run = l_run * alpha + sum;
                 // P (TMEM) and O are free once the previous tile's O MMA has completed
                 if (g > 0 && !uwait(o_done, (g - 1) & 1)) { ok = false; break; }
                 ptx::tc_fence_after();
-                if (__any_sync(0xffffffffu, j > sg.j0 && alpha != 1.f)) {
-                    const float a = j > sg.j0 ? alpha : 1.f;
+                if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
+                    const float a = first ? 1.f : alpha;
 #pragma unroll 1
                     for (int c0 = 0; c0 < 256; c0 += 32) {
                         uint32_t r[32];
@@ -437,26 +557,31 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_ready);
-            }
-            if (!ok) break;
-            // piece epilogue: un-normalised O_r -> part_o[slot][c][h], (m, l) by the owner
-            if (!uwait(o_done, (g - 1) & 1)) { ok = false; break; }
-            ptx::tc_fence_after();
-            float* po = part_o + (long long)sg.slot * 512 * 128 + (long long)(256 * rank) * 128 + h;
+                if (j + 1 == cur.j1) {
+                    // piece epilogue: un-normalised O_r -> part_o[slot][c][h]; (m, l) from CTA 0
+                    if (!uwait(o_done, g & 1)) { ok = false; break; }
+                    ptx::tc_fence_after();
+                    float* po = part_o + (long long)cur.slot * 512 * 128 + (long long)(256 * rank) * 128 + h;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
-                uint32_t r[32];
-                ptx::tmem_ld32(lane_addr + kColO + c0, r);
-                ptx::tmem_wait_ld();
+                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(lane_addr + kColO + c0, r);
+                        ptx::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) po[(long long)(c0 + i) * 128] = __uint_as_float(r[i]);
+                        for (int i = 0; i < 32; ++i) po[(long long)(c0 + i) * 128] = __uint_as_float(r[i]);
+                    }
+                    if (rank == 0) {
+                        part_ml[((long long)cur.slot * 128 + h) * 2] = m_run;
+                        part_ml[((long long)cur.slot * 128 + h) * 2 + 1] = l_run;
+                    }
+                    ptx::tc_fence_before();
+                }
+                ++g;
+                if (++j == cur.j1) {
+                    have = it.next(cur);
+                    j = have ? cur.j0 : 0;
+                }
             }
-            if (owner) {
-                part_ml[((long long)sg.slot * 128 + h) * 2] = m_run;
-                part_ml[((long long)sg.slot * 128 + h) * 2 + 1] = l_run;
-            }
-            ptx::tc_fence_before();
-            ++sidx;
         }
         if (!ok) fail(err_code, err_detail, abort_flag, 3);
     }
@@ -515,7 +640,7 @@ int max_clusters(int num_sms) {
     cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-    cfg.blockDim = dim3(192, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = kSmem;
     int n = 0;
     if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
@@ -569,7 +694,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     const int P = max_clusters(num_sms);
     {
         ProfScope ps(s, "tc_plan");
-        plan_kernel<<<1, 32, 0, s>>>(offsets, B, P, ws.work, err_code, err_detail);
+        plan_kernel<<<1, 256, 0, s>>>(offsets, B, P, ws.work, err_code, err_detail);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     {
@@ -587,7 +712,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         const uint32_t box[2] = {64, (uint32_t)kT};
         if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
         cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        decode_tc_kernel<<<2 * P, 192, kSmem, s>>>(m, ws.q_lat, qr, sQr_b, sQr_h, offsets, B, cache_rows, ws.work,
+        decode_tc_kernel<<<2 * P, kThreads, kSmem, s>>>(m, ws.q_lat, qr, sQr_b, sQr_h, offsets, B, cache_rows, ws.work,
                                                     scale * 1.4426950408889634f, ws.part_o, ws.part_ml, err_code,
                                                     err_detail);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;

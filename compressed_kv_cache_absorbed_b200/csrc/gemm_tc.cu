@@ -22,9 +22,9 @@ struct GemmCfg {
     static constexpr int A_BYTES = kBM * kBK * 2;
     static constexpr int B_BYTES = BN * kBK * 2;
     static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int STAGES = (196608 / STAGE) > 8 ? 8 : (196608 / STAGE);
+    static constexpr int MAX_STAGES = (196608 / STAGE) > 8 ? 8 : (196608 / STAGE);
     static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
-    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
+    static constexpr int smem(int stages) { return stages * STAGE + 1024 + 256; }
 };
 
 __device__ __forceinline__ void fail(int* code, long long* detail, volatile int* abort_flag, int where) {
@@ -35,13 +35,13 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                    int N, int K, GemmOut out, int* err_code, long long* err_detail) {
+                    int N, int K, int stages, GemmOut out, int* err_code, long long* err_detail) {
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
-    uint64_t* full = (uint64_t*)(smem + C::STAGES * C::STAGE);
-    uint64_t* empty = full + C::STAGES;
-    uint64_t* accum = empty + C::STAGES;
+    uint64_t* full = (uint64_t*)(smem + stages * C::STAGE);
+    uint64_t* empty = full + stages;
+    uint64_t* accum = empty + stages;
     uint32_t* tmem_slot = (uint32_t*)(accum + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
@@ -50,7 +50,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     const int nk = (K + kBK - 1) / kBK;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < C::STAGES; ++s) {
+        for (int s = 0; s < stages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
@@ -72,9 +72,9 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             ptx::tma_prefetch(&tmA);
             ptx::tma_prefetch(&tmB);
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % C::STAGES;
-                const uint32_t ph = (kb / C::STAGES) & 1;
-                if (kb >= C::STAGES && !ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+                const int s = kb % stages;
+                const uint32_t ph = (kb / stages) & 1;
+                if (kb >= stages && !ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
                     fail(err_code, err_detail, abort_flag, 1);
                     break;
                 }
@@ -88,8 +88,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN, 0, 0);
             for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % C::STAGES;
-                const uint32_t ph = (kb / C::STAGES) & 1;
+                const int s = kb % stages;
+                const uint32_t ph = (kb / stages) & 1;
                 if (!ptx::mbar_wait(&full[s], ph, abort_flag)) {
                     fail(err_code, err_detail, abort_flag, 2);
                     break;
@@ -145,11 +145,17 @@ template <int BN>
 cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUtensorMap& mb, const GemmOut& out,
                    int* err_code, long long* err_detail, cudaStream_t s) {
     using C = GemmCfg<BN>;
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         C::SMEM);
-    if (e != cudaSuccess) return e;
+    static bool attr_set = false;   // the attribute is per function; set it once
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             C::smem(C::MAX_STAGES));
+        if (e != cudaSuccess) return e;
+        attr_set = true;
+    }
+    const int nk = (K + kBK - 1) / kBK;
+    const int stages = nk < C::MAX_STAGES ? (nk < 2 ? 2 : nk) : C::MAX_STAGES;
     dim3 grid((N + BN - 1) / BN, (M + kBM - 1) / kBM, Z);
-    gemm_bf16_tc_kernel<BN><<<grid, 192, C::SMEM, s>>>(ma, mb, M, N, K, out, err_code, err_detail);
+    gemm_bf16_tc_kernel<BN><<<grid, 192, C::smem(stages), s>>>(ma, mb, M, N, K, stages, out, err_code, err_detail);
     return cudaGetLastError();
 }
 

@@ -328,3 +328,38 @@ def test_prefill_full_size_sampled():
         assert_close(out[b, t_list, h], res[h], "bf16", f"prefill full h={h}")
     frac = check_rows(cache[b * w.ctx:(b + 1) * w.ctx], rows, "bf16", "prefill cache rows")
     assert frac >= CACHE_EXACT_FRAC
+
+
+# ------------------------------------------------ split-KV scheduling edge cases
+
+def test_decode_path_is_tensor_core_for_the_v3_head_shape():
+    w = workloads.WORKLOADS["v3_decode_b32_ctx4096"]
+    assert mla.mla_decode_path(dims_of(w)) == 1
+
+
+@pytest.mark.parametrize("lengths", [
+    [20000],                                   # one sequence split across every cluster
+    [1] * 200 + [20000] + [63, 64, 65],        # B > 256 rows of the planner, many pieces per range
+    [129, 191, 192, 193, 4095, 1, 2, 3],       # tile-boundary lengths
+])
+def test_decode_split_schedules(lengths):
+    w, inp = reduced_attn_inputs(lengths, seed=31)
+    out = run_decode_attn(w, inp)
+    r = np.random.default_rng(4)
+    units = sorted({(int(r.integers(w.B)), int(r.integers(w.H))) for _ in range(48)} |
+                   {(int(np.argmax(lengths)), 0), (int(np.argmax(lengths)), w.H - 1), (w.B - 1, 5)})
+    want = oracle_decode_units(w, inp, units)
+    assert_close(torch.stack([out[b, h] for b, h in units]), want, "bf16", f"schedule {len(lengths)} seqs")
+
+
+def test_decode_invariant_to_cache_row_order():
+    """Attention over a sequence is a function of its set of (already rotated) rows."""
+    lengths = [700, 1300, 65]
+    w, inp = reduced_attn_inputs(lengths, seed=41)
+    out1 = run_decode_attn(w, inp)
+    offs = inp["offsets"].numpy()
+    perm = np.concatenate([offs[b] + np.random.default_rng(b).permutation(lengths[b]) for b in range(len(lengths))])
+    inp2 = dict(inp)
+    inp2["cache"] = inp["cache"][torch.from_numpy(perm)].contiguous()
+    out2 = run_decode_attn(w, inp2)
+    assert_close(out2, out1.double(), "bf16", "row permutation")
