@@ -37,6 +37,29 @@ constexpr int kErrTimeout = 5;
 
 // ---------------------------------------------------------------- launch helpers
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start while the
+// previous kernel in the stream is still running; it must call pdl_wait() before touching
+// anything that kernel (or any earlier one) writes or reads.  pdl_trigger() lets the next
+// kernel start its own independent prologue.  Both are no-ops without the launch attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // per-kernel event timing (profile.cu); no-ops unless mla_profile_enable(1)
 void prof_begin(cudaStream_t s, const char* name);
 void prof_end(cudaStream_t s);

@@ -48,16 +48,20 @@ namespace {
 
 constexpr int kT = 64;                        // tokens per tile
 constexpr int kStages = 4;
+constexpr int kL2Ahead = 6;                   // tiles pulled into L2 ahead of the ring
 constexpr int kChunkBytes = kT * 128;         // one 64-column box of a tile
 constexpr int kTileBytes = 5 * kChunkBytes;   // 4 latent chunks + the rotary chunk
 constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
 constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
-constexpr int kBarBytes = 256;
+constexpr int kBarBytes = 256 + 2048;
 // tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer)
-constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kBarBytes + 1024;
+// The dynamic shared memory of a kernel without static shared memory starts 1024-byte
+// aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
+constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kBarBytes;
+static_assert(kSmem <= 232448, "decode kernel shared memory over the 227 KB limit");
 constexpr uint32_t kColQ = 0, kColS = 160, kColP = 224, kColO = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-constexpr int kThreads = 320;                 // producer, MMA, 4 sender and 4 softmax warps
+constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 softmax warps
 
 // plan layout (int32): [0] total tiles, [1] tiles per cluster, [2] clusters,
 // [4, 4+B+1) first tile of each sequence, [4+B+1, 4+2B+2) first partial slot of each sequence
@@ -101,6 +105,8 @@ plan_kernel(const int32_t* __restrict__ offsets, int B, int P, int32_t* __restri
     __shared__ int s_wp[8];
     __shared__ int s_ptot;
     const int t = threadIdx.x;
+    if (t == 0) pdl_trigger();
+    pdl_wait();
     const int per_thread = (B + 255) / 256;
     const int b0 = min(B, t * per_thread), b1 = min(B, b0 + per_thread);
     auto tiles_of = [&](int b) -> long long {
@@ -164,15 +170,6 @@ __device__ __forceinline__ uint32_t mapa(uint32_t saddr, uint32_t rank) {
     return r;
 }
 
-// Two floats rounded to bf16 (nearest even) with integer operations and packed into one
-// word (first value in the low half).  Both CTAs of a pair round their own partial scores
-// with this, so the sums they form are identical.
-__device__ __forceinline__ uint32_t bf16_pair_rne(float a, float b) {
-    const uint32_t ua = __float_as_uint(a), ub = __float_as_uint(b);
-    const uint32_t ra = ua + 0x7FFFu + ((ua >> 16) & 1u);
-    const uint32_t rb = ub + 0x7FFFu + ((ub >> 16) & 1u);
-    return __byte_perm(ra, rb, 0x7632);
-}
 // 2^x with the hardware approximation (inputs here are <= 8; results below 2^-126 flush to 0)
 __device__ __forceinline__ float ex2_ftz(float x) {
     float y;
@@ -219,8 +216,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
                  const int32_t* __restrict__ work, float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, int* err_code, long long* err_detail) {
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    if (ptx::smem_u32(smem_raw) & 1023) {   // uniform across the CTA: leave before any sync
+        if (threadIdx.x == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 7000000);
+        return;
+    }
+    uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
     uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
     uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
@@ -241,7 +242,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     uint64_t* drain = s_full + 9;    // all MMAs issued by this CTA have completed
     uint64_t* xs_ready = s_full + 10;  // [2] all 128 rows of xstage[g & 1] written
     uint64_t* xs_free = s_full + 12;   // [2] the local softmax has read xstage[g & 1]
-    uint32_t* tmem_slot = (uint32_t*)(s_full + 14);
+    uint64_t* pair_bar = s_full + 14;  // [4] the two softmax warps of a subpartition
+    float* pair_val = (float*)(s_full + 18);   // [2][2][128] values the two warps swap
+    uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
     const uint32_t rank = cluster_rank(), peer = rank ^ 1;
@@ -255,15 +258,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         }
         ptx::mbar_init(s_full, 1);
         ptx::mbar_init(s_free, 128);
-        ptx::mbar_init(p_ready, 128);
+        ptx::mbar_init(p_ready, 256);
+        for (int i = 0; i < 4; ++i) ptx::mbar_init(&pair_bar[i], 64);
         ptx::mbar_init(o_done, 1);
         ptx::mbar_init(q_ready, 128);
         ptx::mbar_init(drain, 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&x_full[i], 1);
-            ptx::mbar_init(&x_empty[i], 4);
+            ptx::mbar_init(&x_empty[i], 8);
             ptx::mbar_init(&xs_ready[i], 128);
-            ptx::mbar_init(&xs_free[i], 128);
+            ptx::mbar_init(&xs_free[i], 256);
         }
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -277,6 +281,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     cluster_sync_all();  // the peer's barriers exist before anyone arrives on them remotely
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) pdl_trigger();
+    pdl_wait();   // everything below reads the plan, the queries and the cache
 
     const int per = work[1];
     const int total = work[0];
@@ -289,6 +295,24 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         if (lane == 0) {
             ptx::tma_prefetch(&tm_cache);
             uint32_t g = 0;
+            // a second cursor kL2Ahead tiles ahead pulls tiles into L2, so that the ring's
+            // loads (which wait for free stages) find them there
+            SegIter itp = it;
+            Seg sp;
+            bool p_have = itp.next(sp);
+            int p_j = p_have ? sp.j0 : 0;
+            auto prefetch_next = [&]() {
+                if (!p_have) return;
+                const int row = (int)(sp.row0 + (long long)p_j * kT);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) ptx::tma_prefetch_l2_2d(&tm_cache, 256 * (int)rank + 64 * i, row);
+                ptx::tma_prefetch_l2_2d(&tm_cache, 512, row);
+                if (++p_j == sp.j1) {
+                    p_have = itp.next(sp);
+                    p_j = p_have ? sp.j0 : 0;
+                }
+            };
+            for (int k = 0; k < kL2Ahead; ++k) prefetch_next();
             while (!*abort_flag && it.next(sg)) {
                 if (sg.row0 + (long long)sg.L > cache_rows) {   // sequence beyond the cache
                     latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
@@ -302,6 +326,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                         fail(err_code, err_detail, abort_flag, 1);
                         break;
                     }
+                    prefetch_next();
                     uint8_t* dst = tiles + s * kTileBytes;
                     const int row = (int)(sg.row0 + (long long)j * kT);
                     ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
@@ -324,61 +349,75 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 256, 0, 1);
             uint32_t g = 0, sidx = 0;
             bool ok = true;
-            auto issue_o = [&](uint32_t gt, bool first) -> bool {
-                if (!ptx::mbar_wait(p_ready, gt & 1, abort_flag)) return false;
-                ptx::tc_fence_after();
-                const uint32_t v = ptx::smem_u32(tiles + (gt % kStages) * kTileBytes);
-#pragma unroll
-                for (int k = 0; k < kT / 16; ++k)
-                    ptx::mma_ts(tmem + kColO, tmem + kColP + 8 * k, ptx::desc_mnmajor_sw128(v + 2048 * k, kChunkBytes),
-                                idesc_o, !(first && k == 0));
-                ptx::mma_commit(o_done);
-                ptx::mma_commit(&tile_empty[gt % kStages]);
-                return true;
-            };
-            // S runs two tiles ahead of O: S of tile t+2 needs only that the softmax warps
-            // have read S of tile t+1 (they do so while finishing tile t), while O of tile t
-            // needs P of tile t.  The tile order is one flat pass over all pieces.
-            SegIter its = it;   // second iterator: tiles whose S is issued next
+            // Event-driven issue: O of the oldest tile as soon as its P is in TMEM (it frees the
+            // P columns for the next tile and the tile's shared-memory stage), otherwise S of
+            // the next tile as soon as that tile has landed and the S columns are free.  S may
+            // run ahead of O by as many tiles as the ring holds.  Tiles are taken in one flat
+            // pass over all pieces (two iterators: one for S, one for O).
+            SegIter its = it;
             Seg ss;
             bool s_have = !*abort_flag && its.next(ss);
             int s_j = s_have ? ss.j0 : 0;
+            bool q_ok = false;
             uint32_t s_g = 0;
-            auto issue_s = [&]() -> bool {   // S of tile s_g (= s_j of piece ss), then advance
-                if (s_j == ss.j0 && !ptx::mbar_wait(q_ready, (sidx++) & 1, abort_flag)) return false;
-                const int st = s_g % kStages;
-                if (!ptx::mbar_wait(&tile_full[st], (s_g / kStages) & 1, abort_flag)) return false;
-                if (s_g > 0 && !ptx::mbar_wait(s_free, (s_g - 1) & 1, abort_flag)) return false;
-                ptx::tc_fence_after();
-                const uint32_t t = ptx::smem_u32(tiles + st * kTileBytes);
+            bool o_have = !*abort_flag && it.next(sg);
+            int o_j = o_have ? sg.j0 : 0;
+            uint32_t idle = 0;
+            while (o_have) {
+                // ---- O of tile g
+                if (g < s_g && ptx::mbar_test(p_ready, g & 1)) {
+                    ptx::tc_fence_after();
+                    const uint32_t v = ptx::smem_u32(tiles + (g % kStages) * kTileBytes);
+                    const bool first = (o_j == sg.j0);
 #pragma unroll
-                for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
-                    ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
-                                ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
-                                ks != 0);
-#pragma unroll
-                for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
-                    ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
-                                ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
-                ptx::mma_commit(s_full);
-                ++s_g;
-                if (++s_j == ss.j1) {
-                    s_have = !*abort_flag && its.next(ss);
-                    s_j = s_have ? ss.j0 : 0;
+                    for (int k = 0; k < kT / 16; ++k)
+                        ptx::mma_ts(tmem + kColO, tmem + kColP + 8 * k,
+                                    ptx::desc_mnmajor_sw128(v + 2048 * k, kChunkBytes), idesc_o, !(first && k == 0));
+                    ptx::mma_commit(o_done);
+                    ptx::mma_commit(&tile_empty[g % kStages]);
+                    ++g;
+                    if (++o_j == sg.j1) {
+                        o_have = it.next(sg);
+                        o_j = o_have ? sg.j0 : 0;
+                    }
+                    idle = 0;
+                    continue;
                 }
-                return true;
-            };
-            // O follows the same flat order with the primary iterator
-            bool have = !*abort_flag && it.next(sg);
-            int j = have ? sg.j0 : 0;
-            for (int k = 0; k < 2 && ok && s_have; ++k) ok = issue_s();
-            while (ok && have) {
-                if (s_have && !issue_s()) { ok = false; break; }
-                if (!issue_o(g, j == sg.j0)) { ok = false; break; }
-                ++g;
-                if (++j == sg.j1) {
-                    have = !*abort_flag && it.next(sg);
-                    j = have ? sg.j0 : 0;
+                // ---- S of tile s_g
+                if (s_have) {
+                    const bool first = (s_j == ss.j0);
+                    if (first && !q_ok && ptx::mbar_test(q_ready, sidx & 1)) {
+                        q_ok = true;
+                        ++sidx;
+                    }
+                    const int st = s_g % kStages;
+                    if ((!first || q_ok) && ptx::mbar_test(&tile_full[st], (s_g / kStages) & 1) &&
+                        (s_g == 0 || ptx::mbar_test(s_free, (s_g - 1) & 1))) {
+                        ptx::tc_fence_after();
+                        const uint32_t t = ptx::smem_u32(tiles + st * kTileBytes);
+#pragma unroll
+                        for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
+                            ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
+                                        ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
+                                        ks != 0);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
+                            ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
+                                        ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
+                        ptx::mma_commit(s_full);
+                        ++s_g;
+                        q_ok = false;
+                        if (++s_j == ss.j1) {
+                            s_have = its.next(ss);
+                            s_j = s_have ? ss.j0 : 0;
+                        }
+                        idle = 0;
+                        continue;
+                    }
+                }
+                if (++idle > (ptx::kWaitLimit << 4) || *abort_flag) {
+                    ok = false;
+                    break;
                 }
             }
             if (!ok) fail(err_code, err_detail, abort_flag, 2);
@@ -387,7 +426,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             if (!ptx::mbar_wait(drain, 0, nullptr)) fail(err_code, err_detail, abort_flag, 4);
         }
     } else {
-        // warps 2-5 send partial scores, warps 6-9 run the softmax; warp w works on TMEM
+        // warps 2-5 send partial scores, warps 6-13 run the softmax; warp w works on TMEM
         // lanes 32 * (w % 4) .. +31, so thread h of either role owns head h
         const int sub = warp & 3;
         const int h = sub * 32 + lane;
@@ -437,7 +476,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             if (have) load_q(cur.b);
             while (have) {
                 const uint32_t b = g & 1, u = g >> 1;
-                // partial scores: TMEM -> registers (log2 units, bf16 pairs)
+                // partial scores: TMEM -> registers -> bf16 pairs
                 if (!uwait(s_full, g & 1)) { ok = false; break; }
                 ptx::tc_fence_after();
                 uint32_t own[32];
@@ -448,8 +487,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                     ptx::tmem_ld32x2_second(lane_addr + kColS + 32, sc, r);
                     ptx::tc_fence_before();
                     ptx::mbar_arrive(s_free);
+                    // raw partial scores rounded to bf16 pairs (nearest even, in hardware);
+                    // both CTAs add the same two rounded partials
 #pragma unroll
-                    for (int i = 0; i < kT; i += 2) own[i / 2] = bf16_pair_rne(sc[i] * scale_log2, sc[i + 1] * scale_log2);
+                    for (int i = 0; i < kT; i += 2) own[i / 2] = ptx::pack_bf16(sc[i], sc[i + 1]);
                 }
                 // staging buffer b is free once the local softmax read it (tile g-2) and the
                 // peer read the copy made from it
@@ -482,58 +523,76 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             }
         } else {
             // ----------------------------------------------------- softmax / epilogue
-            float m_run = -INFINITY, l_run = 0.f;
+            // two warps per TMEM subpartition: `half` 0 takes tokens 0-31 of a tile, half 1
+            // tokens 32-63, of the same 32 heads; they agree on the running max through
+            // shared memory, so the P halves they write share one scale per head
+            const int half = warp >= 10 ? 1 : 0;
+            float m_run = -INFINITY, l_run = 0.f;   // l_run: this half's share of the row sum
+            uint32_t pairs = 0;                     // uses of this pair's barrier
+            auto pair_exchange = [&](float v) -> float {   // the partner warp's value for head h
+                pair_val[(pairs & 1) * 256 + half * 128 + h] = v;
+                ptx::mbar_arrive(&pair_bar[sub]);
+                if (!uwait(&pair_bar[sub], pairs & 1)) ok = false;
+                const float o = pair_val[(pairs & 1) * 256 + (half ^ 1) * 128 + h];
+                ++pairs;
+                return o;
+            };
             while (have) {
                 const uint32_t b = g & 1, u = g >> 1;
-                if (h == 0) ptx::mbar_expect_tx(&x_full[b], kXBytes);
+                if (h == 0 && half == 0) ptx::mbar_expect_tx(&x_full[b], kXBytes);
                 if (!uwait(&xs_ready[b], u & 1)) { ok = false; break; }
                 if (!uwait_cluster(&x_full[b], u & 1)) { ok = false; break; }
-                // full scores = own + peer partial, both bf16-valued (identical in both CTAs)
-                float s[kT];
+                // full scores of this half = own + peer partial, both bf16-valued
+                float s[kT / 2];
                 {
                     const uint4* mine = (const uint4*)(xstage + b * kXBytes + h * kXRowBytes);
                     const uint4* theirs = (const uint4*)(xbuf + b * kXBytes + h * kXRowBytes);
 #pragma unroll
-                    for (int v = 0; v < 8; ++v) {
+                    for (int vv = 0; vv < 4; ++vv) {
+                        const int v = 4 * half + vv;
                         const uint4 x = mine[v ^ (h & 7)], y = theirs[v ^ (h & 7)];
                         const uint32_t a4[4] = {x.x, x.y, x.z, x.w};
                         const uint32_t b4[4] = {y.x, y.y, y.z, y.w};
 #pragma unroll
                         for (int q = 0; q < 4; ++q) {
-                            s[8 * v + 2 * q] = __uint_as_float(a4[q] << 16) + __uint_as_float(b4[q] << 16);
-                            s[8 * v + 2 * q + 1] =
+                            s[8 * vv + 2 * q] = __uint_as_float(a4[q] << 16) + __uint_as_float(b4[q] << 16);
+                            s[8 * vv + 2 * q + 1] =
                                 __uint_as_float(a4[q] & 0xFFFF0000u) + __uint_as_float(b4[q] & 0xFFFF0000u);
                         }
                     }
-                    // both buffers are consumed: the staging one may be refilled (after the
-                    // copy finished), the peer may copy its next tile into ours
                     ptx::mbar_arrive(&xs_free[b]);
                     __syncwarp();
                     if (lane == 31) ptx::mbar_arrive_cluster_relaxed(&x_empty[b], peer);
                 }
-                // online softmax in base 2 over this tile's valid tokens
                 const bool first = (j == cur.j0);
                 if (first) {
                     m_run = -INFINITY;
                     l_run = 0.f;
                 }
-                const int valid = min(kT, cur.L - j * kT);
+                // scores are raw dot products here; scale_log2 (softmax scale x log2 e) turns
+                // them into base-2 exponents inside one FFMA per probability
+                const int valid = min(kT, cur.L - j * kT) - half * (kT / 2);
+                if (valid < kT / 2) {   // only a piece's last tile is partial
+#pragma unroll
+                    for (int i = 0; i < kT / 2; ++i) s[i] = i < valid ? s[i] : -INFINITY;
+                }
                 float mt = -INFINITY;
 #pragma unroll
-                for (int i = 0; i < kT; ++i) {
-                    s[i] = i < valid ? s[i] : -INFINITY;
-                    mt = fmaxf(mt, s[i]);
-                }
+                for (int i = 0; i < kT / 2; ++i) mt = fmaxf(mt, s[i]);
+                mt = fmaxf(mt, pair_exchange(mt));   // tile max over all 64 tokens
+                if (!ok) break;
                 float alpha = 1.f;
-                if (mt > m_run + kRescaleThreshold) {
-                    alpha = ex2_ftz(m_run - mt);
-                    m_run = mt;
+                if (mt * scale_log2 > m_run + kRescaleThreshold) {   // m_run in base-2 units
+                    const float m_new = mt * scale_log2;
+                    alpha = ex2_ftz(m_run - m_new);
+                    m_run = m_new;
                 }
-                uint32_t pw[32];
+                uint32_t pw[kT / 4];
                 float sum = 0.f;
 #pragma unroll
-                for (int i = 0; i < kT; i += 2) {
-                    const float p0 = ex2_ftz(s[i] - m_run), p1 = ex2_ftz(s[i + 1] - m_run);
+                for (int i = 0; i < kT / 2; i += 2) {
+                    const float p0 = ex2_ftz(fmaf(s[i], scale_log2, -m_run));
+                    const float p1 = ex2_ftz(fmaf(s[i + 1], scale_log2, -m_run));
                     sum += p0 + p1;
                     pw[i / 2] = ptx::pack_bf16(p0, p1);
                 }
@@ -544,7 +603,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
                     const float a = first ? 1.f : alpha;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                    for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
                         uint32_t r[32];
                         ptx::tmem_ld32(lane_addr + kColO + c0, r);
                         ptx::tmem_wait_ld();
@@ -553,26 +612,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                         ptx::tmem_st32(lane_addr + kColO + c0, r);
                     }
                 }
-                ptx::tmem_st32(lane_addr + kColP, pw);
+                ptx::tmem_st16(lane_addr + kColP + 16 * half, pw);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_ready);
                 if (j + 1 == cur.j1) {
-                    // piece epilogue: un-normalised O_r -> part_o[slot][c][h]; (m, l) from CTA 0
+                    // piece epilogue: un-normalised O_r -> part_o[slot][c][h] (each half
+                    // writes 128 columns); (m, l) from CTA 0
+                    const float l_all = l_run + pair_exchange(l_run);
+                    if (!ok) break;
                     if (!uwait(o_done, g & 1)) { ok = false; break; }
                     ptx::tc_fence_after();
                     float* po = part_o + (long long)cur.slot * 512 * 128 + (long long)(256 * rank) * 128 + h;
 #pragma unroll 1
-                    for (int c0 = 0; c0 < 256; c0 += 32) {
+                    for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
                         uint32_t r[32];
                         ptx::tmem_ld32(lane_addr + kColO + c0, r);
                         ptx::tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < 32; ++i) po[(long long)(c0 + i) * 128] = __uint_as_float(r[i]);
                     }
-                    if (rank == 0) {
+                    if (rank == 0 && half == 0) {
                         part_ml[((long long)cur.slot * 128 + h) * 2] = m_run;
-                        part_ml[((long long)cur.slot * 128 + h) * 2 + 1] = l_run;
+                        part_ml[((long long)cur.slot * 128 + h) * 2 + 1] = l_all;
                     }
                     ptx::tc_fence_before();
                 }
@@ -593,44 +655,65 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
 
 // ------------------------------------------------------------------- merge
 // o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[c,h] / sum_p 2^(m_p - M) l_p  over the pieces p of b.
-__global__ void __launch_bounds__(256)
+// Block = (sequence b, 32 latent columns), thread = head.  The (m, l) of up to kMergeBatch
+// pieces are fetched together and every piece's 32 partial values are loaded before they
+// are used, so the block waits on memory once per batch rather than once per value.
+constexpr int kMergeBatch = 8;
+
+__global__ void __launch_bounds__(128)
 combine_tc_kernel(const int32_t* __restrict__ work, int B, const float* __restrict__ part_o,
                   const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o_lat) {
-    const int b = blockIdx.x, cb = blockIdx.y;   // 64 latent columns per block
-    const int h = threadIdx.x & 127, half = threadIdx.x >> 7;
+    const int b = blockIdx.x, c0 = blockIdx.y * 32, h = threadIdx.x;
+    if (threadIdx.x == 0) pdl_trigger();
+    pdl_wait();
     const int32_t* ts = plan_tstart(work);
     const int32_t* sb = plan_sbase(work, B);
     const int per = work[1];
-    const int t0 = ts[b], t1 = ts[b + 1];
-    __nv_bfloat16* dst = o_lat + ((long long)b * 128 + h) * 512 + cb * 64 + half * 32;
+    const int t0 = ts[b], t1 = ts[b + 1], base = sb[b];
+    uint4* dst = (uint4*)(o_lat + ((long long)b * 128 + h) * 512 + c0);
     if (t1 == t0) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) dst[i] = __float2bfloat16_rn(0.f);
+        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
         return;
     }
     const int np = (t1 - 1) / per - t0 / per + 1;
-    const int base = sb[b];
-    float M = -INFINITY;
-    for (int p = 0; p < np; ++p) M = fmaxf(M, part_ml[((long long)(base + p) * 128 + h) * 2]);
-    float L = 0.f;
-    for (int p = 0; p < np; ++p) {
-        const long long q = ((long long)(base + p) * 128 + h) * 2;
-        L += exp2f(part_ml[q] - M) * part_ml[q + 1];
-    }
-    float acc[32];
+    const float2* ml = (const float2*)part_ml + (long long)base * 128 + h;   // [slot][h] -> (m, l)
+    // running merge over batches of pieces: (M, L) and the accumulators stay consistent
+    float M = -INFINITY, L = 0.f, acc[32];
 #pragma unroll
     for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    for (int p = 0; p < np; ++p) {
-        const float w = exp2f(part_ml[((long long)(base + p) * 128 + h) * 2] - M) / L;
-        const float* src = part_o + (long long)(base + p) * 512 * 128 + (long long)(cb * 64 + half * 32) * 128 + h;
+    for (int p0 = 0; p0 < np; p0 += kMergeBatch) {
+        float2 v[kMergeBatch];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, src[(long long)i * 128], acc[i]);
-    }
+        for (int q = 0; q < kMergeBatch; ++q)
+            v[q] = p0 + q < np ? ml[(long long)(p0 + q) * 128] : make_float2(-INFINITY, 0.f);
+        float Mb = M;
 #pragma unroll
-    for (int i = 0; i < 32; i += 2) {
-        __nv_bfloat162 v = __floats2bfloat162_rn(acc[i], acc[i + 1]);
-        *reinterpret_cast<__nv_bfloat162*>(dst + i) = v;
+        for (int q = 0; q < kMergeBatch; ++q) Mb = fmaxf(Mb, v[q].x);
+        const float rescale = M == -INFINITY ? 0.f : exp2f(M - Mb);
+        L *= rescale;
+#pragma unroll
+        for (int i = 0; i < 32; ++i) acc[i] *= rescale;
+        M = Mb;
+#pragma unroll
+        for (int q = 0; q < kMergeBatch; ++q) {
+            if (p0 + q >= np) break;
+            const float w = exp2f(v[q].x - M);
+            L += w * v[q].y;
+            const float* src = part_o + (long long)(base + p0 + q) * 512 * 128 + (long long)c0 * 128 + h;
+            float x[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) x[i] = src[(long long)i * 128];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, x[i], acc[i]);
+        }
     }
+    const float inv = 1.f / L;
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) pk[i] = ptx::pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
 }
 
 int g_clusters_cached = 0;
@@ -694,8 +777,9 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     const int P = max_clusters(num_sms);
     {
         ProfScope ps(s, "tc_plan");
-        plan_kernel<<<1, 256, 0, s>>>(offsets, B, P, ws.work, err_code, err_detail);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(plan_kernel, dim3(1), dim3(256), 0, s, offsets, B, P, ws.work, err_code, err_detail)) !=
+            cudaSuccess)
+            return e;
     }
     {
         // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]  (per head: [512 x 128] x [128 x B])
@@ -712,15 +796,16 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         const uint32_t box[2] = {64, (uint32_t)kT};
         if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
         cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-        decode_tc_kernel<<<2 * P, kThreads, kSmem, s>>>(m, ws.q_lat, qr, sQr_b, sQr_h, offsets, B, cache_rows, ws.work,
-                                                    scale * 1.4426950408889634f, ws.part_o, ws.part_ml, err_code,
-                                                    err_detail);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, ws.q_lat, qr, sQr_b, sQr_h,
+                            offsets, B, (long long)cache_rows, (const int32_t*)ws.work, scale * 1.4426950408889634f,
+                            ws.part_o, ws.part_ml, err_code, err_detail)) != cudaSuccess)
+            return e;
     }
     {
         ProfScope ps(s, "tc_combine");
-        combine_tc_kernel<<<dim3(B, 8), 256, 0, s>>>(ws.work, B, ws.part_o, ws.part_ml, ws.o_lat);
-        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        if ((e = launch_pdl(combine_tc_kernel, dim3(B, 16), dim3(128), 0, s, (const int32_t*)ws.work, B,
+                            (const float*)ws.part_o, (const float*)ws.part_ml, ws.o_lat)) != cudaSuccess)
+            return e;
     }
     {
         // o[b,h,:] = W_UV[h] o_lat[b,h,:]  (per head: [128 x 512] x [512 x B])

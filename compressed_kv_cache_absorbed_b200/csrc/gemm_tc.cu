@@ -66,21 +66,32 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) pdl_trigger();
 
     if (warp == 0) {
         if (lane == 0) {
             ptx::tma_prefetch(&tmA);
             ptx::tma_prefetch(&tmB);
+            // A (the weights) of the first stages does not depend on earlier kernels: start it
+            // before waiting for them; B and the output do.
+            const int pre = nk < stages ? nk : stages;
+            for (int kb = 0; kb < pre; ++kb) {
+                ptx::mbar_expect_tx(&full[kb], C::STAGE);
+                ptx::tma_load_3d(smem + kb * C::STAGE, &tmA, &full[kb], kb * kBK, m0, z);
+            }
+            pdl_wait();
             for (int kb = 0; kb < nk; ++kb) {
                 const int s = kb % stages;
                 const uint32_t ph = (kb / stages) & 1;
-                if (kb >= stages && !ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-                    fail(err_code, err_detail, abort_flag, 1);
-                    break;
-                }
                 uint8_t* a = smem + s * C::STAGE;
-                ptx::mbar_expect_tx(&full[s], C::STAGE);
-                ptx::tma_load_3d(a, &tmA, &full[s], kb * kBK, m0, z);
+                if (kb >= pre) {
+                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
+                        fail(err_code, err_detail, abort_flag, 1);
+                        break;
+                    }
+                    ptx::mbar_expect_tx(&full[s], C::STAGE);
+                    ptx::tma_load_3d(a, &tmA, &full[s], kb * kBK, m0, z);
+                }
                 ptx::tma_load_3d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0, z);
             }
         }
@@ -108,6 +119,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
     } else {
         const int sub = warp & 3;
+        pdl_wait();   // the output may still be read by an earlier kernel
         const bool ok = ptx::mbar_wait(accum, 0, nullptr);
         if (!ok) fail(err_code, err_detail, abort_flag, 3);
         ptx::tc_fence_after();
@@ -155,8 +167,8 @@ cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUte
     const int nk = (K + kBK - 1) / kBK;
     const int stages = nk < C::MAX_STAGES ? (nk < 2 ? 2 : nk) : C::MAX_STAGES;
     dim3 grid((N + BN - 1) / BN, (M + kBM - 1) / kBM, Z);
-    gemm_bf16_tc_kernel<BN><<<grid, 192, C::smem(stages), s>>>(ma, mb, M, N, K, stages, out, err_code, err_detail);
-    return cudaGetLastError();
+    return launch_pdl(gemm_bf16_tc_kernel<BN>, grid, dim3(192), C::smem(stages), s, ma, mb, M, N, K, stages, out,
+                      err_code, err_detail);
 }
 
 }  // namespace

@@ -74,6 +74,18 @@ __device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint64_t* bar, uint3
         "r"(rank)
         : "memory");
 }
+// Non-blocking check of a phase.
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -136,6 +148,13 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
             smem_u32(dst)),
         "l"((uint64_t)map), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
         : "memory");
+}
+
+// Prefetch a tile of a tensor into L2 only (no shared memory, no completion to wait for).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* map, int c0, int c1) {
+    asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"((uint64_t)map), "r"(c0),
+                 "r"(c1)
+                 : "memory");
 }
 
 // ------------------------------------------------------------------- tcgen05
