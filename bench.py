@@ -161,7 +161,8 @@ def barrier():
 def max_over_ranks(x: float) -> float:
     import torch.distributed as dist
     if dist.is_available() and dist.is_initialized():
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        dev = "cpu" if dist.get_backend() == "gloo" else "cuda"
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
     return x
