@@ -48,12 +48,11 @@ namespace {
 
 constexpr int kT = 64;                        // tokens per tile
 constexpr int kStages = 4;
-constexpr int kL2Ahead = 6;                   // tiles pulled into L2 ahead of the ring
 constexpr int kChunkBytes = kT * 128;         // one 64-column box of a tile
 constexpr int kTileBytes = 5 * kChunkBytes;   // 4 latent chunks + the rotary chunk
 constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
 constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
-constexpr int kBarBytes = 256 + 2048;
+constexpr int kBarBytes = 256 + 2048 + 256;
 // tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer)
 // The dynamic shared memory of a kernel without static shared memory starts 1024-byte
 // aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
@@ -63,93 +62,11 @@ constexpr uint32_t kColQ = 0, kColS = 160, kColP = 224, kColO = 256, kTmemCols =
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 softmax warps
 
-// plan layout (int32): [0] total tiles, [1] tiles per cluster, [2] clusters,
-// [4, 4+B+1) first tile of each sequence, [4+B+1, 4+2B+2) first partial slot of each sequence
+// Plan written by CTA 0 for the merge kernel (int32): [0] total tiles, [1] tiles per cluster,
+// [2] clusters, [4, 4+B+1) first tile of each sequence (the last entry is the total).
 __device__ __forceinline__ const int32_t* plan_tstart(const int32_t* w) { return w + 4; }
-__device__ __forceinline__ const int32_t* plan_sbase(const int32_t* w, int B) { return w + 4 + B + 1; }
 
-// Block-wide exclusive scan of one value per thread (256 threads) with warp shuffles.
-template <typename T>
-__device__ __forceinline__ T block_exclusive_scan(T v, T* warp_tot, T* total) {
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-    T incl = v;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const T n = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += n;
-    }
-    if (lane == 31) warp_tot[w] = incl;
-    __syncthreads();
-    if (w == 0) {
-        T t = lane < 8 ? warp_tot[lane] : T(0);
-        T ti = t;
-#pragma unroll
-        for (int o = 1; o < 8; o <<= 1) {
-            const T n = __shfl_up_sync(0xffffffffu, ti, o);
-            if (lane >= o) ti += n;
-        }
-        if (lane < 8) warp_tot[lane] = ti - t;
-        if (lane == 7) *total = ti;
-    }
-    __syncthreads();
-    return warp_tot[w] + incl - v;
-}
-
-// One block of 256 threads: each thread takes a contiguous run of sequences; two block
-// scans give every sequence its first tile and its first partial slot.
-__global__ void __launch_bounds__(256)
-plan_kernel(const int32_t* __restrict__ offsets, int B, int P, int32_t* __restrict__ work, int* err_code,
-            long long* err_detail) {
-    __shared__ long long s_wt[8];
-    __shared__ long long s_tot;
-    __shared__ int s_wp[8];
-    __shared__ int s_ptot;
-    const int t = threadIdx.x;
-    if (t == 0) pdl_trigger();
-    pdl_wait();
-    const int per_thread = (B + 255) / 256;
-    const int b0 = min(B, t * per_thread), b1 = min(B, b0 + per_thread);
-    auto tiles_of = [&](int b) -> long long {
-        long long L = (long long)offsets[b + 1] - offsets[b];
-        if (L < 0) {
-            latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
-            L = 0;
-        }
-        return (L + kT - 1) / kT;
-    };
-    long long mine = 0;
-    for (int b = b0; b < b1; ++b) mine += tiles_of(b);
-    const long long t_first = block_exclusive_scan<long long>(mine, s_wt, &s_tot);
-    const long long total = s_tot;
-    const long long per_l = (total + P - 1) / P;
-    const int per = per_l > 0 ? (int)per_l : 1;
-    int32_t* ts = work + 4;
-    long long tcur = t_first;
-    int pieces = 0;
-    for (int b = b0; b < b1; ++b) {
-        const long long nt = tiles_of(b);
-        ts[b] = (int32_t)tcur;
-        if (nt > 0) pieces += (int)((tcur + nt - 1) / per - tcur / per + 1);
-        tcur += nt;
-    }
-    const int p_first = block_exclusive_scan<int>(pieces, s_wp, &s_ptot);
-    int32_t* sb = work + 4 + B + 1;
-    tcur = t_first;
-    int scur = p_first;
-    for (int b = b0; b < b1; ++b) {
-        sb[b] = scur;
-        const long long nt = tiles_of(b);
-        if (nt > 0) scur += (int)((tcur + nt - 1) / per - tcur / per + 1);
-        tcur += nt;
-    }
-    if (t == 0) {
-        work[0] = (int32_t)total;
-        work[1] = per;
-        work[2] = P;
-        work[4 + B] = (int32_t)total;
-        work[4 + B + 1 + B] = s_ptot;
-    }
-}
+__device__ __forceinline__ int tiles_of_len(int L) { return L > 0 ? (L + kT - 1) / kT : 0; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -182,24 +99,31 @@ struct Seg {
     long long row0;
 };
 
-// Iterates over the pieces of sequences in this cluster's tile range (same order in both CTAs).
+// Walks the pieces of sequences in this cluster's tile range [lo, hi), in sequence order,
+// starting from the sequence that holds tile lo (first tile t0).  The same walk runs in
+// every role of both CTAs.  Partial slots: a piece that starts at its sequence's first tile
+// takes slot b; the one piece of a cluster that continues a sequence begun in an earlier
+// cluster takes slot B + cluster.  So B + clusters slots suffice and need no prefix sums.
 struct SegIter {
-    const int32_t* ts;
-    const int32_t* sb;
     const int32_t* offsets;
-    int B, lo, hi, per, cluster, b;
+    int B, lo, hi, cluster, b, t0;
     __device__ bool next(Seg& s) {
-        for (; b < B && ts[b] < hi; ++b) {
-            const int t0 = ts[b], t1 = ts[b + 1];
-            if (t1 <= lo || t1 == t0) continue;
-            s.b = b;
-            s.j0 = (lo > t0 ? lo : t0) - t0;
-            s.j1 = (hi < t1 ? hi : t1) - t0;
-            s.row0 = offsets[b];
-            s.L = offsets[b + 1] - offsets[b];
-            s.slot = sb[b] + cluster - t0 / per;
+        while (b < B && t0 < hi) {
+            const int r0 = offsets[b], r1 = offsets[b + 1];
+            const int L = r1 > r0 ? r1 - r0 : 0;
+            const int t1 = t0 + tiles_of_len(L);
+            const int bb = b, tt0 = t0;
             ++b;
-            return true;
+            t0 = t1;
+            if (t1 > lo && t1 > tt0) {
+                s.b = bb;
+                s.j0 = (lo > tt0 ? lo : tt0) - tt0;
+                s.j1 = (hi < t1 ? hi : t1) - tt0;
+                s.row0 = r0;
+                s.L = L;
+                s.slot = tt0 >= lo ? bb : B + cluster;
+                return true;
+            }
         }
         return false;
     }
@@ -214,13 +138,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
-                 const int32_t* __restrict__ work, float scale_log2,
+                 int32_t* __restrict__ work, float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, int* err_code, long long* err_detail) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if (ptx::smem_u32(smem_raw) & 1023) {   // uniform across the CTA: leave before any sync
         if (threadIdx.x == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 7000000);
         return;
     }
+    // this thread's sequence length for the planning below, requested before the set-up
+    // so that the load overlaps it
+    const int len0 = threadIdx.x < B ? offsets[threadIdx.x + 1] - offsets[threadIdx.x] : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
     uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
@@ -246,6 +173,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     float* pair_val = (float*)(s_full + 18);   // [2][2][128] values the two warps swap
     uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+    int* plan_wsum = (int*)(tmem_slot + 2);   // [16] per-warp sums of the planning scans
+    int* plan_first = plan_wsum + 16;         // [2] sequence holding this cluster's first tile, its first tile
 
     const uint32_t rank = cluster_rank(), peer = rank ^ 1;
     const int cluster = (int)cluster_id_x();
@@ -282,12 +211,77 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     if (threadIdx.x == 0) pdl_trigger();
-    pdl_wait();   // everything below reads the plan, the queries and the cache
 
-    const int per = work[1];
-    const int total = work[0];
-    SegIter it{plan_tstart(work), plan_sbase(work, B), offsets, B, cluster * per,
-               min(total, cluster * per + per), per, cluster, 0};
+    // ---------------------------------------------------------------- planning
+    // Each CTA cuts the tiles of all sequences (in order) into equal ranges itself, from
+    // the offsets alone, so the cache loads start without waiting for another kernel.  The
+    // call's first kernel waits for all earlier work before it lets this kernel launch, so
+    // the offsets and the cache are final; only the absorbed queries (q_lat) come from a
+    // kernel of this call, and only the threads that read them wait for it (pdl_wait).
+    constexpr int kWarps = kThreads / 32;
+    const int P = (int)(gridDim.x / 2);
+    int total = 0;
+    {
+        int mine = 0;
+        for (int b = threadIdx.x; b < B; b += kThreads) {
+            const int L = b == (int)threadIdx.x ? len0 : offsets[b + 1] - offsets[b];
+            if (L < 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
+            mine += tiles_of_len(L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
+        if (lane == 0) plan_wsum[warp] = mine;
+        if (threadIdx.x == 0) {
+            plan_first[0] = B;
+            plan_first[1] = 0;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kWarps; ++i) total += plan_wsum[i];
+        __syncthreads();
+    }
+    const int per = total > 0 ? (total + P - 1) / P : 1;
+    const int lo = cluster * per, hi = min(total, lo + per);
+    const bool writer = blockIdx.x == 0;   // publishes every sequence's first tile for the merge
+    if (lo < total || writer) {
+        int carry = 0;
+        for (int c0 = 0; c0 < B; c0 += kThreads) {
+            const int b = c0 + (int)threadIdx.x;
+            const int n = b < B ? tiles_of_len(c0 == 0 ? len0 : offsets[b + 1] - offsets[b]) : 0;
+            int incl = n;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += v;
+            }
+            if (lane == 31) plan_wsum[warp] = incl;
+            __syncthreads();
+            int before = carry, chunk = 0;
+#pragma unroll
+            for (int i = 0; i < kWarps; ++i) {
+                const int v = plan_wsum[i];
+                before += i < warp ? v : 0;
+                chunk += v;
+            }
+            const int t0 = before + incl - n;
+            if (b < B) {
+                if (writer) work[4 + b] = t0;
+                if (n > 0 && t0 <= lo && lo < t0 + n) {   // unique: the sequence holding tile lo
+                    plan_first[0] = b;
+                    plan_first[1] = t0;
+                }
+            }
+            carry += chunk;
+            __syncthreads();
+        }
+    }
+    if (writer && threadIdx.x == 0) {
+        work[0] = total;
+        work[1] = per;
+        work[2] = P;
+        work[4 + B] = total;
+    }
+    SegIter it{offsets, B, lo, hi, cluster, plan_first[0], plan_first[1]};
     Seg sg;
 
     if (warp == 0) {
@@ -295,24 +289,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         if (lane == 0) {
             ptx::tma_prefetch(&tm_cache);
             uint32_t g = 0;
-            // a second cursor kL2Ahead tiles ahead pulls tiles into L2, so that the ring's
-            // loads (which wait for free stages) find them there
-            SegIter itp = it;
-            Seg sp;
-            bool p_have = itp.next(sp);
-            int p_j = p_have ? sp.j0 : 0;
-            auto prefetch_next = [&]() {
-                if (!p_have) return;
-                const int row = (int)(sp.row0 + (long long)p_j * kT);
-#pragma unroll
-                for (int i = 0; i < 4; ++i) ptx::tma_prefetch_l2_2d(&tm_cache, 256 * (int)rank + 64 * i, row);
-                ptx::tma_prefetch_l2_2d(&tm_cache, 512, row);
-                if (++p_j == sp.j1) {
-                    p_have = itp.next(sp);
-                    p_j = p_have ? sp.j0 : 0;
-                }
-            };
-            for (int k = 0; k < kL2Ahead; ++k) prefetch_next();
             while (!*abort_flag && it.next(sg)) {
                 if (sg.row0 + (long long)sg.L > cache_rows) {   // sequence beyond the cache
                     latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
@@ -326,7 +302,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                         fail(err_code, err_detail, abort_flag, 1);
                         break;
                     }
-                    prefetch_next();
                     uint8_t* dst = tiles + s * kTileBytes;
                     const int row = (int)(sg.row0 + (long long)j * kT);
                     ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
@@ -473,6 +448,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(q_ready);
             };
+            pdl_wait();   // q_lat is written by the previous kernel of this call
             if (have) load_q(cur.b);
             while (have) {
                 const uint32_t b = g & 1, u = g >> 1;
@@ -617,20 +593,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(p_ready);
                 if (j + 1 == cur.j1) {
-                    // piece epilogue: un-normalised O_r -> part_o[slot][c][h] (each half
+                    // piece epilogue: un-normalised O_r -> part_o[slot][h][c] (each half
                     // writes 128 columns); (m, l) from CTA 0
                     const float l_all = l_run + pair_exchange(l_run);
                     if (!ok) break;
                     if (!uwait(o_done, g & 1)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    float* po = part_o + (long long)cur.slot * 512 * 128 + (long long)(256 * rank) * 128 + h;
+                    // fragment order: four threads hold 32 contiguous bytes of one head's row,
+                    // so every store instruction writes whole sectors
+                    const int hq = sub * 32 + (lane >> 2), cq = 2 * (lane & 3);
 #pragma unroll 1
-                    for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
-                        uint32_t r[32];
-                        ptx::tmem_ld32(lane_addr + kColO + c0, r);
-                        ptx::tmem_wait_ld();
+                    for (int k = 0; k < 2; ++k) {
+                        float* poA = part_o + ((long long)cur.slot * 128 + hq + 16 * k) * 512 + 256 * rank + cq;
+                        float* poB = poA + 8 * 512;
+#pragma unroll 1
+                        for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
+                            uint32_t r[16];
+                            ptx::tmem_ld16x256b_x4(lane_addr + ((uint32_t)(16 * k) << 16) + kColO + c0, r);
+                            ptx::tmem_wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 32; ++i) po[(long long)(c0 + i) * 128] = __uint_as_float(r[i]);
+                            for (int j = 0; j < 4; ++j) {
+                                *(uint2*)(poA + c0 + 8 * j) = make_uint2(r[4 * j], r[4 * j + 1]);
+                                *(uint2*)(poB + c0 + 8 * j) = make_uint2(r[4 * j + 2], r[4 * j + 3]);
+                            }
+                        }
                     }
                     if (rank == 0 && half == 0) {
                         part_ml[((long long)cur.slot * 128 + h) * 2] = m_run;
@@ -653,67 +639,185 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     cluster_sync_all();  // neither CTA leaves while its peer may still touch its shared memory
 }
 
-// ------------------------------------------------------------------- merge
-// o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[c,h] / sum_p 2^(m_p - M) l_p  over the pieces p of b.
-// Block = (sequence b, 32 latent columns), thread = head.  The (m, l) of up to kMergeBatch
-// pieces are fetched together and every piece's 32 partial values are loaded before they
-// are used, so the block waits on memory once per batch rather than once per value.
-constexpr int kMergeBatch = 8;
+// ------------------------------------------------------------- merge + W_UV
+// o[b,h,:] = W_UV[h] o_lat[b,h,:],  o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[h,c] / sum_p 2^(m_p - M) l_p
+// over the pieces p of sequence b (M = max_p m_p; an empty sequence gives o = 0).
+// One CTA per (head h, block of BN sequences).  Thread 0 starts the TMA loads of W_UV[h]
+// (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
+// then merge the partials of their rows (warp per row, lane per 16 columns) straight into
+// the B operand in shared memory (K-major, 128-byte swizzle, as TMA would lay it out);
+// one thread issues the 32 MMAs (M = 128, N = BN) and four warps store D = o[:, h, :]^T.
+constexpr int kMergeThreads = 512;
+constexpr int kMergeABytes = 8 * 128 * 128;   // W_UV[h]: 8 chunks of 128 rows x 64 columns
 
-__global__ void __launch_bounds__(128)
-combine_tc_kernel(const int32_t* __restrict__ work, int B, const float* __restrict__ part_o,
-                  const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o_lat) {
-    const int b = blockIdx.x, c0 = blockIdx.y * 32, h = threadIdx.x;
-    if (threadIdx.x == 0) pdl_trigger();
-    pdl_wait();
-    const int32_t* ts = plan_tstart(work);
-    const int32_t* sb = plan_sbase(work, B);
-    const int per = work[1];
-    const int t0 = ts[b], t1 = ts[b + 1], base = sb[b];
-    uint4* dst = (uint4*)(o_lat + ((long long)b * 128 + h) * 512 + c0);
-    if (t1 == t0) {
+template <int BN>
+constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
+
+template <int BN>
+__global__ void __launch_bounds__(kMergeThreads, 1)
+merge_wuv_kernel(const __grid_constant__ CUtensorMap tm_wuv, const int32_t* __restrict__ work, int B,
+                 const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
+                 long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
+    extern __shared__ uint8_t merge_smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)merge_smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + kMergeABytes;
+    uint64_t* a_full = (uint64_t*)(sB + 8 * BN * 128);
+    uint64_t* d_full = a_full + 1;
+    uint32_t* tmem_slot = (uint32_t*)(d_full + 1);
+    const int h = blockIdx.x, n0 = blockIdx.y * BN;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(a_full, 1);
+        ptx::mbar_init(d_full, 1);
+        ptx::fence_mbar_init();
+        ptx::tma_prefetch(&tm_wuv);
+        // the weights are not written by earlier kernels: load them before waiting
+        ptx::mbar_expect_tx(a_full, kMergeABytes);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(0, 0, 0, 0);
-        return;
+        for (int kc = 0; kc < 8; ++kc) ptx::tma_load_2d(sA + kc * 16384, &tm_wuv, a_full, 64 * kc, 128 * h);
     }
-    const int np = (t1 - 1) / per - t0 / per + 1;
-    const float2* ml = (const float2*)part_ml + (long long)base * 128 + h;   // [slot][h] -> (m, l)
-    // running merge over batches of pieces: (M, L) and the accumulators stay consistent
-    float M = -INFINITY, L = 0.f, acc[32];
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, BN);
+        ptx::tmem_relinquish();
+    }
+    if (threadIdx.x == 0) pdl_trigger();
+    pdl_wait();   // the partials and the plan come from the decode kernel
+
+    const int32_t* ts = plan_tstart(work);
+    const int per = work[1];
+    constexpr int kW = kMergeThreads / 32;
+    constexpr int kRowsPerWarp = BN / kW;
+    // first tiles of this warp's rows, fetched together
+    int t0r[kRowsPerWarp], t1r[kRowsPerWarp];
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[i] = 0.f;
-    for (int p0 = 0; p0 < np; p0 += kMergeBatch) {
-        float2 v[kMergeBatch];
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int b = n0 + warp + kW * i;
+        t0r[i] = b < B ? ts[b] : 0;
+        t1r[i] = b < B ? ts[b + 1] : 0;
+    }
 #pragma unroll
-        for (int q = 0; q < kMergeBatch; ++q)
-            v[q] = p0 + q < np ? ml[(long long)(p0 + q) * 128] : make_float2(-INFINITY, 0.f);
-        float Mb = M;
+    for (int i = 0; i < kRowsPerWarp; ++i) {
+        const int r = warp + kW * i, b = n0 + r;
+        const int t0 = t0r[i], t1 = t1r[i];
+        float acc[16];
 #pragma unroll
-        for (int q = 0; q < kMergeBatch; ++q) Mb = fmaxf(Mb, v[q].x);
-        const float rescale = M == -INFINITY ? 0.f : exp2f(M - Mb);
-        L *= rescale;
+        for (int k = 0; k < 16; ++k) acc[k] = 0.f;
+        if (t1 > t0) {
+            // piece 0 (from cluster t0 / per) is in slot b; piece p > 0 continues the
+            // sequence in cluster t0 / per + p and is in slot B + t0 / per + p
+            const int cfirst = t0 / per;
+            const int np = (t1 - 1) / per - cfirst + 1;
+            auto slot_of = [&](int p) -> long long { return p == 0 ? b : B + cfirst + p; };
+            // (m, l) of up to 32 pieces (lane p) and the first 4 pieces' partial rows are
+            // requested together; the weights need the maximum, the loads do not
+            float2 ml = lane < np ? *(const float2*)(part_ml + (slot_of(lane) * 128 + h) * 2)
+                                  : make_float2(-INFINITY, 0.f);
+            float4 x[4][4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) acc[i] *= rescale;
-        M = Mb;
+            for (int q = 0; q < 4; ++q) {
+                const float4* src = (const float4*)(part_o + (slot_of(q < np ? q : 0) * 128 + h) * 512 + 16 * lane);
 #pragma unroll
-        for (int q = 0; q < kMergeBatch; ++q) {
-            if (p0 + q >= np) break;
-            const float w = exp2f(v[q].x - M);
-            L += w * v[q].y;
-            const float* src = part_o + (long long)(base + p0 + q) * 512 * 128 + (long long)c0 * 128 + h;
-            float x[32];
+                for (int v = 0; v < 4; ++v) x[q][v] = q < np ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float M = ml.x;
+            for (int p = 32 + lane; p < np; p += 32) M = fmaxf(M, part_ml[(slot_of(p) * 128 + h) * 2]);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) x[i] = src[(long long)i * 128];
+            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+            const float w_lane = lane < np ? exp2f(ml.x - M) : 0.f;
+            float L = w_lane * ml.y;
+            for (int p = 32 + lane; p < np; p += 32) {
+                const float2 v = *(const float2*)(part_ml + (slot_of(p) * 128 + h) * 2);
+                L += exp2f(v.x - M) * v.y;
+            }
 #pragma unroll
-            for (int i = 0; i < 32; ++i) acc[i] = fmaf(w, x[i], acc[i]);
+            for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+            for (int p0 = 0;; p0 += 4) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int p = p0 + q;
+                    float w = __shfl_sync(0xffffffffu, w_lane, p & 31);
+                    if (p >= 32) w = p < np ? exp2f(part_ml[(slot_of(p) * 128 + h) * 2] - M) : 0.f;
+                    if (p >= np) w = 0.f;
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) {
+                        acc[4 * v] = fmaf(w, x[q][v].x, acc[4 * v]);
+                        acc[4 * v + 1] = fmaf(w, x[q][v].y, acc[4 * v + 1]);
+                        acc[4 * v + 2] = fmaf(w, x[q][v].z, acc[4 * v + 2]);
+                        acc[4 * v + 3] = fmaf(w, x[q][v].w, acc[4 * v + 3]);
+                    }
+                }
+                if (p0 + 4 >= np) break;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {   // the next four pieces
+                    const int p = p0 + 4 + q;
+                    const float4* src = (const float4*)(part_o + (slot_of(p < np ? p : 0) * 128 + h) * 512 + 16 * lane);
+#pragma unroll
+                    for (int v = 0; v < 4; ++v) x[q][v] = p < np ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+            }
+            const float inv = 1.f / L;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) acc[k] *= inv;
+        }
+        // columns 16 lane .. +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
+        uint8_t* rowp = sB + (lane >> 2) * (BN * 128) + r * 128;
+#pragma unroll
+        for (int hv = 0; hv < 2; ++hv) {
+            const int u = 2 * (lane & 3) + hv;
+            *(uint4*)(rowp + ((u ^ (r & 7)) << 4)) =
+                make_uint4(ptx::pack_bf16(acc[8 * hv], acc[8 * hv + 1]), ptx::pack_bf16(acc[8 * hv + 2], acc[8 * hv + 3]),
+                           ptx::pack_bf16(acc[8 * hv + 4], acc[8 * hv + 5]),
+                           ptx::pack_bf16(acc[8 * hv + 6], acc[8 * hv + 7]));
         }
     }
-    const float inv = 1.f / L;
-    uint32_t pk[16];
+    ptx::fence_proxy_async_smem();   // the tensor cores read what the threads wrote
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    bool ok = true;
+    if (threadIdx.x == 32) {
+        if (!ptx::mbar_wait(a_full, 0, nullptr)) {
+            latch(DevErr{err_code, err_detail}, kErrTimeout, 8000000 + h);
+            ok = false;
+        } else {
+            ptx::tc_fence_after();
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, BN, 0, 0);
 #pragma unroll
-    for (int i = 0; i < 16; ++i) pk[i] = ptx::pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+            for (int kc = 0; kc < 8; ++kc)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                for (int k = 0; k < 4; ++k)
+                    ptx::mma_ss(tmem, ptx::desc_kmajor_sw128(ptx::smem_u32(sA + kc * 16384) + 32 * k),
+                                ptx::desc_kmajor_sw128(ptx::smem_u32(sB + kc * BN * 128) + 32 * k), idesc,
+                                (kc | k) != 0);
+        }
+        ptx::mma_commit(d_full);   // also after a timeout: nothing issued, completes at once
+    }
+    if (warp < 4) {
+        if (!ptx::mbar_wait(d_full, 0, nullptr)) {
+            if (lane == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 8100000 + h);
+        } else {
+            ptx::tc_fence_after();
+            const int m = warp * 32 + lane;   // output row = TMEM lane
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int b = n0 + c0 + j;
+                    if (b < B) o[b * sO_b + h * sO_h + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                }
+            }
+        }
+    }
+    (void)ok;
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, BN);
 }
 
 int g_clusters_cached = 0;
@@ -776,16 +880,13 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     const int P = max_clusters(num_sms);
     {
-        ProfScope ps(s, "tc_plan");
-        if ((e = launch_pdl(plan_kernel, dim3(1), dim3(256), 0, s, offsets, B, P, ws.work, err_code, err_detail)) !=
-            cudaSuccess)
-            return e;
-    }
-    {
         // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]  (per head: [512 x 128] x [128 x B])
         ProfScope ps(s, "tc_q_absorb");
         GemmOut out{ws.q_lat, 512, 1, 128LL * 512, 0};
-        e = gemm_bf16_tc(128, 512, B, 128, W_UKT, 512LL * 128, 128, qn, sQn_h, sQn_b, out, err_code, err_detail, s);
+        // first kernel of the call: it waits for all earlier work before the next kernels may
+        // launch (the decode kernel reads the cache and offsets without waiting)
+        e = gemm_bf16_tc(128, 512, B, 128, W_UKT, 512LL * 128, 128, qn, sQn_h, sQn_b, out, err_code, err_detail, s,
+                         /*chain_head=*/true);
         if (e != cudaSuccess) return e;
     }
     {
@@ -797,22 +898,29 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
         cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, ws.q_lat, qr, sQr_b, sQr_h,
-                            offsets, B, (long long)cache_rows, (const int32_t*)ws.work, scale * 1.4426950408889634f,
+                            offsets, B, (long long)cache_rows, ws.work, scale * 1.4426950408889634f,
                             ws.part_o, ws.part_ml, err_code, err_detail)) != cudaSuccess)
             return e;
     }
     {
-        ProfScope ps(s, "tc_combine");
-        if ((e = launch_pdl(combine_tc_kernel, dim3(B, 16), dim3(128), 0, s, (const int32_t*)ws.work, B,
-                            (const float*)ws.part_o, (const float*)ws.part_ml, ws.o_lat)) != cudaSuccess)
-            return e;
-    }
-    {
-        // o[b,h,:] = W_UV[h] o_lat[b,h,:]  (per head: [128 x 512] x [512 x B])
-        ProfScope ps(s, "tc_w_uv");
-        GemmOut out{o, 128, 1, 128LL * 128, 0};
-        e = gemm_bf16_tc(128, 128, B, 512, W_UV, 128LL * 512, 512, ws.o_lat, 512, 128LL * 512, out, err_code,
-                         err_detail, s);
+        // merge of the pieces fused with o[b,h,:] = W_UV[h] o_lat[b,h,:]
+        ProfScope ps(s, "tc_merge_w_uv");
+        CUtensorMap m;
+        const uint64_t dims[2] = {512, 128ull * 128};
+        const uint64_t strides[1] = {512 * 2};
+        const uint32_t box[2] = {64, 128};
+        if (!make_tmap_bf16(&m, W_UV, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        if (B <= 32) {
+            cudaFuncSetAttribute(merge_wuv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, merge_smem<32>());
+            e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, m,
+                           (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           128LL * 128, 128LL, err_code, err_detail);
+        } else {
+            cudaFuncSetAttribute(merge_wuv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, merge_smem<64>());
+            e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
+                           m, (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           128LL * 128, 128LL, err_code, err_detail);
+        }
     }
     return e;
 }

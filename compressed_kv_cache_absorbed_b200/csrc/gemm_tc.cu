@@ -35,7 +35,7 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                    int N, int K, int stages, GemmOut out, int* err_code, long long* err_detail) {
+                    int N, int K, int stages, GemmOut out, int chain_head, int* err_code, long long* err_detail) {
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -66,7 +66,13 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __syncthreads();
     ptx::tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    if (threadIdx.x == 0) pdl_trigger();
+    // Dependents may launch once every CTA got here.  As the first kernel of a chain this
+    // waits for all earlier work first, so that later kernels of the chain may read the
+    // chain's inputs without waiting.
+    if (threadIdx.x == 64) {
+        if (chain_head) pdl_wait();
+        pdl_trigger();
+    }
 
     if (warp == 0) {
         if (lane == 0) {
@@ -155,7 +161,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 template <int BN>
 cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUtensorMap& mb, const GemmOut& out,
-                   int* err_code, long long* err_detail, cudaStream_t s) {
+                   bool chain_head, int* err_code, long long* err_detail, cudaStream_t s) {
     using C = GemmCfg<BN>;
     static bool attr_set = false;   // the attribute is per function; set it once
     if (!attr_set) {
@@ -168,14 +174,14 @@ cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUte
     const int stages = nk < C::MAX_STAGES ? (nk < 2 ? 2 : nk) : C::MAX_STAGES;
     dim3 grid((N + BN - 1) / BN, (M + kBM - 1) / kBM, Z);
     return launch_pdl(gemm_bf16_tc_kernel<BN>, grid, dim3(192), C::smem(stages), s, ma, mb, M, N, K, stages, out,
-                      err_code, err_detail);
+                      (int)chain_head, err_code, err_detail);
 }
 
 }  // namespace
 
 cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, long long sAz, long long sAm,
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
-                         int* err_code, long long* err_detail, cudaStream_t s) {
+                         int* err_code, long long* err_detail, cudaStream_t s, bool chain_head) {
     if (Z <= 0 || M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
     const int BN = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
     if (Z == 1) {
@@ -192,10 +198,10 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     if (!make_tmap_bf16(&ma, A, 3, da, sa, ba) || !make_tmap_bf16(&mb, B, 3, db, sb, bb))
         return cudaErrorInvalidValue;
     switch (BN) {
-        case 32: return launch<32>(Z, M, N, K, ma, mb, out, err_code, err_detail, s);
-        case 64: return launch<64>(Z, M, N, K, ma, mb, out, err_code, err_detail, s);
-        case 128: return launch<128>(Z, M, N, K, ma, mb, out, err_code, err_detail, s);
-        default: return launch<256>(Z, M, N, K, ma, mb, out, err_code, err_detail, s);
+        case 32: return launch<32>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
+        case 64: return launch<64>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
+        case 128: return launch<128>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
+        default: return launch<256>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
     }
 }
 

@@ -223,6 +223,17 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
 }
+// 16 lanes x 32 columns in the accumulator-fragment order: thread i of the warp gets, for
+// each 8-column group j, columns 8j + 2(i % 4) and +1 of lane base + i / 4 (r[4j], r[4j+1])
+// and of lane base + i / 4 + 8 (r[4j+2], r[4j+3]).  Four threads thus hold 32 contiguous
+// bytes of one lane, which lets a warp store whole 32-byte sectors of a lane-major matrix.
+__device__ __forceinline__ void tmem_ld16x256b_x4(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.16x256b.x4.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+}
 // Finishes a pair of 32-column loads: `first` was issued by the caller at column c; this
 // issues column c + 32, waits for both and writes all 64 values to out as floats.
 __device__ __forceinline__ void tmem_ld32x2_second(uint32_t taddr2, float (&out)[64], uint32_t (&first)[32]) {
