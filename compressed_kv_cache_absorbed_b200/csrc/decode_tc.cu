@@ -38,7 +38,6 @@
 
 #include "common.cuh"
 #include "decode_tc.cuh"
-#include "gemm_tc.cuh"
 #include "tc_common.cuh"
 
 namespace mla {
@@ -139,7 +138,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
                  int32_t* __restrict__ work, float scale_log2,
-                 float* __restrict__ part_o, float* __restrict__ part_ml, int* err_code, long long* err_detail) {
+                 float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
+                 long long next_weight_bytes, int* err_code, long long* err_detail) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if (ptx::smem_u32(smem_raw) & 1023) {   // uniform across the CTA: leave before any sync
         if (threadIdx.x == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 7000000);
@@ -288,6 +288,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::tma_prefetch(&tm_cache);
+            // the cache is streamed once: let L2 drop it first, keeping the partials and weights
+            const uint64_t stream_policy = ptx::policy_evict_first();
             uint32_t g = 0;
             while (!*abort_flag && it.next(sg)) {
                 if (sg.row0 + (long long)sg.L > cache_rows) {   // sequence beyond the cache
@@ -307,9 +309,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                     ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
-                        ptx::tma_load_2d(dst + i * kChunkBytes, &tm_cache, &tile_full[s], 256 * (int)rank + 64 * i, row);
-                    ptx::tma_load_2d(dst + 4 * kChunkBytes, &tm_cache, &tile_full[s], 512, row);
+                        ptx::tma_load_2d_hint(dst + i * kChunkBytes, &tm_cache, &tile_full[s], 256 * (int)rank + 64 * i,
+                                              row, stream_policy);
+                    ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_cache, &tile_full[s], 512, row, stream_policy);
                 }
+            }
+            // All tiles requested: pull this CTA's share of the next kernel's weights (W_UV)
+            // into L2 while the last tiles are processed.
+            if (next_weights != nullptr && next_weight_bytes > 0) {
+                const long long share = ((next_weight_bytes + gridDim.x - 1) / gridDim.x + 15) & ~15LL;
+                const long long a = share * blockIdx.x;
+                const long long e = min(next_weight_bytes, a + share);
+                const uint64_t keep = ptx::policy_evict_last();
+                for (long long o = a; o < e; o += 16384)
+                    ptx::bulk_prefetch_l2(next_weights + o, (uint32_t)min(16384LL, e - o), keep);
             }
             // loads still in flight after an abort complete before the CTA leaves
             for (uint32_t k = 0; k < (uint32_t)kStages && k < g; ++k) {
@@ -820,11 +833,126 @@ merge_wuv_kernel(const __grid_constant__ CUtensorMap tm_wuv, const int32_t* __re
     if (warp == 1) ptx::tmem_dealloc(tmem, BN);
 }
 
+// Kernel attributes, set once per kernel: the dynamic shared memory it needs, and the
+// largest shared-memory carve-out for every kernel of the chain, so that consecutive kernels
+// find the SMs already configured.
+template <typename K>
+cudaError_t set_smem_attrs(K kernel, int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+    return e;
+}
+
+// ----------------------------------------------------------------- q absorption
+// q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:], as D[512 x BN] = W_UK^T[h] (512 x 128) . Q_h^T with
+// Q_h = q_nope[n0 .. n0+BN, h, :].  One CTA per (head, block of BN sequences) holds the whole
+// W_UK^T[h] (8 TMA boxes of 128 x 64, 128 KB) and Q_h (2 boxes), issues 4 x 8 MMAs into four
+// BN-column TMEM accumulators (one per 128-row tile) and stores q_lat.
+// This is the first kernel of the decode chain: it waits for all earlier work before it lets
+// the next kernel launch (the decode kernel then reads the cache without waiting).
+constexpr int kAbsorbThreads = 128;
+
+template <int BN>
+constexpr int absorb_smem() { return 8 * 16384 + 2 * BN * 128 + 1024 + 64; }
+
+template <int BN>
+__global__ void __launch_bounds__(kAbsorbThreads, 1)
+absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q, int B,
+                __nv_bfloat16* __restrict__ q_lat, int* err_code, long long* err_detail) {
+    extern __shared__ uint8_t absorb_smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)absorb_smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sA = smem;                  // [m tile][k chunk] boxes of 128 rows x 128 B
+    uint8_t* sB = smem + 8 * 16384;      // [k chunk] boxes of BN rows x 128 B
+    uint64_t* full = (uint64_t*)(sB + 2 * BN * 128);
+    uint64_t* d_full = full + 1;
+    uint32_t* tmem_slot = (uint32_t*)(d_full + 1);
+    const int h = blockIdx.x, n0 = blockIdx.y * BN;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(full, 1);
+        ptx::mbar_init(d_full, 1);
+        ptx::fence_mbar_init();
+        ptx::tma_prefetch(&tm_w);
+        ptx::tma_prefetch(&tm_q);
+        ptx::mbar_expect_tx(full, 8 * 16384 + 2 * BN * 128);
+        // weights first: earlier kernels do not write them
+#pragma unroll
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int kc = 0; kc < 2; ++kc)
+                ptx::tma_load_2d(sA + (mt * 2 + kc) * 16384, &tm_w, full, 64 * kc, 512 * h + 128 * mt);
+        pdl_wait();      // the queries may come from the previous kernel; all earlier work is done
+        pdl_trigger();   // only now may the next kernel launch
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) ptx::tma_load_3d(sB + kc * BN * 128, &tm_q, full, 64 * kc, n0, h);
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, 4 * BN);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 32) {
+        if (!ptx::mbar_wait(full, 0, nullptr)) {
+            latch(DevErr{err_code, err_detail}, kErrTimeout, 8200000 + h);
+        } else {
+            ptx::tc_fence_after();
+            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, BN, 0, 0);
+#pragma unroll
+            for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+                for (int kc = 0; kc < 2; ++kc)
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        ptx::mma_ss(tmem + mt * BN, ptx::desc_kmajor_sw128(ptx::smem_u32(sA + (mt * 2 + kc) * 16384) + 32 * k),
+                                    ptx::desc_kmajor_sw128(ptx::smem_u32(sB + kc * BN * 128) + 32 * k), idesc,
+                                    (kc | k) != 0);
+        }
+        ptx::mma_commit(d_full);   // after a timeout nothing was issued and this completes at once
+    }
+    if (!ptx::mbar_wait(d_full, 0, nullptr)) {
+        if (lane == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 8300000 + h);
+    } else {
+        ptx::tc_fence_after();
+        const int m = warp * 32 + lane;   // row of the 128-row tile = TMEM lane
+#pragma unroll 1
+        for (int mt = 0; mt < 4; ++mt)
+#pragma unroll
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) {
+                    const int b = n0 + c0 + j;
+                    if (b < B)
+                        q_lat[((long long)b * 128 + h) * 512 + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                }
+            }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, 4 * BN);
+}
+
+template <int BN>
+cudaError_t launch_absorb(const CUtensorMap& mw, const CUtensorMap& mq, int B, __nv_bfloat16* q_lat, int* err_code,
+                          long long* err_detail, cudaStream_t s) {
+    static const cudaError_t attr = set_smem_attrs(absorb_q_kernel<BN>, absorb_smem<BN>());
+    if (attr != cudaSuccess) return attr;
+    return launch_pdl(absorb_q_kernel<BN>, dim3(128, (B + BN - 1) / BN), dim3(kAbsorbThreads), absorb_smem<BN>(), s,
+                      mw, mq, B, q_lat, err_code, err_detail);
+}
+
 int g_clusters_cached = 0;
 
 int max_clusters(int num_sms) {
     if (g_clusters_cached > 0) return g_clusters_cached;
-    cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    set_smem_attrs(decode_tc_kernel, kSmem);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
@@ -880,13 +1008,21 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     const int P = max_clusters(num_sms);
     {
-        // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]  (per head: [512 x 128] x [128 x B])
+        // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]
         ProfScope ps(s, "tc_q_absorb");
-        GemmOut out{ws.q_lat, 512, 1, 128LL * 512, 0};
-        // first kernel of the call: it waits for all earlier work before the next kernels may
-        // launch (the decode kernel reads the cache and offsets without waiting)
-        e = gemm_bf16_tc(128, 512, B, 128, W_UKT, 512LL * 128, 128, qn, sQn_h, sQn_b, out, err_code, err_detail, s,
-                         /*chain_head=*/true);
+        CUtensorMap mw, mq;
+        const uint64_t dw[2] = {128, 128ull * 512};
+        const uint64_t sw[1] = {128 * 2};
+        const uint32_t bw[2] = {64, 128};
+        const int BN = B <= 32 ? 32 : B <= 64 ? 64 : 128;
+        const uint64_t dq[3] = {128, (uint64_t)B, 128};
+        const uint64_t sq[2] = {(uint64_t)sQn_b * 2, (uint64_t)sQn_h * 2};
+        const uint32_t bq[3] = {64, (uint32_t)BN, 1};
+        if (!make_tmap_bf16(&mw, W_UKT, 2, dw, sw, bw) || !make_tmap_bf16(&mq, qn, 3, dq, sq, bq))
+            return cudaErrorInvalidValue;
+        e = BN == 32   ? launch_absorb<32>(mw, mq, B, ws.q_lat, err_code, err_detail, s)
+            : BN == 64 ? launch_absorb<64>(mw, mq, B, ws.q_lat, err_code, err_detail, s)
+                       : launch_absorb<128>(mw, mq, B, ws.q_lat, err_code, err_detail, s);
         if (e != cudaSuccess) return e;
     }
     {
@@ -896,10 +1032,12 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         const uint64_t strides[1] = {576 * 2};
         const uint32_t box[2] = {64, (uint32_t)kT};
         if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
-        cudaFuncSetAttribute(decode_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+        static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
+        if (attr != cudaSuccess) return attr;
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, ws.q_lat, qr, sQr_b, sQr_h,
                             offsets, B, (long long)cache_rows, ws.work, scale * 1.4426950408889634f,
-                            ws.part_o, ws.part_ml, err_code, err_detail)) != cudaSuccess)
+                            ws.part_o, ws.part_ml, (const uint8_t*)W_UV, 128LL * 128 * 512 * 2, err_code,
+                            err_detail)) != cudaSuccess)
             return e;
     }
     {
@@ -911,12 +1049,14 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         const uint32_t box[2] = {64, 128};
         if (!make_tmap_bf16(&m, W_UV, 2, dims, strides, box)) return cudaErrorInvalidValue;
         if (B <= 32) {
-            cudaFuncSetAttribute(merge_wuv_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, merge_smem<32>());
+            static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
+            if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, m,
                            (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         } else {
-            cudaFuncSetAttribute(merge_wuv_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, merge_smem<64>());
+            static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
+            if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
                            m, (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
