@@ -16,23 +16,26 @@
 // which costs 64 exponentials per thread per tile and saves a second exchange hop.
 //
 // TMEM of one CTA (512 columns x 128 lanes; lane = head):
-//     [0, 144)   Q_r as the MMA A operand (288 bf16, two per column)
-//     [160, 224) S_r partial scores, fp32, 64 tokens
-//     [224, 256) P probabilities as the A operand (64 bf16)
+//     [0, 128)   Q_r latent part as the MMA A operand (256 bf16, two per column)
+//     [128, 192) S_r partial scores, fp32, 64 tokens
+//     [192, 256) P probabilities as the A operand, two buffers of 64 bf16 (tile g uses g & 1)
 //     [256, 512) O_r accumulator, fp32
-// Both MMAs read A from TMEM and only the tile from shared memory, which keeps shared
-// memory bandwidth at 64 B/clk (a 128x64 MMA with both operands in shared memory needs
-// 192 B/clk, more than the SM supplies).
+// The 32 rotary query columns of the CTA live in shared memory (64-byte swizzle) and enter
+// the score MMA as an SS operand; that frees the TMEM for the second P buffer, so the
+// softmax of tile g + 1 does not wait for the O MMAs of tile g.  The latent score MMAs and
+// the O MMAs read A from TMEM and only the tile from shared memory.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads of 64-token tiles (4 latent chunks of
-// 64 columns + the 64 rotary columns, 128-byte swizzle) into a 3-stage ring; warp 1 owns
-// TMEM and issues the MMAs; warps 2-5 (thread = head = TMEM lane) load Q, swap partial
-// scores, run the online softmax (base-2, lazy rescale: the running max moves only when a
-// tile exceeds it by more than 8, so p <= 256), write P, and read O back at the end.
+// Warp roles (448 threads): warp 0 issues TMA loads of 64-token tiles (4 latent boxes of
+// 64 columns with 128-byte swizzle + this CTA's 32 rotary columns with 64-byte swizzle,
+// 36 KB) into a 4-stage ring; warp 1 owns TMEM and issues the MMAs; warps 2-5 (thread = head
+// = TMEM lane) load Q and send partial scores to the peer; warps 6-13 (two per TMEM
+// subpartition, one per half tile) run the online softmax (base-2, lazy rescale: the running
+// max moves only when a tile exceeds it by more than 8, so p <= 256), write P, and read O
+// back at the end of each piece.
 //
 // Work split: the tiles of all sequences, in order, are cut into equal ranges, one per
 // cluster; a range may hold pieces of several sequences.  Each piece writes an
-// un-normalised partial (O, running max, row sum) that a merge kernel combines.
+// un-normalised partial (O, running max, row sum) that the merge kernel combines.
 // Every wait is bounded; a timeout latches an error and the kernel drains and exits.
 #include <math.h>
 
@@ -47,17 +50,19 @@ namespace {
 
 constexpr int kT = 64;                        // tokens per tile
 constexpr int kStages = 4;
-constexpr int kChunkBytes = kT * 128;         // one 64-column box of a tile
-constexpr int kTileBytes = 5 * kChunkBytes;   // 4 latent chunks + the rotary chunk
+constexpr int kChunkBytes = kT * 128;         // one 64-column latent box of a tile (128-byte swizzle)
+constexpr int kRopeBytes = kT * 64;           // this CTA's 32 rotary columns of a tile (64-byte swizzle)
+constexpr int kTileBytes = 4 * kChunkBytes + kRopeBytes;
+constexpr int kQRopeBytes = 128 * 64;         // this CTA's 32 rotary query columns, 128 heads
 constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
 constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
 constexpr int kBarBytes = 256 + 2048 + 256;
 // tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer)
 // The dynamic shared memory of a kernel without static shared memory starts 1024-byte
 // aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
-constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kBarBytes;
+constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kQRopeBytes + kBarBytes;
 static_assert(kSmem <= 232448, "decode kernel shared memory over the 227 KB limit");
-constexpr uint32_t kColQ = 0, kColS = 160, kColP = 224, kColO = 256, kTmemCols = 512;
+constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 softmax warps
 
@@ -134,7 +139,8 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
-decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat16* __restrict__ q_lat,
+decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_rope,
+                 const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
                  int32_t* __restrict__ work, float scale_log2,
@@ -152,25 +158,26 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
     uint8_t* tiles = smem;
     uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
     uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
-    uint64_t* bars = (uint64_t*)(xstage + 2 * kXBytes);
+    uint8_t* qrope = xstage + 2 * kXBytes;         // rotary query columns (A operand, 64-byte swizzle)
+    uint64_t* bars = (uint64_t*)(qrope + kQRopeBytes);
     uint64_t* tile_full = bars;
     uint64_t* tile_empty = bars + kStages;
     uint64_t* s_full = bars + 2 * kStages;
     uint64_t* s_free = s_full + 1;
-    uint64_t* p_ready = s_full + 2;
-    uint64_t* o_done = s_full + 3;
-    uint64_t* q_ready = s_full + 4;
+    uint64_t* p_ready = s_full + 2;    // [2] P of tile g is in P buffer g & 1
+    uint64_t* o_done = s_full + 4;     // [2] the O MMAs of tile g (and all before) completed
+    uint64_t* q_ready = s_full + 6;
     // [2] the peer's partial scores for tile g landed in xbuf[g & 1]: armed locally with the
     // byte count, completed by the peer's bulk copy
-    uint64_t* x_full = s_full + 5;
+    uint64_t* x_full = s_full + 7;
     // [2] the peer has read what this CTA sent into its xbuf[g & 1]; that copy therefore also
     // finished reading this CTA's xstage[g & 1] (one arrive per peer warp)
-    uint64_t* x_empty = s_full + 7;
-    uint64_t* drain = s_full + 9;    // all MMAs issued by this CTA have completed
-    uint64_t* xs_ready = s_full + 10;  // [2] all 128 rows of xstage[g & 1] written
-    uint64_t* xs_free = s_full + 12;   // [2] the local softmax has read xstage[g & 1]
-    uint64_t* pair_bar = s_full + 14;  // [4] the two softmax warps of a subpartition
-    float* pair_val = (float*)(s_full + 18);   // [2][2][128] values the two warps swap
+    uint64_t* x_empty = s_full + 9;
+    uint64_t* drain = s_full + 11;     // all MMAs issued by this CTA have completed
+    uint64_t* xs_ready = s_full + 12;  // [2] all 128 rows of xstage[g & 1] written
+    uint64_t* xs_free = s_full + 14;   // [2] the local softmax has read xstage[g & 1]
+    uint64_t* pair_bar = s_full + 16;  // [4] the two softmax warps of a subpartition
+    float* pair_val = (float*)(s_full + 20);   // [2][2][128] values the two warps swap
     uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* plan_wsum = (int*)(tmem_slot + 2);   // [16] per-warp sums of the planning scans
@@ -187,9 +194,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         }
         ptx::mbar_init(s_full, 1);
         ptx::mbar_init(s_free, 128);
-        ptx::mbar_init(p_ready, 256);
+        ptx::mbar_init(&p_ready[0], 256);
+        ptx::mbar_init(&p_ready[1], 256);
         for (int i = 0; i < 4; ++i) ptx::mbar_init(&pair_bar[i], 64);
-        ptx::mbar_init(o_done, 1);
+        ptx::mbar_init(&o_done[0], 1);
+        ptx::mbar_init(&o_done[1], 1);
         ptx::mbar_init(q_ready, 128);
         ptx::mbar_init(drain, 1);
         for (int i = 0; i < 2; ++i) {
@@ -288,6 +297,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
             ptx::tma_prefetch(&tm_cache);
+            ptx::tma_prefetch(&tm_rope);
             // the cache is streamed once: let L2 drop it first, keeping the partials and weights
             const uint64_t stream_policy = ptx::policy_evict_first();
             uint32_t g = 0;
@@ -311,7 +321,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                     for (int i = 0; i < 4; ++i)
                         ptx::tma_load_2d_hint(dst + i * kChunkBytes, &tm_cache, &tile_full[s], 256 * (int)rank + 64 * i,
                                               row, stream_policy);
-                    ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_cache, &tile_full[s], 512, row, stream_policy);
+                    ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_rope, &tile_full[s], 512 + 32 * (int)rank, row,
+                                          stream_policy);
                 }
             }
             // All tiles requested: pull this CTA's share of the next kernel's weights (W_UV)
@@ -353,15 +364,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
             uint32_t idle = 0;
             while (o_have) {
                 // ---- O of tile g
-                if (g < s_g && ptx::mbar_test(p_ready, g & 1)) {
+                if (g < s_g && ptx::mbar_test(&p_ready[g & 1], (g >> 1) & 1)) {
                     ptx::tc_fence_after();
                     const uint32_t v = ptx::smem_u32(tiles + (g % kStages) * kTileBytes);
                     const bool first = (o_j == sg.j0);
 #pragma unroll
                     for (int k = 0; k < kT / 16; ++k)
-                        ptx::mma_ts(tmem + kColO, tmem + kColP + 8 * k,
+                        ptx::mma_ts(tmem + kColO, tmem + kColP + 32 * (g & 1) + 8 * k,
                                     ptx::desc_mnmajor_sw128(v + 2048 * k, kChunkBytes), idesc_o, !(first && k == 0));
-                    ptx::mma_commit(o_done);
+                    ptx::mma_commit(&o_done[g & 1]);
                     ptx::mma_commit(&tile_empty[g % kStages]);
                     ++g;
                     if (++o_j == sg.j1) {
@@ -390,8 +401,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                                         ks != 0);
 #pragma unroll
                         for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
-                            ptx::mma_ts(tmem + kColS, tmem + kColQ + 128 + 8 * ks,
-                                        ptx::desc_kmajor_sw128(t + 4 * kChunkBytes + 64 * rank + 32 * ks), idesc_s, 1);
+                            ptx::mma_ss(tmem + kColS, ptx::desc_kmajor_sw64(ptx::smem_u32(qrope) + 32 * ks),
+                                        ptx::desc_kmajor_sw64(t + 4 * kChunkBytes + 32 * ks), idesc_s, 1);
                         ptx::mma_commit(s_full);
                         ++s_g;
                         q_ok = false;
@@ -436,7 +447,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
         uint32_t g = 0;
         if (sender) {
             // ------------------------------------------------------- score senders
-            // Q_r of sequence b -> TMEM: 256 latent columns + 32 rotary columns of this head
+            // Q_r of sequence b: 256 latent columns of this head -> TMEM, 32 rotary columns -> smem
             auto load_q = [&](int b) {
                 const uint4* ql = (const uint4*)(q_lat + ((long long)b * 128 + h) * 512 + 256 * rank);
                 const uint4* qr = (const uint4*)(q_rope + b * sQr_b + h * sQr_h + 32 * rank);
@@ -450,13 +461,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                     }
                     ptx::tmem_st32(lane_addr + kColQ + 32 * c, r);
                 }
-                uint32_t r16[16];
+                // rotary part: row h of the shared-memory A operand (64 B, 64-byte swizzle)
 #pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 x = qr[v];
-                    r16[4 * v] = x.x; r16[4 * v + 1] = x.y; r16[4 * v + 2] = x.z; r16[4 * v + 3] = x.w;
-                }
-                ptx::tmem_st16(lane_addr + kColQ + 128, r16);
+                for (int v = 0; v < 4; ++v) *(uint4*)(qrope + h * 64 + ((v ^ ((h >> 1) & 3)) << 4)) = qr[v];
+                ptx::fence_proxy_async_smem();   // read by the tensor cores
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(q_ready);
@@ -586,10 +594,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                     pw[i / 2] = ptx::pack_bf16(p0, p1);
                 }
                 l_run = l_run * alpha + sum;
-                // P (TMEM) and O are free once the previous tile's O MMA has completed
-                if (g > 0 && !uwait(o_done, (g - 1) & 1)) { ok = false; break; }
+                const uint32_t pb = g & 1;
+                // P buffer pb is free once O of tile g - 2 has completed
+                if (g >= 2 && !uwait(&o_done[pb], ((g - 2) >> 1) & 1)) { ok = false; break; }
                 ptx::tc_fence_after();
                 if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
+                    // O is scaled only once it holds every earlier tile (rare: the running max
+                    // moves only when a tile exceeds it by more than the threshold)
+                    if (g >= 1 && !uwait(&o_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) { ok = false; break; }
+                    ptx::tc_fence_after();
                     const float a = first ? 1.f : alpha;
 #pragma unroll 1
                     for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
@@ -601,16 +614,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __nv_bfloat
                         ptx::tmem_st32(lane_addr + kColO + c0, r);
                     }
                 }
-                ptx::tmem_st16(lane_addr + kColP + 16 * half, pw);
+                ptx::tmem_st16(lane_addr + kColP + 32 * pb + 16 * half, pw);
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::mbar_arrive(p_ready);
+                ptx::mbar_arrive(&p_ready[pb]);
                 if (j + 1 == cur.j1) {
                     // piece epilogue: un-normalised O_r -> part_o[slot][h][c] (each half
                     // writes 128 columns); (m, l) from CTA 0
                     const float l_all = l_run + pair_exchange(l_run);
                     if (!ok) break;
-                    if (!uwait(o_done, g & 1)) { ok = false; break; }
+                    if (!uwait(&o_done[g & 1], (g >> 1) & 1)) { ok = false; break; }
                     ptx::tc_fence_after();
                     // fragment order: four threads hold 32 contiguous bytes of one head's row,
                     // so every store instruction writes whole sectors
@@ -1027,14 +1040,17 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     }
     {
         ProfScope ps(s, "tc_flash_decode");
-        CUtensorMap m;
+        CUtensorMap m, mr;
         const uint64_t dims[2] = {576, (uint64_t)cache_rows};
         const uint64_t strides[1] = {576 * 2};
         const uint32_t box[2] = {64, (uint32_t)kT};
-        if (!make_tmap_bf16(&m, cache, 2, dims, strides, box)) return cudaErrorInvalidValue;
+        const uint32_t box_rope[2] = {32, (uint32_t)kT};
+        if (!make_tmap_bf16(&m, cache, 2, dims, strides, box) ||
+            !make_tmap_bf16(&mr, cache, 2, dims, strides, box_rope, 64))
+            return cudaErrorInvalidValue;
         static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
         if (attr != cudaSuccess) return attr;
-        if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, ws.q_lat, qr, sQr_b, sQr_h,
+        if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
                             offsets, B, (long long)cache_rows, ws.work, scale * 1.4426950408889634f,
                             ws.part_o, ws.part_ml, (const uint8_t*)W_UV, 128LL * 128 * 512 * 2, err_code,
                             err_detail)) != cudaSuccess)

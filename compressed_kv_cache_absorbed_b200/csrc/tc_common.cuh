@@ -288,14 +288,17 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 
 // ----------------------------------------------------------- MMA descriptors
 // Shared-memory matrix descriptor (Blackwell, version 1): start address, leading and
-// stride byte offsets (all >> 4), swizzle mode in bits 61-63 (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+// stride byte offsets (all >> 4), swizzle mode in bits 61-63 (2 = 128-byte, 4 = 64-byte).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout = 2) {
     return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
 }
 // K-major operand in 128-byte-swizzled atoms: rows of 64 bf16 (128 B), 8-row groups
 // 1024 B apart.  Advance `saddr` by 32 B per 16-element K step inside an atom.
 __device__ __forceinline__ uint64_t desc_kmajor_sw128(uint32_t saddr) { return smem_desc(saddr, 16, 1024); }
+// K-major operand in 64-byte-swizzled atoms: rows of 32 bf16 (64 B), 8-row groups 512 B
+// apart; 16-byte unit u of row r sits at unit u ^ ((r >> 1) & 3).  Advance 32 B per K step.
+__device__ __forceinline__ uint64_t desc_kmajor_sw64(uint32_t saddr) { return smem_desc(saddr, 16, 512, 4); }
 // MN-major operand in 128-byte-swizzled atoms: 64 contiguous MN elements per 128-B row,
 // 8 K-rows per 1024-B atom; `mn_group_bytes` = distance between 64-element MN groups.
 __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t saddr, uint32_t mn_group_bytes) {
@@ -316,7 +319,8 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
 
 // --------------------------------------------------------------- host: TMA maps
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+// swizzle_bytes: 128 (default) or 64; the box's inner extent must not exceed it.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
-                    const uint64_t* strides_bytes, const uint32_t* box);
+                    const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
 
 }  // namespace mla
