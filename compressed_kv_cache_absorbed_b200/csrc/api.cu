@@ -58,6 +58,8 @@ struct mla_weights_s {
     void* W_UK;    // [H, qk_nope, d_c]   copy, storage type
     void* W_UKT;   // [H, d_c, qk_nope]   per-head transpose (K-major for the q absorption)
     void* W_UV;    // [H, v_head, d_c]    copy
+    void* ukt_tiled;   // W_UKT and W_UV as the tensor-core kernels' shared-memory images
+    void* uv_tiled;    //   (bf16 V2/V3 head shape only; else null)
     const void* W_Q;
     const void* W_O;
 };
@@ -186,10 +188,26 @@ extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, co
         e = d->dtype == MLA_BF16
                 ? mla::launch_transpose_heads((const bf16*)W_UK, (bf16*)w->W_UKT, d->H, d->qk_nope, d->d_c, s)
                 : mla::launch_transpose_heads((const float*)W_UK, (float*)w->W_UKT, d->H, d->qk_nope, d->d_c, s);
+    if (e == cudaSuccess && tc_decode_ok(d)) {
+        if (cudaMalloc(&w->ukt_tiled, mla::tc::kTiledWeightBytes) != cudaSuccess ||
+            cudaMalloc(&w->uv_tiled, mla::tc::kTiledWeightBytes) != cudaSuccess) {
+            cudaGetLastError();
+            cudaFree(w->ukt_tiled);
+            cudaFree(w->W_UK);
+            cudaFree(w->W_UKT);
+            cudaFree(w->W_UV);
+            delete w;
+            return MLA_ERR_NO_MEMORY;
+        }
+        e = mla::tc::tile_weights_tc((const bf16*)w->W_UKT, (const bf16*)w->W_UV, (bf16*)w->ukt_tiled,
+                                     (bf16*)w->uv_tiled, s);
+    }
     if (e != cudaSuccess) {
         cudaFree(w->W_UK);
         cudaFree(w->W_UKT);
         cudaFree(w->W_UV);
+        cudaFree(w->ukt_tiled);
+        cudaFree(w->uv_tiled);
         delete w;
         return cuda_fail(e, "mla_absorb_weights");
     }
@@ -203,6 +221,8 @@ extern "C" mla_status mla_weights_destroy(mla_weights w) {
     cudaFree(w->W_UK);
     cudaFree(w->W_UKT);
     cudaFree(w->W_UV);
+    cudaFree(w->ukt_tiled);
+    cudaFree(w->uv_tiled);
     delete w;
     return MLA_OK;
 }
@@ -329,7 +349,7 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     T* o_dst = w->W_O ? (T*)ws.o_buf : (T*)out;
     if (tc_path) {
         e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
-                                        (const bf16*)w->W_UKT, (const bf16*)w->W_UV,
+                                        (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
                                         (const bf16*)cache, cache_rows, offsets, B, scale_of(d), (bf16*)o_dst,
                                         ws.tc, num_sms(), err.code, err.detail, s);
     } else {

@@ -668,8 +668,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 // ------------------------------------------------------------- merge + W_UV
 // o[b,h,:] = W_UV[h] o_lat[b,h,:],  o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[h,c] / sum_p 2^(m_p - M) l_p
 // over the pieces p of sequence b (M = max_p m_p; an empty sequence gives o = 0).
-// One CTA per (head h, block of BN sequences).  Thread 0 starts the TMA loads of W_UV[h]
-// (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
+// One CTA per (head h, block of BN sequences).  Thread 0 starts the bulk loads of the tiled
+// W_UV[h] (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
 // then merge the partials of their rows (warp per row, lane per 16 columns) straight into
 // the B operand in shared memory (K-major, 128-byte swizzle, as TMA would lay it out);
 // one thread issues the 32 MMAs (M = 128, N = BN) and four warps store D = o[:, h, :]^T.
@@ -681,7 +681,7 @@ constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kMergeThreads, 1)
-merge_wuv_kernel(const __grid_constant__ CUtensorMap tm_wuv, const int32_t* __restrict__ work, int B,
+merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict__ work, int B,
                  const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
@@ -698,11 +698,12 @@ merge_wuv_kernel(const __grid_constant__ CUtensorMap tm_wuv, const int32_t* __re
         ptx::mbar_init(a_full, 1);
         ptx::mbar_init(d_full, 1);
         ptx::fence_mbar_init();
-        ptx::tma_prefetch(&tm_wuv);
-        // the weights are not written by earlier kernels: load them before waiting
+        // the weights are not written by earlier kernels: load them before waiting; the tiled
+        // copy is already the shared-memory image, 8 contiguous 16 KB chunks per head
         ptx::mbar_expect_tx(a_full, kMergeABytes);
+        const uint8_t* src = (const uint8_t*)uv + (size_t)h * kMergeABytes;
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) ptx::tma_load_2d(sA + kc * 16384, &tm_wuv, a_full, 64 * kc, 128 * h);
+        for (int kc = 0; kc < 8; ++kc) ptx::bulk_load(sA + kc * 16384, src + kc * 16384, 16384, a_full);
     }
     if (warp == 1) {
         ptx::tmem_alloc(tmem_slot, BN);
@@ -826,24 +827,50 @@ merge_wuv_kernel(const __grid_constant__ CUtensorMap tm_wuv, const int32_t* __re
             if (lane == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 8100000 + h);
         } else {
             ptx::tc_fence_after();
-            const int m = warp * 32 + lane;   // output row = TMEM lane
+            // D (row m = TMEM lane, column = sequence) -> bf16 stage[b][m] in the A buffer
+            // (free once the MMAs completed), then whole 256-byte rows o[b, h, :]
+            const int m = warp * 32 + lane;
+            __nv_bfloat16* stage = (__nv_bfloat16*)sA;
 #pragma unroll
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t r[32];
                 ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + c0, r);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int b = n0 + c0 + j;
-                    if (b < B) o[b * sO_b + h * sO_h + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
-                }
+                for (int j = 0; j < 32; ++j) stage[(c0 + j) * 128 + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
+        }
+        ptx::named_barrier_sync(1, 128);   // the four epilogue warps
+        for (int i = threadIdx.x; i < BN * 16; i += 128) {
+            const int b = n0 + (i >> 4);
+            if (b < B) ((uint4*)(o + b * sO_b + h * sO_h))[i & 15] = ((const uint4*)sA)[i];
         }
     }
     (void)ok;
     ptx::tc_fence_before();
     __syncthreads();
     if (warp == 1) ptx::tmem_dealloc(tmem, BN);
+}
+
+// ------------------------------------------------------------- weight tiling
+// One thread per 16-byte unit of the tiled copies: unit u of row r of chunk c of head h goes
+// to unit u ^ (r % 8) of that row (the 128-byte swizzle of a 1024-byte-aligned operand).
+__global__ void __launch_bounds__(256)
+tile_weights_kernel(const __nv_bfloat16* __restrict__ W_UKT, const __nv_bfloat16* __restrict__ W_UV,
+                    __nv_bfloat16* __restrict__ ukt, __nv_bfloat16* __restrict__ uv) {
+    const long long n = (long long)kH * 8 * 128 * 8;   // units per tensor
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < 2 * n; i += (long long)gridDim.x * blockDim.x) {
+        const bool is_uv = i >= n;
+        const long long k = is_uv ? i - n : i;
+        const int u = (int)(k & 7), r = (int)((k >> 3) & 127), c = (int)((k >> 10) & 7), h = (int)(k >> 13);
+        const uint4* src;
+        if (!is_uv)   // chunk c = 2t + kk: W_UK^T[h][128t + r][64kk + 8u ..]
+            src = (const uint4*)(W_UKT + ((long long)h * kDc + 128 * (c >> 1) + r) * 128 + 64 * (c & 1) + 8 * u);
+        else          // chunk c: W_UV[h][r][64c + 8u ..]
+            src = (const uint4*)(W_UV + ((long long)h * 128 + r) * kDc + 64 * c + 8 * u);
+        uint4* dst = (uint4*)((is_uv ? uv : ukt) + (((long long)h * 8 + c) * 128 + r) * 64) + (u ^ (r & 7));
+        *dst = *src;
+    }
 }
 
 // Kernel attributes, set once per kernel: the dynamic shared memory it needs, and the
@@ -860,7 +887,7 @@ cudaError_t set_smem_attrs(K kernel, int bytes) {
 // ----------------------------------------------------------------- q absorption
 // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:], as D[512 x BN] = W_UK^T[h] (512 x 128) . Q_h^T with
 // Q_h = q_nope[n0 .. n0+BN, h, :].  One CTA per (head, block of BN sequences) holds the whole
-// W_UK^T[h] (8 TMA boxes of 128 x 64, 128 KB) and Q_h (2 boxes), issues 4 x 8 MMAs into four
+// W_UK^T[h] (8 contiguous 16 KB chunks of the tiled copy, 128 KB) and Q_h (2 TMA boxes), issues 4 x 8 MMAs into four
 // BN-column TMEM accumulators (one per 128-row tile) and stores q_lat.
 // This is the first kernel of the decode chain: it waits for all earlier work before it lets
 // the next kernel launch (the decode kernel then reads the cache without waiting).
@@ -871,7 +898,7 @@ constexpr int absorb_smem() { return 8 * 16384 + 2 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kAbsorbThreads, 1)
-absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_q, int B,
+absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ CUtensorMap tm_q, int B,
                 __nv_bfloat16* __restrict__ q_lat, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t absorb_smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)absorb_smem_raw + 1023) & ~(uintptr_t)1023);
@@ -887,15 +914,13 @@ absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         ptx::mbar_init(full, 1);
         ptx::mbar_init(d_full, 1);
         ptx::fence_mbar_init();
-        ptx::tma_prefetch(&tm_w);
         ptx::tma_prefetch(&tm_q);
         ptx::mbar_expect_tx(full, 8 * 16384 + 2 * BN * 128);
-        // weights first: earlier kernels do not write them
+        // weights first (earlier kernels do not write them): the tiled copy is already the
+        // shared-memory image, chunk (t, k) at (2t + k) x 16 KB
+        const uint8_t* src = (const uint8_t*)ukt + (size_t)h * 8 * 16384;
 #pragma unroll
-        for (int mt = 0; mt < 4; ++mt)
-#pragma unroll
-            for (int kc = 0; kc < 2; ++kc)
-                ptx::tma_load_2d(sA + (mt * 2 + kc) * 16384, &tm_w, full, 64 * kc, 512 * h + 128 * mt);
+        for (int c = 0; c < 8; ++c) ptx::bulk_load(sA + c * 16384, src + c * 16384, 16384, full);
         pdl_wait();      // the queries may come from the previous kernel; all earlier work is done
         pdl_trigger();   // only now may the next kernel launch
 #pragma unroll
@@ -931,7 +956,10 @@ absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
         if (lane == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 8300000 + h);
     } else {
         ptx::tc_fence_after();
+        // D (row = latent index, column = sequence) -> bf16 stage[b][512] in the A buffer (free
+        // once the MMAs completed), then whole 1 KB rows q_lat[b, h, :]
         const int m = warp * 32 + lane;   // row of the 128-row tile = TMEM lane
+        __nv_bfloat16* stage = (__nv_bfloat16*)sA;
 #pragma unroll 1
         for (int mt = 0; mt < 4; ++mt)
 #pragma unroll
@@ -940,12 +968,13 @@ absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
                 ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) {
-                    const int b = n0 + c0 + j;
-                    if (b < B)
-                        q_lat[((long long)b * 128 + h) * 512 + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
-                }
+                for (int j = 0; j < 32; ++j) stage[(c0 + j) * 512 + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < BN * 64; i += kAbsorbThreads) {
+        const int b = n0 + (i >> 6);
+        if (b < B) ((uint4*)(q_lat + ((long long)b * 128 + h) * 512))[i & 63] = ((const uint4*)sA)[i];
     }
     ptx::tc_fence_before();
     __syncthreads();
@@ -953,12 +982,12 @@ absorb_q_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant_
 }
 
 template <int BN>
-cudaError_t launch_absorb(const CUtensorMap& mw, const CUtensorMap& mq, int B, __nv_bfloat16* q_lat, int* err_code,
+cudaError_t launch_absorb(const __nv_bfloat16* ukt, const CUtensorMap& mq, int B, __nv_bfloat16* q_lat, int* err_code,
                           long long* err_detail, cudaStream_t s) {
     static const cudaError_t attr = set_smem_attrs(absorb_q_kernel<BN>, absorb_smem<BN>());
     if (attr != cudaSuccess) return attr;
     return launch_pdl(absorb_q_kernel<BN>, dim3(128, (B + BN - 1) / BN), dim3(kAbsorbThreads), absorb_smem<BN>(), s,
-                      mw, mq, B, q_lat, err_code, err_detail);
+                      ukt, mq, B, q_lat, err_code, err_detail);
 }
 
 int g_clusters_cached = 0;
@@ -980,6 +1009,12 @@ int max_clusters(int num_sms) {
 }
 
 }  // namespace
+
+cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
+                            __nv_bfloat16* uv, cudaStream_t s) {
+    tile_weights_kernel<<<1184, 256, 0, s>>>(W_UKT, W_UV, ukt, uv);
+    return cudaGetLastError();
+}
 
 size_t decode_ws_bytes(int B, int num_sms) {
     const size_t P = (size_t)(num_sms / 2);
@@ -1011,8 +1046,8 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
 }
 
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h, const __nv_bfloat16* qr,
-                               long long sQr_b, long long sQr_h, const __nv_bfloat16* W_UKT,
-                               const __nv_bfloat16* W_UV, const __nv_bfloat16* cache, long long cache_rows,
+                               long long sQr_b, long long sQr_h, const __nv_bfloat16* ukt,
+                               const __nv_bfloat16* uv, const __nv_bfloat16* cache, long long cache_rows,
                                const int32_t* offsets, int B, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s) {
@@ -1023,19 +1058,15 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     {
         // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]
         ProfScope ps(s, "tc_q_absorb");
-        CUtensorMap mw, mq;
-        const uint64_t dw[2] = {128, 128ull * 512};
-        const uint64_t sw[1] = {128 * 2};
-        const uint32_t bw[2] = {64, 128};
+        CUtensorMap mq;
         const int BN = B <= 32 ? 32 : B <= 64 ? 64 : 128;
         const uint64_t dq[3] = {128, (uint64_t)B, 128};
         const uint64_t sq[2] = {(uint64_t)sQn_b * 2, (uint64_t)sQn_h * 2};
         const uint32_t bq[3] = {64, (uint32_t)BN, 1};
-        if (!make_tmap_bf16(&mw, W_UKT, 2, dw, sw, bw) || !make_tmap_bf16(&mq, qn, 3, dq, sq, bq))
-            return cudaErrorInvalidValue;
-        e = BN == 32   ? launch_absorb<32>(mw, mq, B, ws.q_lat, err_code, err_detail, s)
-            : BN == 64 ? launch_absorb<64>(mw, mq, B, ws.q_lat, err_code, err_detail, s)
-                       : launch_absorb<128>(mw, mq, B, ws.q_lat, err_code, err_detail, s);
+        if (!make_tmap_bf16(&mq, qn, 3, dq, sq, bq)) return cudaErrorInvalidValue;
+        e = BN == 32   ? launch_absorb<32>(ukt, mq, B, ws.q_lat, err_code, err_detail, s)
+            : BN == 64 ? launch_absorb<64>(ukt, mq, B, ws.q_lat, err_code, err_detail, s)
+                       : launch_absorb<128>(ukt, mq, B, ws.q_lat, err_code, err_detail, s);
         if (e != cudaSuccess) return e;
     }
     {
@@ -1052,29 +1083,24 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         if (attr != cudaSuccess) return attr;
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
                             offsets, B, (long long)cache_rows, ws.work, scale * 1.4426950408889634f,
-                            ws.part_o, ws.part_ml, (const uint8_t*)W_UV, 128LL * 128 * 512 * 2, err_code,
+                            ws.part_o, ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code,
                             err_detail)) != cudaSuccess)
             return e;
     }
     {
         // merge of the pieces fused with o[b,h,:] = W_UV[h] o_lat[b,h,:]
         ProfScope ps(s, "tc_merge_w_uv");
-        CUtensorMap m;
-        const uint64_t dims[2] = {512, 128ull * 128};
-        const uint64_t strides[1] = {512 * 2};
-        const uint32_t box[2] = {64, 128};
-        if (!make_tmap_bf16(&m, W_UV, 2, dims, strides, box)) return cudaErrorInvalidValue;
         if (B <= 32) {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
             if (attr != cudaSuccess) return attr;
-            e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, m,
+            e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
                            (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         } else {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                           m, (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           uv, (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         }
     }

@@ -20,21 +20,34 @@ constexpr bool kEnabled = true;
 struct DecodeWs {
     __nv_bfloat16* q_lat;   // [B, H, d_c] absorbed query, bf16
     __nv_bfloat16* q_cat;   // unused
-    float* part_o;          // [max_parts, d_c, H] un-normalised partial o_lat
+    float* part_o;          // [max_parts, H, d_c] un-normalised partial o_lat
     float* part_ml;         // [max_parts, H, 2] running max (log2 domain) and sum
-    int32_t* work;          // split plan: totals, first tile and first partial slot per sequence
-    __nv_bfloat16* o_lat;   // [B, H, d_c] merged, normalised o_lat (bf16, W_UV operand)
+    int32_t* work;          // split plan: totals and the first tile of each sequence
+    __nv_bfloat16* o_lat;   // unused
     int max_parts;
 };
 
 size_t decode_ws_bytes(int B, int num_sms);
 DecodeWs carve_decode_ws(char* base, int B, int num_sms);
 
+// Bytes of one tiled weight tensor (W_UK^T or W_UV) for the tensor-core kernels.
+constexpr size_t kTiledWeightBytes = (size_t)kH * kDc * 128 * 2;
+
+// The weights laid out as the shared-memory operand images of the q-absorb and merge
+// kernels, so that a CTA loads a head's matrix with contiguous bulk copies: per head, 8
+// chunks of 128 rows x 64 columns (16 KB), each row 128 bytes with its 16-byte units in the
+// 128-byte-swizzle order (unit u of row r at u ^ (r % 8)).
+//   ukt: chunk (t, k) = rows 128t .. +127 of W_UK^T[h] (latent index), columns 64k .. +63 (qk_nope)
+//   uv:  chunk k      = rows 0 .. 127 of W_UV[h] (v_head), columns 64k .. +63 (latent)
+// W_UKT [H, d_c, qk_nope] and W_UV [H, v_head, d_c] are the plain layouts.
+cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
+                            __nv_bfloat16* uv, cudaStream_t s);
+
 // q_nope rows at qn + b*sQn_b + h*sQn_h (qk_nope = 128), q_rope rows at qr + b*sQr_b + h*sQr_h.
-// W_UKT [H, d_c, qk_nope]; W_UV [H, v_head = 128, d_c]; out o [B, H, 128] bf16.
+// ukt / uv: the tiled weights written by tile_weights_tc; out o [B, H, 128] bf16.
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
-                               const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV,
+                               const __nv_bfloat16* ukt, const __nv_bfloat16* uv,
                                const __nv_bfloat16* cache, long long cache_rows, const int32_t* offsets,
                                int B, float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s);

@@ -150,6 +150,15 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
+// Contiguous global -> shared copy (16-byte aligned, size a multiple of 16) that completes
+// `bytes` of transaction on `bar`.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_u32(dst)),
+                 "l"((uint64_t)src), "r"(bytes), "r"(smem_u32(bar))
+                 : "memory");
+}
+
 // L2 eviction policies for cache hints: data read once (evict first) or wanted again soon
 // (evict last).
 __device__ __forceinline__ uint64_t policy_evict_first() {
