@@ -66,11 +66,20 @@ constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols =
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 softmax warps
 
-// Plan written by CTA 0 for the merge kernel (int32): [0] total tiles, [1] tiles per cluster,
-// [2] clusters, [4, 4+B+1) first tile of each sequence (the last entry is the total).
-__device__ __forceinline__ const int32_t* plan_tstart(const int32_t* w) { return w + 4; }
+// The work split counts cost units: one per tile plus kPieceCost for every sequence start
+// (a new piece costs its partial's epilogue and a query reload, measured at about three
+// tiles), so clusters whose range starts sequences get fewer tiles.  Tile j of sequence b
+// sits at cost position first[b] + j, with first[b] = (cost of all earlier sequences) +
+// kPieceCost.
+constexpr int kPieceCost = 3;
+
+// Plan written by CTA 0 for the merge kernel (int32): [0] total cost, [1] cost units per
+// cluster, [2] clusters, [4, 4+B) first[b], [4+B+1, 4+2B+1) first[b] + tiles of b.
+__device__ __forceinline__ const int32_t* plan_first_pos(const int32_t* w) { return w + 4; }
+__device__ __forceinline__ const int32_t* plan_end_pos(const int32_t* w, int B) { return w + 4 + B + 1; }
 
 __device__ __forceinline__ int tiles_of_len(int L) { return L > 0 ? (L + kT - 1) / kT : 0; }
+__device__ __forceinline__ int cost_of_tiles(int n) { return n > 0 ? n + kPieceCost : 0; }
 
 __device__ __forceinline__ uint32_t cluster_rank() {
     uint32_t r;
@@ -103,29 +112,33 @@ struct Seg {
     long long row0;
 };
 
-// Walks the pieces of sequences in this cluster's tile range [lo, hi), in sequence order,
-// starting from the sequence that holds tile lo (first tile t0).  The same walk runs in
-// every role of both CTAs.  Partial slots: a piece that starts at its sequence's first tile
-// takes slot b; the one piece of a cluster that continues a sequence begun in an earlier
-// cluster takes slot B + cluster.  So B + clusters slots suffice and need no prefix sums.
+// Walks the pieces of sequences in this cluster's cost range [lo, hi), in sequence order,
+// starting from the sequence whose cost region holds lo (cost start cs).  The same walk runs
+// in every role of both CTAs.  Partial slots: a piece that starts at its sequence's first
+// tile takes slot b; the one piece of a cluster that continues a sequence begun in an
+// earlier cluster takes slot B + cluster.  So B + clusters slots suffice.
 struct SegIter {
     const int32_t* offsets;
-    int B, lo, hi, cluster, b, t0;
+    int B, lo, hi, cluster, b, cs;
     __device__ bool next(Seg& s) {
-        while (b < B && t0 < hi) {
+        while (b < B && cs < hi) {
             const int r0 = offsets[b], r1 = offsets[b + 1];
             const int L = r1 > r0 ? r1 - r0 : 0;
-            const int t1 = t0 + tiles_of_len(L);
-            const int bb = b, tt0 = t0;
+            const int n = tiles_of_len(L);
+            const int f = cs + kPieceCost;   // cost position of tile 0
+            const int bb = b;
             ++b;
-            t0 = t1;
-            if (t1 > lo && t1 > tt0) {
+            cs += cost_of_tiles(n);
+            if (n == 0) continue;
+            const int j0 = lo > f ? lo - f : 0;
+            const int j1 = hi - f < n ? hi - f : n;
+            if (j0 < j1) {
                 s.b = bb;
-                s.j0 = (lo > tt0 ? lo : tt0) - tt0;
-                s.j1 = (hi < t1 ? hi : t1) - tt0;
+                s.j0 = j0;
+                s.j1 = j1;
                 s.row0 = r0;
                 s.L = L;
-                s.slot = tt0 >= lo ? bb : B + cluster;
+                s.slot = j0 == 0 ? bb : B + cluster;
                 return true;
             }
         }
@@ -235,7 +248,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         for (int b = threadIdx.x; b < B; b += kThreads) {
             const int L = b == (int)threadIdx.x ? len0 : offsets[b + 1] - offsets[b];
             if (L < 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
-            mine += tiles_of_len(L);
+            mine += cost_of_tiles(tiles_of_len(L));
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, o);
@@ -251,13 +264,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     }
     const int per = total > 0 ? (total + P - 1) / P : 1;
     const int lo = cluster * per, hi = min(total, lo + per);
-    const bool writer = blockIdx.x == 0;   // publishes every sequence's first tile for the merge
+    const bool writer = blockIdx.x == 0;   // publishes every sequence's tile positions for the merge
     if (lo < total || writer) {
         int carry = 0;
         for (int c0 = 0; c0 < B; c0 += kThreads) {
             const int b = c0 + (int)threadIdx.x;
             const int n = b < B ? tiles_of_len(c0 == 0 ? len0 : offsets[b + 1] - offsets[b]) : 0;
-            int incl = n;
+            const int cb = cost_of_tiles(n);
+            int incl = cb;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const int v = __shfl_up_sync(0xffffffffu, incl, o);
@@ -272,12 +286,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                 before += i < warp ? v : 0;
                 chunk += v;
             }
-            const int t0 = before + incl - n;
+            const int cs = before + incl - cb;   // cost of the sequences before b
             if (b < B) {
-                if (writer) work[4 + b] = t0;
-                if (n > 0 && t0 <= lo && lo < t0 + n) {   // unique: the sequence holding tile lo
+                if (writer) {
+                    work[4 + b] = cs + kPieceCost;
+                    work[4 + B + 1 + b] = cs + kPieceCost + n;
+                }
+                if (cb > 0 && cs <= lo && lo < cs + cb) {   // unique: the cost region holding lo
                     plan_first[0] = b;
-                    plan_first[1] = t0;
+                    plan_first[1] = cs;
                 }
             }
             carry += chunk;
@@ -288,7 +305,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         work[0] = total;
         work[1] = per;
         work[2] = P;
-        work[4 + B] = total;
     }
     SegIter it{offsets, B, lo, hi, cluster, plan_first[0], plan_first[1]};
     Seg sg;
@@ -712,7 +728,8 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict
     if (threadIdx.x == 0) pdl_trigger();
     pdl_wait();   // the partials and the plan come from the decode kernel
 
-    const int32_t* ts = plan_tstart(work);
+    const int32_t* fpos = plan_first_pos(work);
+    const int32_t* epos = plan_end_pos(work, B);
     const int per = work[1];
     constexpr int kW = kMergeThreads / 32;
     constexpr int kRowsPerWarp = BN / kW;
@@ -721,8 +738,8 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         const int b = n0 + warp + kW * i;
-        t0r[i] = b < B ? ts[b] : 0;
-        t1r[i] = b < B ? ts[b + 1] : 0;
+        t0r[i] = b < B ? fpos[b] : 0;   // cost positions of the first and one past the last tile
+        t1r[i] = b < B ? epos[b] : 0;
     }
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
