@@ -55,6 +55,34 @@ def alg_step(w: workloads.Workload) -> dict:
             "attn_flops": flops_attn, "tokens": tokens}
 
 
+def alg_layer(w: workloads.Workload) -> dict:
+    """Bytes and flops of one full decode-layer step: append the new token, project the
+    query, absorbed attention over L + 1 rows, W_UV, W_O."""
+    L = workloads.lengths(w) + 1
+    tokens = int(L.sum())
+    e = 2 if w.dtype == "bf16" else 4
+    qh = w.qk_nope + w.d_hR
+    w_bytes = (w.row * w.d_model + w.H * qh * w.d_model + w.d_model * w.H * w.v_head
+               + 2 * w.H * w.qk_nope * w.d_c) * e
+    act = (w.B * w.d_model * 2 + w.B * w.row) * e
+    flops = (2 * w.B * w.d_model * (w.row + w.H * qh) + tokens * w.H * (2 * w.row + 2 * w.d_c)
+             + 4 * w.B * w.H * w.qk_nope * w.d_c + 2 * w.B * w.H * w.v_head * w.d_model)
+    return {"bytes": tokens * w.row * e + w_bytes + act, "flops": flops, "tokens": w.B}
+
+
+def alg_prefill(w: workloads.Workload) -> dict:
+    """Bytes and flops of one causal prefill step (K/V materialised)."""
+    n = w.B * w.ctx
+    e = 2
+    qh = w.qk_nope + w.d_hR
+    w_bytes = (w.row * w.d_model + w.H * qh * w.d_model + 2 * w.H * w.qk_nope * w.d_c) * e
+    io = (n * w.d_model + n * w.row + n * w.H * w.v_head) * e
+    causal_pairs = w.B * w.ctx * (w.ctx + 1) // 2
+    flops = (2 * n * w.d_model * (w.row + w.H * qh) + 2 * n * w.d_c * w.H * (w.qk_nope + w.v_head)
+             + causal_pairs * w.H * 2 * (qh + w.v_head))
+    return {"bytes": w_bytes + io, "flops": flops, "tokens": n}
+
+
 def alg_kernel_bytes(name: str, w: workloads.Workload) -> int:
     """Algorithmic bytes of one launch of the kernel that dominates the step: the cache rows
     it attends over (1152 B per token) plus the queries it reads."""
@@ -243,23 +271,62 @@ def config_of(w, world):
             "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write, outside the step events)"}
 
 
+def build_step(w, inp, dev, mla):
+    """Device inputs, the library call of one step, and what an end-to-end step copies."""
+    g = {k: v.to(dev) for k, v in inp.items()}
+    dims = mla.make_dims(w.H, w.d_model, w.d_c, w.d_hR, w.qk_nope, w.v_head, w.dtype)
+    dt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+    if w.kind == "decode_attn":
+        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+        out = torch.empty(w.B, w.H, w.v_head, dtype=dt, device=dev)
+        ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
+
+        def step():
+            mla.mla_decode_absorbed(dims, weights, g["cache"], g["offsets"], out, ws, q_nope=g["q_nope"],
+                                    q_rope=g["q_rope"])
+        h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
+        return g, dims, weights, out, step, h2d, alg_step(w), w.B
+    if w.kind == "decode_layer":
+        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"])
+        out = torch.empty(w.B, w.d_model, dtype=dt, device=dev)
+        ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
+        L = workloads.lengths(w)
+        offs = inp["offsets"].numpy().astype(np.int64)
+        q_pos = torch.from_numpy(L.astype(np.int32)).to(dev)
+        slot = torch.from_numpy(offs[:-1] + L).to(dev)
+        if w.history == "hidden":   # small fp32 layer: build the history by appending
+            cache = torch.zeros(int(offs[-1]), w.row, dtype=dt, device=dev)
+            pos = np.tile(np.arange(w.ctx), w.B).astype(np.int32)
+            hs = (offs[:-1, None] + np.arange(w.ctx)[None]).reshape(-1)
+            mla.mla_append_cache(dims, g["h_hist"].reshape(-1, w.d_model), g["W_DKV"], g["W_KR"],
+                                 torch.from_numpy(pos).to(dev), torch.from_numpy(hs).to(dev), cache)
+        else:
+            cache = g["cache"]
+
+        def step():   # append the new token at position L, then decode it over L + 1 rows
+            mla.mla_append_cache(dims, g["h_new"], g["W_DKV"], g["W_KR"], q_pos, slot, cache)
+            mla.mla_decode_absorbed(dims, weights, cache, g["offsets"], out, ws, h=g["h_new"], q_pos=q_pos)
+        return g, dims, weights, out, step, [("h_new", inp["h_new"])], alg_layer(w), w.B
+    # prefill
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"])
+    cache = torch.zeros(w.B * w.ctx, w.row, dtype=dt, device=dev)
+    out = torch.empty(w.B, w.ctx, w.H, w.v_head, dtype=dt, device=dev)
+    ws = mla.workspace(mla.mla_prefill_workspace_size(dims, w.B, w.ctx), dev)
+
+    def step():
+        mla.mla_prefill_causal(dims, weights, g["h"], g["W_DKV"], g["W_KR"], cache, out, ws)
+    return g, dims, weights, out, step, [("h", inp["h"])], alg_prefill(w), w.B * w.ctx
+
+
 def run_ours(args, w0):
     world, rank, local = dist_init()
     import compressed_kv_cache_absorbed_b200 as mla
     w = rank_workload(w0, rank)
     inp = workloads.make_inputs(w)
     dev = torch.device("cuda", local)
-    g = {k: v.to(dev) for k, v in inp.items()}
-    dims = mla.make_dims(w.H, w.d_model, w.d_c, w.d_hR, w.qk_nope, w.v_head, w.dtype)
-    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
-    out = torch.empty(w.B, w.H, w.v_head, dtype=torch.bfloat16, device=dev)
-    ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
+    g, dims, weights, out, step, h2d, a, units = build_step(w, inp, dev, mla)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
-
-    def step():
-        mla.mla_decode_absorbed(dims, weights, g["cache"], g["offsets"], out, ws, q_nope=g["q_nope"],
-                                q_rope=g["q_rope"])
 
     # warm-up
     for _ in range(args.warmup):
@@ -294,7 +361,7 @@ def run_ours(args, w0):
         if profile:
             mla.mla_profile_enable(False)
             prof = mla.mla_profile_report(reset=True)
-        return float(np.mean([a.elapsed_time(b) for a, b in ev])), prof, t0, t1
+        return float(np.mean([a_.elapsed_time(b_) for a_, b_ in ev])), prof, t0, t1
 
     # timed region: per-step CUDA events, the L2 flush between them (outside the events);
     # the library's kernels chain with programmatic dependent launch
@@ -309,9 +376,9 @@ def run_ours(args, w0):
     if clocks:
         clocks.stop()
 
-    # end to end through the same call with host buffers: H2D of the queries, D2H of o
-    qn_h = inp["q_nope"].pin_memory()
-    qr_h = inp["q_rope"].pin_memory()
+    # end to end through the same call with host buffers: H2D of the step's inputs from
+    # pinned memory, D2H of its output
+    pinned = [(g[k], v.pin_memory()) for k, v in h2d]
     out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
     ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps + args.warmup):
@@ -319,58 +386,73 @@ def run_ours(args, w0):
         j = i - args.warmup
         if j >= 0:
             ev3[j][0].record(stream)
-        g["q_nope"].copy_(qn_h, non_blocking=True)
-        g["q_rope"].copy_(qr_h, non_blocking=True)
+        for dst, src in pinned:
+            dst.copy_(src, non_blocking=True)
         step()
         out_h.copy_(out, non_blocking=True)
         if j >= 0:
             ev3[j][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(float(np.mean([a.elapsed_time(b) for a, b in ev3])))
+    e2e_ms = max_over_ranks(float(np.mean([a_.elapsed_time(b_) for a_, b_ in ev3])))
     st, det = mla.mla_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error {st} ({det})")
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kind == "decode_attn":
         cpu = time_oracle_units(w, inp, args.cpu_seconds)
         cpu.pop("step_s_extrapolated", None)
 
     if rank == 0:
-        a = alg_step(w)
         pk, pk_kind = peaks()
         dom = max(prof, key=lambda k: prof[k][1])
         n_launch, dom_ms = prof[dom]
         launch_s = dom_ms / n_launch * 1e-3
-        kbytes = alg_kernel_bytes(dom, w)
-        achieved = kbytes / launch_s / 1e9
         launches_per_step = sum(v[0] for v in prof.values()) / args.steps
         step_s = ms * 1e-3
         roof_s = max(a["bytes"] / (pk["hbm_gbs"] * 1e9), a["flops"] / (pk["bf16_tflops"] * 1e12))
+        if w.kind == "decode_attn":
+            kbytes = alg_kernel_bytes(dom, w)
+            achieved = kbytes / launch_s / 1e9
+            roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
+                        "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom),
+                        "alg_bytes_per_launch": kbytes, "launch_us": launch_s * 1e6,
+                        "peak_source": f"{pk_kind} hbm_gbs"}
+            metric, unit = METRIC, "tokens/s"
+        else:
+            # whole-step roofline: these steps chain several kernels of different bounds
+            bound = "tensor" if a["flops"] / (pk["bf16_tflops"] * 1e12) > a["bytes"] / (pk["hbm_gbs"] * 1e9) else "hbm"
+            achieved = a["flops"] / step_s / 1e12 if bound == "tensor" else a["bytes"] / step_s / 1e9
+            peak = pk["bf16_tflops"] if bound == "tensor" else pk["hbm_gbs"]
+            roofline = {"kernel": "step", "bound": bound, "achieved": achieved, "peak": peak,
+                        "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak,
+                        "traffic": None, "dominant_kernel": dom, "dominant_launch_us": launch_s * 1e6,
+                        "peak_source": f"{pk_kind} " + ("bf16_tflops" if bound == "tensor" else "hbm_gbs")}
+            metric = ("MLA decode-layer tokens/s (append + q proj + absorbed attention + W_UV + W_O)"
+                      if w.kind == "decode_layer" else "MLA causal prefill tokens/s (K/V materialised)")
+            unit = "tokens/s"
         line = {
-            "metric": METRIC, "value": world * w.B / step_s, "unit": "tokens/s", "n_gpus": world,
+            "metric": metric, "value": world * units / step_s, "unit": unit, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": config_of(w, world),
-            "latent_cache_GBps": a["cache_bytes"] / step_s / 1e9,
             "step_roofline": {"alg_bytes": a["bytes"], "alg_flops": a["flops"], "roofline_us": roof_s * 1e6,
                               "frac": roof_s / step_s, "tflops": a["flops"] / step_s / 1e12,
                               "peaks": f"{pk_kind}: hbm {pk['hbm_gbs']} GB/s, bf16 {pk['bf16_tflops']} TFLOP/s"},
-            "roofline": {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
-                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom),
-                         "alg_bytes_per_launch": kbytes, "launch_us": launch_s * 1e6,
-                         "peak_source": f"{pk_kind} hbm_gbs"},
+            "roofline": roofline,
             "kernels": {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in prof.items()},
             "ms_per_step_with_kernel_events": ms_prof,
-            "e2e": {"value": world * w.B / (e2e_ms * 1e-3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": int(inp["q_nope"].numel() * 2 + inp["q_rope"].numel() * 2),
-                    "d2h_bytes_per_step": int(out.numel() * 2), "ms_per_step": e2e_ms,
+            "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": unit,
+                    "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for _, v in h2d)),
+                    "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms,
                     "note": "latent cache and weights stay resident in HBM (decode state)"},
             "gpu_launches": int(round(launches_per_step * args.steps)),
             "clocks": clk,
             "cpu_baseline": cpu,
             "decode_path": "tcgen05" if mla.mla_decode_path(dims) == 1 else "cuda-core",
         }
+        if w.kind == "decode_attn":
+            line["latent_cache_GBps"] = a["cache_bytes"] / step_s / 1e9
         print(json.dumps(line), flush=True)
     weights.close()
     if world > 1:
@@ -393,9 +475,9 @@ def main():
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     w = workloads.WORKLOADS[args.workload]
-    if w.kind != "decode_attn":
-        ap.error("the benchmark step is the absorbed decode of a decode_attn workload")
     if args.impl == "reference":
+        if w.kind != "decode_attn":
+            ap.error("the reference arm times the oracle on the decode workloads")
         return run_reference(args, w)
     return run_ours(args, w)
 

@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "decode_tc.cuh"
+#include "gemm_tc.cuh"
 #include "mla.h"
 
 using mla::DevErr;
@@ -147,6 +148,16 @@ static bool tc_decode_ok(const mla_dims* d) {
            d->v_head == 128;
 }
 
+// The projections (append, query, W_O, prefill K/V) run on the tcgen05 GEMM for bf16 when
+// every row stride is a multiple of 16 bytes and the operands are 16-byte aligned (TMA);
+// otherwise on the CUDA-core kernels.
+static bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+static bool tc_proj_ok(const mla_dims* d) {
+    return d->dtype == MLA_BF16 && d->d_model % 8 == 0 && d->d_c % 8 == 0 && (d->d_c + d->d_hR) % 8 == 0 &&
+           (d->H * (d->qk_nope + d->d_hR)) % 8 == 0 && (d->H * d->v_head) % 8 == 0 && d->d_hR % 2 == 0 &&
+           (d->qk_nope + d->d_hR) % 2 == 0 && d->qk_nope % 2 == 0;
+}
+
 extern "C" int32_t mla_decode_path(const mla_dims* d) {
     if (dims_supported(d) != MLA_OK) return -1;
     return tc_decode_ok(d) ? 1 : 0;
@@ -229,10 +240,39 @@ extern "C" mla_status mla_weights_destroy(mla_weights w) {
 
 // ------------------------------------------------------------------------ append
 
+// [c | k_r] = h [W_DKV; W_KR]^T on the tensor cores: two GEMMs whose epilogues write the
+// cache rows (slot scatter) and rotate the k_r columns [L1 "La compresion de MLA",
+// "Truco de codificacion posicional"]
+static cudaError_t append_tc(const mla_dims* d, const void* h, const void* W_DKV, const void* W_KR,
+                             const int32_t* pos, int pos_mod, const int64_t* slot, int n, void* cache,
+                             long long capacity, DevErr err, cudaStream_t s) {
+    const int row = d->d_c + d->d_hR;
+    mla::ProfScope ps(s, "tc_append_proj_rope");
+    mla::tc::GemmOut oc{cache, 0, 1, row, 0};
+    oc.slot = slot;
+    oc.cap = capacity;
+    cudaError_t e = mla::tc::gemm_bf16_tc(1, d->d_c, n, d->d_model, (const bf16*)W_DKV, 0, d->d_model,
+                                          (const bf16*)h, 0, d->d_model, oc, err.code, err.detail, s);
+    if (e != cudaSuccess) return e;
+    mla::tc::GemmOut orope{(bf16*)cache + d->d_c, 0, 1, row, 0};
+    orope.slot = slot;
+    orope.cap = capacity;
+    orope.period = d->d_hR;
+    orope.rope_start = 0;
+    orope.d_rope = d->d_hR;
+    orope.pos = pos;
+    orope.pos_mod = pos_mod;
+    orope.theta = theta_of(d);
+    return mla::tc::gemm_bf16_tc(1, d->d_hR, n, d->d_model, (const bf16*)W_KR, 0, d->d_model, (const bf16*)h,
+                                 0, d->d_model, orope, err.code, err.detail, s);
+}
+
 template <typename T>
 static cudaError_t append_impl(const mla_dims* d, const void* h, const void* W_DKV, const void* W_KR,
                                const int32_t* pos, int pos_mod, const int64_t* slot, int n,
                                void* cache, long long capacity, DevErr err, cudaStream_t s) {
+    if (tc_proj_ok(d) && aligned16(h) && aligned16(W_DKV) && aligned16(W_KR) && aligned16(cache))
+        return append_tc(d, h, W_DKV, W_KR, pos, pos_mod, slot, n, cache, capacity, err, s);
     const int row = d->d_c + d->d_hR;
     mla::ProfScope ps(s, "simt_append_proj_rope");
     return mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)W_DKV, d->d_c,
@@ -267,6 +307,7 @@ struct DecodeWs {
     float* part_ml;  // [nsplit, B, H, 2]
     float* o_lat;    // [B, H, d_c]
     void* o_buf;     // [B, H, v_head] (storage type) when W_O follows
+    double2* rope_tab;   // [B, d_hR / 2] (cos, sin) of the query rotation (tensor-core projection)
     mla::tc::DecodeWs tc;  // tcgen05 path
     size_t bytes;
 };
@@ -277,6 +318,7 @@ static DecodeWs carve_decode(const mla_dims* d, int B, void* base, bool tc_path)
     const size_t es = esize(d), BH = (size_t)B * d->H;
     w.q_buf = c.take(BH * (d->qk_nope + d->d_hR) * es);
     w.o_buf = c.take(BH * d->v_head * es);
+    w.rope_tab = (double2*)c.take((size_t)B * (d->d_hR / 2) * sizeof(double2));
     if (tc_path) {
         w.tc = mla::tc::carve_decode_ws(c.base ? c.base + c.used : nullptr, B, num_sms());
         c.used += mla::tc::decode_ws_bytes(B, num_sms());
@@ -333,7 +375,27 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     const T* qr = (const T*)q_rope;
     long long sQn_b = (long long)H * qk, sQn_h = qk, sQr_b = (long long)H * dR, sQr_h = dR;
     cudaError_t e;
-    if (!q_nope) {
+    const bool tc_proj = tc_proj_ok(d) && (q_nope || aligned16(h)) && (q_nope || aligned16(w->W_Q)) &&
+                         (!w->W_O || (aligned16(w->W_O) && aligned16(out)));
+    if (!q_nope && tc_proj) {
+        // q = W_Q h with RoPE on each head's rotary part at q_pos [L1 "Multi-head attention estandar"]
+        const int qh = qk + dR;
+        mla::ProfScope ps(s, "tc_q_proj_rope");
+        e = mla::tc::rope_table(q_pos, 1, B, dR, theta_of(d), ws.rope_tab, s);
+        if (e != cudaSuccess) return e;
+        mla::tc::GemmOut oq{ws.q_buf, 0, 1, (long long)H * qh, 0};
+        oq.period = qh;
+        oq.rope_start = qk;
+        oq.d_rope = dR;
+        oq.rope_tab = ws.rope_tab;
+        e = mla::tc::gemm_bf16_tc(1, H * qh, B, d->d_model, (const bf16*)w->W_Q, 0, d->d_model, (const bf16*)h, 0,
+                                  d->d_model, oq, err.code, err.detail, s);
+        if (e != cudaSuccess) return e;
+        qn = (const T*)ws.q_buf;
+        qr = (const T*)ws.q_buf + qk;
+        sQn_b = sQr_b = (long long)H * qh;
+        sQn_h = sQr_h = qh;
+    } else if (!q_nope) {
         // q = W_Q h with RoPE on each head's rotary part [L1 "Multi-head attention estandar"]
         const int qh = qk + dR;
         mla::ProfScope ps(s, "simt_q_proj_rope");
@@ -357,7 +419,14 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
                            o_dst, ws, err, s);
     }
     if (e != cudaSuccess) return e;
-    if (w->W_O) {
+    if (w->W_O && tc_proj) {
+        // out[b] = W_O concat_h o[b,h] [L2 "Informacion tecnica": output projection]
+        const int Hv = H * vh;
+        mla::ProfScope ps(s, "tc_w_o");
+        mla::tc::GemmOut oo{out, 0, 1, d->d_model, 0};
+        e = mla::tc::gemm_bf16_tc(1, d->d_model, B, Hv, (const bf16*)w->W_O, 0, Hv, (const bf16*)ws.o_buf, 0, Hv,
+                                  oo, err.code, err.detail, s);
+    } else if (w->W_O) {
         // out[b] = W_O concat_h o[b,h] [L2 "Informacion tecnica": output projection]
         const int Hv = H * vh;
         mla::ProfScope ps(s, "simt_w_o");
@@ -399,6 +468,7 @@ struct PrefillWs {
     void* q_buf;   // [B*S, H, qk_nope + d_hR]
     void* k_buf;   // [B*S, H, qk_nope]
     void* v_buf;   // [B*S, H, v_head]
+    double2* rope_tab;   // [B*S, d_hR / 2] (cos, sin) of the query rotation (tensor-core projection)
     size_t bytes;
 };
 
@@ -409,6 +479,7 @@ static PrefillWs carve_prefill(const mla_dims* d, int B, int S, void* base) {
     w.q_buf = c.take(nH * (d->qk_nope + d->d_hR) * es);
     w.k_buf = c.take(nH * d->qk_nope * es);
     w.v_buf = c.take(nH * d->v_head * es);
+    w.rope_tab = (double2*)c.take((size_t)B * S * (d->d_hR / 2) * sizeof(double2));
     w.bytes = c.used;
     return w;
 }
@@ -428,6 +499,37 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
     // 1. cache rows for every token, position t = i % S, row b*S + t
     e = append_impl<T>(d, h, W_DKV, W_KR, nullptr, S, nullptr, n, cache, n, err, s);
     if (e != cudaSuccess) return e;
+    const bool tc_proj = tc_proj_ok(d) && aligned16(h) && aligned16(w->W_Q) && aligned16(cache) &&
+                         aligned16(w->W_UK) && aligned16(w->W_UV);
+    if (tc_proj) {
+        // 2. queries with RoPE at t = i % S
+        { mla::ProfScope ps(s, "tc_q_proj_rope");
+        e = mla::tc::rope_table(nullptr, S, n, dR, theta_of(d), ws.rope_tab, s);
+        if (e != cudaSuccess) return e;
+        mla::tc::GemmOut oq{ws.q_buf, 0, 1, (long long)H * qh, 0};
+        oq.period = qh;
+        oq.rope_start = qk;
+        oq.d_rope = dR;
+        oq.rope_tab = ws.rope_tab;
+        e = mla::tc::gemm_bf16_tc(1, H * qh, n, d->d_model, (const bf16*)w->W_Q, 0, d->d_model, (const bf16*)h, 0,
+                                  d->d_model, oq, err.code, err.detail, s); }
+        if (e != cudaSuccess) return e;
+        // 3. K_nope[t, h] = W_UK[h] c_t and V[t, h] = W_UV[h] c_t: one B (the cache rows) for all heads
+        { mla::ProfScope ps(s, "tc_k_materialise");
+        mla::tc::GemmOut okb{ws.k_buf, qk, 1, (long long)H * qk, 0};
+        e = mla::tc::gemm_bf16_tc(H, qk, n, dc, (const bf16*)w->W_UK, (long long)qk * dc, dc, (const bf16*)cache, 0,
+                                  row, okb, err.code, err.detail, s); }
+        if (e != cudaSuccess) return e;
+        { mla::ProfScope ps(s, "tc_v_materialise");
+        mla::tc::GemmOut ovb{ws.v_buf, vh, 1, (long long)H * vh, 0};
+        e = mla::tc::gemm_bf16_tc(H, vh, n, dc, (const bf16*)w->W_UV, (long long)vh * dc, dc, (const bf16*)cache, 0,
+                                  row, ovb, err.code, err.detail, s); }
+        if (e != cudaSuccess) return e;
+        mla::ProfScope ps(s, "simt_prefill_attn");
+        return mla::launch_prefill_attn_simt<T>((const T*)ws.q_buf, (const T*)ws.k_buf, (const T*)cache,
+                                                (const T*)ws.v_buf, B, S, H, qk, dR, dc, vh, scale_of(d),
+                                                (T*)out, s);
+    }
     // 2. queries with RoPE at t
     { mla::ProfScope ps(s, "simt_q_proj_rope");
     e = mla::launch_proj_rope<T>((const T*)h, n, d->d_model, (const T*)w->W_Q, H * qh, nullptr, H * qh,

@@ -35,7 +35,8 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
 gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                    int N, int K, int stages, GemmOut out, int chain_head, int* err_code, long long* err_detail) {
+                    int N, int K, int stages, GemmOut out, int chain_head, int b_bcast, int* err_code,
+                    long long* err_detail) {
     using C = GemmCfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -98,7 +99,10 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     ptx::mbar_expect_tx(&full[s], C::STAGE);
                     ptx::tma_load_3d(a, &tmA, &full[s], kb * kBK, m0, z);
                 }
-                ptx::tma_load_3d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0, z);
+                if (b_bcast)
+                    ptx::tma_load_2d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0);
+                else
+                    ptx::tma_load_3d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0, z);
             }
         }
     } else if (warp == 1) {
@@ -130,26 +134,53 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (!ok) fail(err_code, err_detail, abort_flag, 3);
         ptx::tc_fence_after();
         const int row = m0 + sub * 32 + lane;
+        const int within = out.period > 0 ? row % out.period : -1;
+        const bool rope_row = out.period > 0 && within >= out.rope_start;
         if (ok && !*abort_flag && nk > 0) {
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t r[32];
                 ptx::tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + c0, r);
                 ptx::tmem_wait_ld();
-                if (row < M) {
-                    char* base = (char*)out.C;
+                char* base = (char*)out.C;
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        const int n = n0 + c0 + j;
-                        if (n < N) {
-                            const long long idx = (long long)z * out.sz + (long long)row * out.sm + (long long)n * out.sn;
-                            const float v = __uint_as_float(r[j]);
-                            if (out.f32)
-                                ((float*)base)[idx] = v;
-                            else
-                                ((__nv_bfloat16*)base)[idx] = __float2bfloat16_rn(v);
+                for (int j = 0; j < 32; ++j) {
+                    const int n = n0 + c0 + j;   // the same for the whole warp
+                    if (n >= N) continue;
+                    float v = __uint_as_float(r[j]);
+                    if (out.period > 0) {
+                        // rows m and m ^ 1 are adjacent lanes: the pair (even, odd) is rotated
+                        const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
+                        if (rope_row) {
+                            const int pi = (within - out.rope_start) >> 1;
+                            double cs, sn;
+                            if (out.rope_tab) {
+                                const double2 t = out.rope_tab[(long long)n * (out.d_rope >> 1) + pi];
+                                cs = t.x;
+                                sn = t.y;
+                            } else {
+                                const int p = out.pos ? out.pos[n] : n % out.pos_mod;
+                                const double inv = pow((double)out.theta, -2.0 * (double)pi / (double)out.d_rope);
+                                sincos((double)p * inv, &sn, &cs);
+                            }
+                            v = (row & 1) ? (float)((double)partner * sn + (double)v * cs)
+                                          : (float)((double)v * cs - (double)partner * sn);
                         }
                     }
+                    if (row >= M) continue;
+                    long long orow = n;
+                    if (out.slot) {
+                        orow = out.slot[n];
+                        if (orow < 0 || orow >= out.cap) {
+                            if (lane == 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, n);
+                            continue;
+                        }
+                    }
+                    const long long idx = (long long)z * out.sz + (long long)row * out.sm + orow * out.sn;
+                    if (out.f32)
+                        ((float*)base)[idx] = v;
+                    else
+                        ((__nv_bfloat16*)base)[idx] = __float2bfloat16_rn(v);
                 }
             }
         }
@@ -161,7 +192,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
 template <int BN>
 cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUtensorMap& mb, const GemmOut& out,
-                   bool chain_head, int* err_code, long long* err_detail, cudaStream_t s) {
+                   bool chain_head, bool b_bcast, int* err_code, long long* err_detail, cudaStream_t s) {
     using C = GemmCfg<BN>;
     static bool attr_set = false;   // the attribute is per function; set it once
     if (!attr_set) {
@@ -174,16 +205,39 @@ cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUte
     const int stages = nk < C::MAX_STAGES ? (nk < 2 ? 2 : nk) : C::MAX_STAGES;
     dim3 grid((N + BN - 1) / BN, (M + kBM - 1) / kBM, Z);
     return launch_pdl(gemm_bf16_tc_kernel<BN>, grid, dim3(192), C::smem(stages), s, ma, mb, M, N, K, stages, out,
-                      (int)chain_head, err_code, err_detail);
+                      (int)chain_head, (int)b_bcast, err_code, err_detail);
+}
+
+__global__ void __launch_bounds__(256)
+rope_table_kernel(const int32_t* __restrict__ pos, int pos_mod, int N, int half, float theta, double2* __restrict__ tab) {
+    const long long total = (long long)N * half;
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total; i += (long long)gridDim.x * blockDim.x) {
+        const int n = (int)(i / half), pi = (int)(i % half);
+        const int p = pos ? pos[n] : n % pos_mod;
+        const double inv = pow((double)theta, -2.0 * (double)pi / (double)(2 * half));
+        double sn, cs;
+        sincos((double)p * inv, &sn, &cs);
+        tab[i] = make_double2(cs, sn);
+    }
 }
 
 }  // namespace
+
+cudaError_t rope_table(const int32_t* pos, int pos_mod, int N, int d_rope, float theta, double2* tab,
+                       cudaStream_t s) {
+    if (N <= 0) return cudaSuccess;
+    const long long total = (long long)N * (d_rope / 2);
+    const int blocks = (int)min(4096LL, (total + 255) / 256);
+    rope_table_kernel<<<blocks, 256, 0, s>>>(pos, pos_mod, N, d_rope / 2, theta, tab);
+    return cudaGetLastError();
+}
 
 cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, long long sAz, long long sAm,
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
                          int* err_code, long long* err_detail, cudaStream_t s, bool chain_head) {
     if (Z <= 0 || M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
     const int BN = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    const bool b_bcast = sBz == 0;   // one B for every z: a 2-D map
     if (Z == 1) {
         sAz = (long long)M * sAm;
         sBz = (long long)N * sBn;
@@ -195,13 +249,13 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     const uint64_t db[3] = {(uint64_t)K, (uint64_t)N, (uint64_t)Z};
     const uint64_t sb[2] = {(uint64_t)sBn * 2, (uint64_t)sBz * 2};
     const uint32_t bb[3] = {(uint32_t)kBK, (uint32_t)BN, 1};
-    if (!make_tmap_bf16(&ma, A, 3, da, sa, ba) || !make_tmap_bf16(&mb, B, 3, db, sb, bb))
+    if (!make_tmap_bf16(&ma, A, 3, da, sa, ba) || !make_tmap_bf16(&mb, B, b_bcast ? 2 : 3, db, sb, bb))
         return cudaErrorInvalidValue;
     switch (BN) {
-        case 32: return launch<32>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
-        case 64: return launch<64>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
-        case 128: return launch<128>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
-        default: return launch<256>(Z, M, N, K, ma, mb, out, chain_head, err_code, err_detail, s);
+        case 32: return launch<32>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
+        case 64: return launch<64>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
+        case 128: return launch<128>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
+        default: return launch<256>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
     }
 }
 

@@ -8,15 +8,33 @@ namespace mla {
 namespace tc {
 
 // Where and how the fp32 accumulator tile is written: element (z, m, n) goes to
-// C + z*sz + m*sm + n*sn, as bf16 (f32 == 0) or fp32 (f32 == 1).
+// C + z*sz + m*sm + row(n)*sn, as bf16 (f32 == 0) or fp32 (f32 == 1), where row(n) = n, or
+// slot[n] when slot is set (a slot outside [0, cap) is skipped and latched as out of range).
+// Rotary post-processing (period > 0): output rows m with (m % period) >= rope_start come in
+// pairs (m, m + 1) that are rotated by the angle pos(n) * theta^(-2i/d_rope), i the pair
+// index within the rotary block, pos(n) = pos ? pos[n] : n % pos_mod; with rope_tab set the
+// (cos, sin) of that angle are read from rope_tab[n * d_rope / 2 + i] instead of computed.
+// Rotation is done in double precision and the result rounded once.
 struct GemmOut {
     void* C;
     long long sz, sm, sn;
     int f32;
+    const int64_t* slot = nullptr;
+    long long cap = 0;
+    int period = 0, rope_start = 0, d_rope = 0;
+    const int32_t* pos = nullptr;
+    int pos_mod = 1;
+    float theta = 10000.f;
+    const double2* rope_tab = nullptr;
 };
 
+// rope_tab[n * d_rope / 2 + i] = (cos, sin)(pos(n) * theta^(-2i/d_rope)), computed in double.
+cudaError_t rope_table(const int32_t* pos, int pos_mod, int N, int d_rope, float theta, double2* tab,
+                       cudaStream_t s);
+
 // C[z][m][n] = sum_k A[z][m][k] * B[z][n][k] for z < Z, m < M, n < N.
-// A rows are K-contiguous with element strides (sAz, sAm); B rows likewise (sBz, sBn).
+// A rows are K-contiguous with element strides (sAz, sAm); B rows likewise (sBz, sBn);
+// sBz = 0 shares one B among all z.
 // Row strides must be multiples of 8 elements (16 bytes) and the bases 16-byte aligned.
 // The launch uses programmatic dependent launch.  A (read before waiting for the previous
 // kernel) must not be written by it.  chain_head: wait for all earlier work before letting
