@@ -909,9 +909,10 @@ cudaError_t set_smem_attrs(K kernel, int bytes) {
 // This is the first kernel of the decode chain: it waits for all earlier work before it lets
 // the next kernel launch (the decode kernel then reads the cache without waiting).
 constexpr int kAbsorbThreads = 128;
+constexpr int kAbsorbTiles = 2;   // 128-row tiles of W_UK^T[h] per CTA (two CTAs per head)
 
 template <int BN>
-constexpr int absorb_smem() { return 8 * 16384 + 2 * BN * 128 + 1024 + 64; }
+constexpr int absorb_smem() { return 2 * kAbsorbTiles * 16384 + 2 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kAbsorbThreads, 1)
@@ -919,12 +920,14 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
                 __nv_bfloat16* __restrict__ q_lat, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t absorb_smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)absorb_smem_raw + 1023) & ~(uintptr_t)1023);
-    uint8_t* sA = smem;                  // [m tile][k chunk] boxes of 128 rows x 128 B
-    uint8_t* sB = smem + 8 * 16384;      // [k chunk] boxes of BN rows x 128 B
+    uint8_t* sA = smem;                                 // [m tile][k chunk] chunks of 128 rows x 128 B
+    uint8_t* sB = smem + 2 * kAbsorbTiles * 16384;      // [k chunk] boxes of BN rows x 128 B
     uint64_t* full = (uint64_t*)(sB + 2 * BN * 128);
     uint64_t* d_full = full + 1;
     uint32_t* tmem_slot = (uint32_t*)(d_full + 1);
-    const int h = blockIdx.x, n0 = blockIdx.y * BN;
+    constexpr int W = 128 * kAbsorbTiles;   // latent columns of q_lat this CTA writes
+    const int h = blockIdx.x / (4 / kAbsorbTiles), t0 = (blockIdx.x % (4 / kAbsorbTiles)) * kAbsorbTiles;
+    const int n0 = blockIdx.y * BN;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -932,19 +935,20 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
         ptx::mbar_init(d_full, 1);
         ptx::fence_mbar_init();
         ptx::tma_prefetch(&tm_q);
-        ptx::mbar_expect_tx(full, 8 * 16384 + 2 * BN * 128);
+        ptx::mbar_expect_tx(full, 2 * kAbsorbTiles * 16384 + 2 * BN * 128);
         // weights first (earlier kernels do not write them): the tiled copy is already the
-        // shared-memory image, chunk (t, k) at (2t + k) x 16 KB
-        const uint8_t* src = (const uint8_t*)ukt + (size_t)h * 8 * 16384;
+        // shared-memory image, chunk (t, k) at (2t + k) x 16 KB; this CTA takes tiles t0 ..
+        const uint8_t* src = (const uint8_t*)ukt + ((size_t)h * 8 + 2 * t0) * 16384;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) ptx::bulk_load(sA + c * 16384, src + c * 16384, 16384, full);
+        for (int c = 0; c < 2 * kAbsorbTiles; ++c) ptx::bulk_load(sA + c * 16384, src + c * 16384, 16384, full);
         pdl_wait();      // the queries may come from the previous kernel; all earlier work is done
         pdl_trigger();   // only now may the next kernel launch
 #pragma unroll
         for (int kc = 0; kc < 2; ++kc) ptx::tma_load_3d(sB + kc * BN * 128, &tm_q, full, 64 * kc, n0, h);
     }
+    constexpr uint32_t kCols = kAbsorbTiles * BN < 32 ? 32 : kAbsorbTiles * BN;
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, 4 * BN);
+        ptx::tmem_alloc(tmem_slot, kCols);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -958,7 +962,7 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
             ptx::tc_fence_after();
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, BN, 0, 0);
 #pragma unroll
-            for (int mt = 0; mt < 4; ++mt)
+            for (int mt = 0; mt < kAbsorbTiles; ++mt)
 #pragma unroll
                 for (int kc = 0; kc < 2; ++kc)
 #pragma unroll
@@ -973,29 +977,29 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
         if (lane == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 8300000 + h);
     } else {
         ptx::tc_fence_after();
-        // D (row = latent index, column = sequence) -> bf16 stage[b][512] in the A buffer (free
-        // once the MMAs completed), then whole 1 KB rows q_lat[b, h, :]
+        // D (row = latent index, column = sequence) -> bf16 stage[b][128 x kAbsorbTiles] in the
+        // A buffer (free once the MMAs completed), then whole rows of q_lat[b, h, 128 t0 ..]
         const int m = warp * 32 + lane;   // row of the 128-row tile = TMEM lane
         __nv_bfloat16* stage = (__nv_bfloat16*)sA;
 #pragma unroll 1
-        for (int mt = 0; mt < 4; ++mt)
+        for (int mt = 0; mt < kAbsorbTiles; ++mt)
 #pragma unroll
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t r[32];
                 ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) stage[(c0 + j) * 512 + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                for (int j = 0; j < 32; ++j) stage[(c0 + j) * W + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
             }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < BN * 64; i += kAbsorbThreads) {
-        const int b = n0 + (i >> 6);
-        if (b < B) ((uint4*)(q_lat + ((long long)b * 128 + h) * 512))[i & 63] = ((const uint4*)sA)[i];
+    for (int i = threadIdx.x; i < BN * (W / 8); i += kAbsorbThreads) {
+        const int b = n0 + i / (W / 8);
+        if (b < B) ((uint4*)(q_lat + ((long long)b * 128 + h) * 512 + 128 * t0))[i % (W / 8)] = ((const uint4*)sA)[i];
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) ptx::tmem_dealloc(tmem, 4 * BN);
+    if (warp == 1) ptx::tmem_dealloc(tmem, kCols);
 }
 
 template <int BN>
@@ -1003,7 +1007,8 @@ cudaError_t launch_absorb(const __nv_bfloat16* ukt, const CUtensorMap& mq, int B
                           long long* err_detail, cudaStream_t s) {
     static const cudaError_t attr = set_smem_attrs(absorb_q_kernel<BN>, absorb_smem<BN>());
     if (attr != cudaSuccess) return attr;
-    return launch_pdl(absorb_q_kernel<BN>, dim3(128, (B + BN - 1) / BN), dim3(kAbsorbThreads), absorb_smem<BN>(), s,
+    return launch_pdl(absorb_q_kernel<BN>, dim3(128 * (4 / kAbsorbTiles), (B + BN - 1) / BN), dim3(kAbsorbThreads),
+                      absorb_smem<BN>(), s,
                       ukt, mq, B, q_lat, err_code, err_detail);
 }
 

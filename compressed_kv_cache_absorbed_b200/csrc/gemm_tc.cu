@@ -236,7 +236,17 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
                          int* err_code, long long* err_detail, cudaStream_t s, bool chain_head) {
     if (Z <= 0 || M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
-    const int BN = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    // the narrowest tile that covers N, narrowed further while the grid has fewer CTAs than a
+    // quarter of the SMs (very skinny weight-streaming GEMMs: A is then re-read from L2)
+    static int sms = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaGetDevice(&dev);
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
+    }
+    int BN = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
+    const long long mtiles = (long long)Z * ((M + 127) / 128);
+    while (BN > 32 && mtiles * ((N + BN - 1) / BN) < sms / 4) BN >>= 1;
     const bool b_bcast = sBz == 0;   // one B for every z: a 2-D map
     if (Z == 1) {
         sAz = (long long)M * sAm;
