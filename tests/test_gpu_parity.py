@@ -363,3 +363,34 @@ def test_decode_invariant_to_cache_row_order():
     inp2["cache"] = inp["cache"][torch.from_numpy(perm)].contiguous()
     out2 = run_decode_attn(w, inp2)
     assert_close(out2, out1.double(), "bf16", "row permutation")
+
+
+# --------------------------------------------- which kernels run (no silent fallback)
+
+def test_v3_bf16_paths_run_the_tensor_core_kernels():
+    """A reduced V3-shaped decode layer and prefill: the library's per-launch profile names
+    show the tcgen05 kernels ran for every projection and for the attention chain."""
+    w = workloads.shrink(workloads.WORKLOADS["v3_layer_b128_ctx8192"], B=3, ctx=70, seed=91)
+    inp = workloads.make_inputs(w)
+    mla.mla_profile_report(reset=True)
+    mla.mla_profile_enable(True)
+    try:
+        out, _ = run_decode_layer(w, inp)
+    finally:
+        mla.mla_profile_enable(False)
+    names = set(mla.mla_profile_report(reset=True))
+    assert {"tc_append_proj_rope", "tc_q_proj_rope", "tc_q_absorb", "tc_flash_decode", "tc_merge_w_uv",
+            "tc_w_o"} <= names, names
+    assert not any(n.startswith("simt_") for n in names), names
+    want, _ = oracle_decode_layer(w, inp, [0, 2], absorbed=True)
+    assert_close(out[[0, 2]], want, "bf16", "reduced v3 layer")
+
+    p = workloads.shrink(workloads.WORKLOADS["v2_prefill_b4_s4096"], B=1, ctx=130, seed=92)
+    pin = workloads.make_inputs(p)
+    mla.mla_profile_enable(True)
+    try:
+        run_prefill(p, pin)
+    finally:
+        mla.mla_profile_enable(False)
+    names = set(mla.mla_profile_report(reset=True))
+    assert {"tc_append_proj_rope", "tc_q_proj_rope", "tc_k_materialise", "tc_v_materialise"} <= names, names
