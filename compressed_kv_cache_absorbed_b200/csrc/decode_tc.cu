@@ -73,10 +73,8 @@ constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 s
 // kPieceCost.
 constexpr int kPieceCost = 3;
 
-// Plan written by CTA 0 for the merge kernel (int32): [0] total cost, [1] cost units per
-// cluster, [2] clusters, [4, 4+B) first[b], [4+B+1, 4+2B+1) first[b] + tiles of b.
-__device__ __forceinline__ const int32_t* plan_first_pos(const int32_t* w) { return w + 4; }
-__device__ __forceinline__ const int32_t* plan_end_pos(const int32_t* w, int B) { return w + 4 + B + 1; }
+// The merge kernel recomputes this split from the offsets (it needs each sequence's first
+// and last cost positions and the cost units per cluster).
 
 __device__ __forceinline__ int tiles_of_len(int L) { return L > 0 ? (L + kT - 1) / kT : 0; }
 __device__ __forceinline__ int cost_of_tiles(int n) { return n > 0 ? n + kPieceCost : 0; }
@@ -156,7 +154,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                  const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const int32_t* __restrict__ offsets, int B, long long cache_rows,
-                 int32_t* __restrict__ work, float scale_log2,
+                 float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -264,8 +262,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     }
     const int per = total > 0 ? (total + P - 1) / P : 1;
     const int lo = cluster * per, hi = min(total, lo + per);
-    const bool writer = blockIdx.x == 0;   // publishes every sequence's tile positions for the merge
-    if (lo < total || writer) {
+    if (lo < total) {
         int carry = 0;
         for (int c0 = 0; c0 < B; c0 += kThreads) {
             const int b = c0 + (int)threadIdx.x;
@@ -288,10 +285,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             }
             const int cs = before + incl - cb;   // cost of the sequences before b
             if (b < B) {
-                if (writer) {
-                    work[4 + b] = cs + kPieceCost;
-                    work[4 + B + 1 + b] = cs + kPieceCost + n;
-                }
                 if (cb > 0 && cs <= lo && lo < cs + cb) {   // unique: the cost region holding lo
                     plan_first[0] = b;
                     plan_first[1] = cs;
@@ -300,11 +293,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             carry += chunk;
             __syncthreads();
         }
-    }
-    if (writer && threadIdx.x == 0) {
-        work[0] = total;
-        work[1] = per;
-        work[2] = P;
     }
     SegIter it{offsets, B, lo, hi, cluster, plan_first[0], plan_first[1]};
     Seg sg;
@@ -697,7 +685,7 @@ constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kMergeThreads, 1)
-merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict__ work, int B,
+merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict__ offsets, int P, int B,
                  const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
@@ -726,20 +714,64 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict
         ptx::tmem_relinquish();
     }
     if (threadIdx.x == 0) pdl_trigger();
-    pdl_wait();   // the partials and the plan come from the decode kernel
-
-    const int32_t* fpos = plan_first_pos(work);
-    const int32_t* epos = plan_end_pos(work, B);
-    const int per = work[1];
+    // The split of the decode kernel (same cost model, same cluster count), recomputed from
+    // the offsets before waiting for that kernel: cost positions of the first and one past
+    // the last tile of this CTA's sequences.
+    __shared__ int s_wsum[kMergeThreads / 32];
+    __shared__ int s_pos[2][BN];
     constexpr int kW = kMergeThreads / 32;
+    int total = 0;
+    {
+        int mine = 0;
+        for (int b = threadIdx.x; b < B; b += kMergeThreads) mine += cost_of_tiles(tiles_of_len(offsets[b + 1] - offsets[b]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
+        if (lane == 0) s_wsum[warp] = mine;
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < kW; ++i) total += s_wsum[i];
+        __syncthreads();
+    }
+    const int per = total > 0 ? (total + P - 1) / P : 1;
+    {
+        int carry = 0;
+        for (int c0 = 0; c0 < B && c0 < n0 + BN; c0 += kMergeThreads) {
+            const int b = c0 + (int)threadIdx.x;
+            const int nt = b < B ? tiles_of_len(offsets[b + 1] - offsets[b]) : 0;
+            const int cb = cost_of_tiles(nt);
+            int incl = cb;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            if (lane == 31) s_wsum[warp] = incl;
+            __syncthreads();
+            int before = carry, chunk = 0;
+#pragma unroll
+            for (int i = 0; i < kW; ++i) {
+                const int v = s_wsum[i];
+                before += i < warp ? v : 0;
+                chunk += v;
+            }
+            const int cs = before + incl - cb;
+            if (b < B && b >= n0 && b < n0 + BN) {
+                s_pos[0][b - n0] = cs + kPieceCost;
+                s_pos[1][b - n0] = cs + kPieceCost + nt;
+            }
+            carry += chunk;
+            __syncthreads();
+        }
+    }
+    pdl_wait();   // the partials come from the decode kernel
+
     constexpr int kRowsPerWarp = BN / kW;
-    // first tiles of this warp's rows, fetched together
     int t0r[kRowsPerWarp], t1r[kRowsPerWarp];
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
         const int b = n0 + warp + kW * i;
-        t0r[i] = b < B ? fpos[b] : 0;   // cost positions of the first and one past the last tile
-        t1r[i] = b < B ? epos[b] : 0;
+        t0r[i] = b < B ? s_pos[0][warp + kW * i] : 0;
+        t1r[i] = b < B ? s_pos[1][warp + kW * i] : 0;
     }
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
@@ -1042,8 +1074,7 @@ size_t decode_ws_bytes(int B, int num_sms) {
     const size_t P = (size_t)(num_sms / 2);
     const size_t slots = (size_t)B + P + 1;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    return up((size_t)B * 128 * 512 * 2) + up((4 + 2 * ((size_t)B + 1)) * 4) + up(slots * 512 * 128 * 4) +
-           up(slots * 128 * 2 * 4) + up((size_t)B * 128 * 512 * 2);
+    return up((size_t)B * 128 * 512 * 2) + up(slots * 512 * 128 * 4) + up(slots * 128 * 2 * 4);
 }
 
 DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
@@ -1058,11 +1089,8 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
         return p;
     };
     w.q_lat = (__nv_bfloat16*)take((size_t)B * 128 * 512 * 2);
-    w.work = (int32_t*)take((4 + 2 * ((size_t)B + 1)) * 4);
     w.part_o = (float*)take(slots * 512 * 128 * 4);
     w.part_ml = (float*)take(slots * 128 * 2 * 4);
-    w.o_lat = (__nv_bfloat16*)take((size_t)B * 128 * 512 * 2);
-    w.q_cat = nullptr;
     w.max_parts = (int)slots;
     return w;
 }
@@ -1104,7 +1132,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
         if (attr != cudaSuccess) return attr;
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
-                            offsets, B, (long long)cache_rows, ws.work, scale * 1.4426950408889634f,
+                            offsets, B, (long long)cache_rows, scale * 1.4426950408889634f,
                             ws.part_o, ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code,
                             err_detail)) != cudaSuccess)
             return e;
@@ -1116,13 +1144,13 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                           (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           offsets, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         } else {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                           uv, (const int32_t*)ws.work, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           uv, offsets, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         }
     }

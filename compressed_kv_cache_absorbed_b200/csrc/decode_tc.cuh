@@ -19,11 +19,8 @@ constexpr bool kEnabled = true;
 // Workspace pieces of the tensor-core decode (all device memory, carved by the caller).
 struct DecodeWs {
     __nv_bfloat16* q_lat;   // [B, H, d_c] absorbed query, bf16
-    __nv_bfloat16* q_cat;   // unused
     float* part_o;          // [max_parts, H, d_c] un-normalised partial o_lat
     float* part_ml;         // [max_parts, H, 2] running max (log2 domain) and sum
-    int32_t* work;          // split plan: totals and the first tile of each sequence
-    __nv_bfloat16* o_lat;   // unused
     int max_parts;
 };
 
