@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(_HERE, "libmla_b200.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError(f"{LIB_PATH} is missing: build it with "
-                      "`python -m compressed_kv_cache_absorbed_b200._build` (nvcc, sm_100a)")
+                      "`python compressed_kv_cache_absorbed_b200/_build.py` (nvcc, sm_100a)")
 _lib = ctypes.CDLL(LIB_PATH)
 
 MLA_OK, MLA_ERR_INVALID_ARG, MLA_ERR_UNSUPPORTED, MLA_ERR_WORKSPACE = 0, 1, 2, 3
@@ -54,6 +54,8 @@ SIGNATURES = {
     "mla_get_device_error": (_S, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "mla_decode_absorbed_noalloc": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P,
                                          _P]),
+    "mla_decode_absorbed_host": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
+                                      ctypes.c_size_t, _P]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
     "mla_profile_report": (ctypes.c_int32, [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_int32]),
 }
@@ -178,6 +180,17 @@ def mla_decode_absorbed_noalloc(dims, weights: MLAWeights, cache, offsets, out, 
     _check(_lib.mla_decode_absorbed_noalloc(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
                                             _ptr(h), _ptr(q_pos), _ptr(cache), cache.shape[0], _ptr(offsets), B,
                                             _ptr(out), _stream(stream)), "mla_decode_absorbed_noalloc")
+
+
+def mla_decode_absorbed_host(dims, weights: MLAWeights, cache, offsets, q_nope_host, q_rope_host, out_host, ws,
+                             stream=None) -> None:
+    """mla_decode_absorbed with q_nope, q_rope and the output in host (CPU, ideally pinned)
+    tensors; the copies run on the stream inside the call.  Synchronise the stream before
+    reading out_host."""
+    B = offsets.numel() - 1
+    _check(_lib.mla_decode_absorbed_host(ctypes.byref(dims), weights.handle, _ptr(q_nope_host), _ptr(q_rope_host),
+                                         _ptr(cache), cache.shape[0], _ptr(offsets), B, _ptr(out_host), _ptr(ws),
+                                         ws.numel(), _stream(stream)), "mla_decode_absorbed_host")
 
 
 def mla_prefill_causal(dims, weights: MLAWeights, h, W_DKV, W_KR, cache, out, ws, stream=None) -> None:

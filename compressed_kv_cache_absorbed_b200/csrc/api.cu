@@ -462,6 +462,39 @@ extern "C" mla_status mla_decode_absorbed(const mla_dims* d, mla_weights w, cons
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed");
 }
 
+extern "C" mla_status mla_decode_absorbed_host(const mla_dims* d, mla_weights w, const void* q_nope_host,
+                                               const void* q_rope_host, const void* cache, int64_t cache_rows,
+                                               const int32_t* offsets, int32_t B, void* out_host, void* workspace,
+                                               size_t ws_bytes, mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if (w->W_O) return MLA_ERR_UNSUPPORTED;
+    if (B == 0) return MLA_OK;
+    if (!q_nope_host || !q_rope_host || !out_host) return MLA_ERR_INVALID_ARG;
+    if (!cache || !offsets || cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return MLA_ERR_INVALID_ARG;
+    const bool tc_path = tc_decode_ok(d);
+    DecodeWs ws = carve_decode(d, B, workspace, tc_path);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the query staging area (q_buf, [B*H*(qk + dR)] elements) holds q_nope then q_rope,
+    // each in its plain [B, H, .] layout; o goes through o_buf ([B, H, v_head])
+    const size_t es = esize(d), BH = (size_t)B * d->H;
+    char* qn = (char*)ws.q_buf;
+    char* qr = qn + BH * d->qk_nope * es;
+    cudaError_t e = cudaMemcpyAsync(qn, q_nope_host, BH * d->qk_nope * es, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(qr, q_rope_host, BH * d->d_hR * es, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_fail(e, "mla_decode_absorbed_host");
+    e = d->dtype == MLA_BF16
+            ? decode_impl<bf16>(d, w, qn, qr, nullptr, nullptr, cache, cache_rows, offsets, B, ws.o_buf, ws, tc_path, err, s)
+            : decode_impl<float>(d, w, qn, qr, nullptr, nullptr, cache, cache_rows, offsets, B, ws.o_buf, ws, false, err, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, ws.o_buf, BH * d->v_head * es, cudaMemcpyDeviceToHost, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_host");
+}
+
 // ----------------------------------------------------------------------- prefill
 
 struct PrefillWs {

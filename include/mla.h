@@ -155,6 +155,21 @@ mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* 
                                int32_t B, void* out, void* workspace, size_t ws_bytes,
                                mla_stream_t stream);
 
+/* mla_decode_absorbed with the queries and the output in HOST memory: the call copies
+ * q_nope [B,H,qk_nope] and q_rope [B,H,d_hR] (storage type, rotated) host->device into the
+ * workspace, runs the same decode on the stream, and copies o [B,H,v_head] device->host.
+ * Everything is enqueued on `stream` and the call returns at once; out_host is valid after
+ * the stream has been synchronised.  Host buffers should be page-locked (cudaHostAlloc or
+ * cudaHostRegister) for the copies to be asynchronous; pageable memory works but the copies
+ * then block the calling thread.  The workspace is the one of mla_decode_absorbed.
+ * Handles holding W_O are not accepted here (MLA_ERR_UNSUPPORTED): use mla_decode_absorbed.
+ * The pages have no counterpart to this call; it is the end-to-end path of a server that
+ * keeps the cache on the GPU and exchanges only the step's queries and outputs. */
+mla_status mla_decode_absorbed_host(const mla_dims* dims, mla_weights w, const void* q_nope_host,
+                                    const void* q_rope_host, const void* cache, int64_t cache_rows,
+                                    const int32_t* offsets, int32_t B, void* out_host, void* workspace,
+                                    size_t ws_bytes, mla_stream_t stream);
+
 /* Size of the fixed device scratch used by mla_decode_absorbed_noalloc (64 MiB). */
 #define MLA_NOALLOC_SCRATCH_BYTES (64u << 20)
 

@@ -394,3 +394,24 @@ def test_v3_bf16_paths_run_the_tensor_core_kernels():
         mla.mla_profile_enable(False)
     names = set(mla.mla_profile_report(reset=True))
     assert {"tc_append_proj_rope", "tc_q_proj_rope", "tc_k_materialise", "tc_v_materialise"} <= names, names
+
+
+# ------------------------------------------------------------ host-buffer decode
+
+def test_decode_with_host_buffers_matches_the_oracle_and_the_device_call():
+    w, inp = reduced_attn_inputs([300, 1, 77, 513, 64], seed=23)
+    dims = dims_of(w)
+    g = to_dev({k: inp[k] for k in ("cache", "offsets", "W_UK", "W_UV")})
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B))
+    qn_h = inp["q_nope"].contiguous().pin_memory()
+    qr_h = inp["q_rope"].contiguous().pin_memory()
+    out_h = torch.empty(w.B, w.H, w.v_head, dtype=torch.bfloat16).pin_memory()
+    mla.mla_decode_absorbed_host(dims, weights, g["cache"], g["offsets"], qn_h, qr_h, out_h, ws)
+    torch.cuda.synchronize()
+    assert mla.mla_get_device_error() == (0, 0)
+    dev = run_decode_attn(w, inp)
+    assert torch.equal(out_h, dev), "the host-buffer call runs the same kernels on the same data"
+    units = [(b, h) for b in range(w.B) for h in (0, 31, 127)]
+    want = oracle_decode_units(w, inp, units)
+    assert_close(torch.stack([out_h[b, h] for b, h in units]), want, "bf16", "host-buffer decode")
