@@ -54,6 +54,8 @@ SIGNATURES = {
     "mla_get_device_error": (_S, [_P, ctypes.POINTER(ctypes.c_int64)]),
     "mla_decode_absorbed_noalloc": (_S, [_D, _P, _P, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P,
                                          _P]),
+    "mla_decode_absorbed_paged": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, ctypes.c_int32,
+                                       _P, _P, ctypes.c_size_t, _P]),
     "mla_decode_absorbed_host": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
                                       ctypes.c_size_t, _P]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
@@ -180,6 +182,17 @@ def mla_decode_absorbed_noalloc(dims, weights: MLAWeights, cache, offsets, out, 
     _check(_lib.mla_decode_absorbed_noalloc(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
                                             _ptr(h), _ptr(q_pos), _ptr(cache), cache.shape[0], _ptr(offsets), B,
                                             _ptr(out), _stream(stream)), "mla_decode_absorbed_noalloc")
+
+
+def mla_decode_absorbed_paged(dims, weights: MLAWeights, cache_pages, block_table, seq_lens, out, ws, q_nope,
+                              q_rope, stream=None) -> None:
+    """Absorbed decode over a paged cache: cache_pages [num_pages, 64, d_c + d_hR],
+    block_table int32 [B, max_blocks] (page of each 64-token block), seq_lens int32 [B]."""
+    B, max_blocks = block_table.shape
+    _check(_lib.mla_decode_absorbed_paged(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
+                                          _ptr(cache_pages), cache_pages.shape[0], _ptr(block_table), max_blocks,
+                                          _ptr(seq_lens), B, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
+           "mla_decode_absorbed_paged")
 
 
 def mla_decode_absorbed_host(dims, weights: MLAWeights, cache, offsets, q_nope_host, q_rope_host, out_host, ws,

@@ -412,7 +412,8 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (tc_path) {
         e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
                                         (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                        (const bf16*)cache, cache_rows, offsets, B, scale_of(d), (bf16*)o_dst,
+                                        (const bf16*)cache, cache_rows, offsets, nullptr, nullptr, 0, B, scale_of(d),
+                                        (bf16*)o_dst,
                                         ws.tc, num_sms(), err.code, err.detail, s);
     } else {
         e = decode_simt<T>(d, w, qn, sQn_b, sQn_h, qr, sQr_b, sQr_h, (const T*)cache, cache_rows, offsets, B,
@@ -493,6 +494,34 @@ extern "C" mla_status mla_decode_absorbed_host(const mla_dims* d, mla_weights w,
             : decode_impl<float>(d, w, qn, qr, nullptr, nullptr, cache, cache_rows, offsets, B, ws.o_buf, ws, false, err, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(out_host, ws.o_buf, BH * d->v_head * es, cudaMemcpyDeviceToHost, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_host");
+}
+
+extern "C" mla_status mla_decode_absorbed_paged(const mla_dims* d, mla_weights w, const void* q_nope,
+                                                const void* q_rope, const void* cache, int64_t num_pages,
+                                                const int32_t* block_table, int32_t max_blocks,
+                                                const int32_t* seq_lens, int32_t B, void* out, void* workspace,
+                                                size_t ws_bytes, mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if (!tc_decode_ok(d) || w->W_O) return MLA_ERR_UNSUPPORTED;
+    if (B == 0) return MLA_OK;
+    if (!q_nope || !q_rope || !cache || !block_table || !seq_lens || !out || max_blocks <= 0 || num_pages <= 0)
+        return MLA_ERR_INVALID_ARG;
+    const long long rows = (long long)num_pages * mla::tc::kPageTokens;
+    if (rows > 0x7FFFFFFFLL) return MLA_ERR_UNSUPPORTED;
+    DecodeWs ws = carve_decode(d, B, workspace, true);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    const long long H = d->H;
+    cudaError_t e = mla::tc::decode_absorbed_tc(
+        (const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope, H * d->d_hR, d->d_hR,
+        (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, (const bf16*)cache, rows, nullptr, seq_lens,
+        block_table, max_blocks, B, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged");
 }
 
 // ----------------------------------------------------------------------- prefill

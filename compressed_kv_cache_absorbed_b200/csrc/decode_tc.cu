@@ -110,18 +110,31 @@ struct Seg {
     long long row0;
 };
 
+// Where the cache rows of a sequence live: rows [offsets[b], offsets[b+1]) of the cache, or,
+// with a block table (paged cache), seq_lens[b] tokens in 64-token pages, tile j of sequence
+// b in page block_table[b * bt_stride + j] (cache rows 64 page .. 64 page + 63).
+struct SeqSrc {
+    const int32_t* offsets;
+    const int32_t* seq_lens;
+    const int32_t* block_table;
+    int bt_stride;
+    __device__ int len(int b) const { return block_table ? seq_lens[b] : offsets[b + 1] - offsets[b]; }
+    __device__ long long row0(int b) const { return block_table ? 0 : offsets[b]; }
+};
+
 // Walks the pieces of sequences in this cluster's cost range [lo, hi), in sequence order,
 // starting from the sequence whose cost region holds lo (cost start cs).  The same walk runs
 // in every role of both CTAs.  Partial slots: a piece that starts at its sequence's first
 // tile takes slot b; the one piece of a cluster that continues a sequence begun in an
 // earlier cluster takes slot B + cluster.  So B + clusters slots suffice.
 struct SegIter {
-    const int32_t* offsets;
+    SeqSrc src;
     int B, lo, hi, cluster, b, cs;
     __device__ bool next(Seg& s) {
         while (b < B && cs < hi) {
-            const int r0 = offsets[b], r1 = offsets[b + 1];
-            const int L = r1 > r0 ? r1 - r0 : 0;
+            const int Lraw = src.len(b);
+            const int L = Lraw > 0 ? Lraw : 0;
+            const long long r0 = src.row0(b);
             const int n = tiles_of_len(L);
             const int f = cs + kPieceCost;   // cost position of tile 0
             const int bb = b;
@@ -153,7 +166,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_rope,
                  const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
-                 const int32_t* __restrict__ offsets, int B, long long cache_rows,
+                 const SeqSrc src, int B, long long cache_rows,
                  float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
@@ -164,7 +177,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     }
     // this thread's sequence length for the planning below, requested before the set-up
     // so that the load overlaps it
-    const int len0 = threadIdx.x < B ? offsets[threadIdx.x + 1] - offsets[threadIdx.x] : 0;
+    const int len0 = threadIdx.x < B ? src.len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
     uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
@@ -244,7 +257,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     {
         int mine = 0;
         for (int b = threadIdx.x; b < B; b += kThreads) {
-            const int L = b == (int)threadIdx.x ? len0 : offsets[b + 1] - offsets[b];
+            const int L = b == (int)threadIdx.x ? len0 : src.len(b);
             if (L < 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
             mine += cost_of_tiles(tiles_of_len(L));
         }
@@ -266,7 +279,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         int carry = 0;
         for (int c0 = 0; c0 < B; c0 += kThreads) {
             const int b = c0 + (int)threadIdx.x;
-            const int n = b < B ? tiles_of_len(c0 == 0 ? len0 : offsets[b + 1] - offsets[b]) : 0;
+            const int n = b < B ? tiles_of_len(c0 == 0 ? len0 : src.len(b)) : 0;
             const int cb = cost_of_tiles(n);
             int incl = cb;
 #pragma unroll
@@ -294,7 +307,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             __syncthreads();
         }
     }
-    SegIter it{offsets, B, lo, hi, cluster, plan_first[0], plan_first[1]};
+    SegIter it{src, B, lo, hi, cluster, plan_first[0], plan_first[1]};
     Seg sg;
 
     if (warp == 0) {
@@ -306,7 +319,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             const uint64_t stream_policy = ptx::policy_evict_first();
             uint32_t g = 0;
             while (!*abort_flag && it.next(sg)) {
-                if (sg.row0 + (long long)sg.L > cache_rows) {   // sequence beyond the cache
+                if (src.block_table ? sg.L > src.bt_stride * kT                 // more pages than the table row
+                                    : sg.row0 + (long long)sg.L > cache_rows) {  // sequence beyond the cache
                     latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
                     *abort_flag = 1;
                     break;
@@ -319,7 +333,17 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         break;
                     }
                     uint8_t* dst = tiles + s * kTileBytes;
-                    const int row = (int)(sg.row0 + (long long)j * kT);
+                    long long row_l = sg.row0 + (long long)j * kT;
+                    if (src.block_table) {
+                        const long long page = src.block_table[(long long)sg.b * src.bt_stride + j];
+                        if (page < 0 || (page + 1) * kT > cache_rows) {   // page outside the cache
+                            latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
+                            *abort_flag = 1;
+                            break;
+                        }
+                        row_l = page * kT;
+                    }
+                    const int row = (int)row_l;
                     ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
 #pragma unroll
                     for (int i = 0; i < 4; ++i)
@@ -619,6 +643,20 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     }
                 }
                 ptx::tmem_st16(lane_addr + kColP + 32 * pb + 16 * half, pw);
+                const int n_valid = min(kT, cur.L - j * kT);
+                if (n_valid < kT) {
+                    // The rows past the sequence end in this tile hold whatever follows it
+                    // (another sequence, unused capacity, the rest of a page), possibly NaN or
+                    // Inf bit patterns, which the O MMA would turn into NaN even with P = 0:
+                    // zero them (the score MMA that also read them has completed).
+                    uint4* t4 = (uint4*)(tiles + (g % kStages) * kTileBytes);
+                    const int tid = (warp - 6) * 32 + lane;   // 0 .. 255 over the softmax warps
+                    for (int e = tid; e < (kT - n_valid) * 4 * 8; e += 256) {
+                        const int r = n_valid + (e >> 5), c = (e >> 3) & 3, u = e & 7;
+                        t4[(c * kChunkBytes + r * 128) / 16 + u] = make_uint4(0, 0, 0, 0);
+                    }
+                    ptx::fence_proxy_async_smem();   // read by the tensor cores
+                }
                 ptx::tmem_wait_st();
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&p_ready[pb]);
@@ -685,7 +723,7 @@ constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kMergeThreads, 1)
-merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict__ offsets, int P, int B,
+merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B,
                  const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
@@ -723,7 +761,7 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict
     int total = 0;
     {
         int mine = 0;
-        for (int b = threadIdx.x; b < B; b += kMergeThreads) mine += cost_of_tiles(tiles_of_len(offsets[b + 1] - offsets[b]));
+        for (int b = threadIdx.x; b < B; b += kMergeThreads) mine += cost_of_tiles(tiles_of_len(src.len(b)));
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) mine += __shfl_xor_sync(0xffffffffu, mine, off);
         if (lane == 0) s_wsum[warp] = mine;
@@ -737,7 +775,7 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const int32_t* __restrict
         int carry = 0;
         for (int c0 = 0; c0 < B && c0 < n0 + BN; c0 += kMergeThreads) {
             const int b = c0 + (int)threadIdx.x;
-            const int nt = b < B ? tiles_of_len(offsets[b + 1] - offsets[b]) : 0;
+            const int nt = b < B ? tiles_of_len(src.len(b)) : 0;
             const int cb = cost_of_tiles(nt);
             int incl = cb;
 #pragma unroll
@@ -1098,12 +1136,15 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h, const __nv_bfloat16* qr,
                                long long sQr_b, long long sQr_h, const __nv_bfloat16* ukt,
                                const __nv_bfloat16* uv, const __nv_bfloat16* cache, long long cache_rows,
-                               const int32_t* offsets, int B, float scale, __nv_bfloat16* o, const DecodeWs& ws,
+                               const int32_t* offsets, const int32_t* seq_lens, const int32_t* block_table,
+                               int bt_stride, int B, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s) {
     if (B <= 0) return cudaSuccess;
     cudaError_t e;
     if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
+    if (block_table && (!seq_lens || bt_stride <= 0)) return cudaErrorInvalidValue;
+    const SeqSrc seqs{offsets, seq_lens, block_table, bt_stride};
     const int P = max_clusters(num_sms);
     {
         // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]
@@ -1132,7 +1173,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
         if (attr != cudaSuccess) return attr;
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
-                            offsets, B, (long long)cache_rows, scale * 1.4426950408889634f,
+                            seqs, B, (long long)cache_rows, scale * 1.4426950408889634f,
                             ws.part_o, ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code,
                             err_detail)) != cudaSuccess)
             return e;
@@ -1144,13 +1185,13 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                           offsets, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           seqs, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         } else {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                           uv, offsets, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           uv, seqs, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         }
     }

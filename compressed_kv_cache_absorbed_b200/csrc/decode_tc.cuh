@@ -14,6 +14,7 @@ constexpr int kH = 128;
 constexpr int kDc = 512;
 constexpr int kDr = 64;
 constexpr int kRow = kDc + kDr;  // 576 cache elements per token
+constexpr int kPageTokens = 64;  // tokens per page of a paged cache (one decode tile)
 constexpr bool kEnabled = true;
 
 // Workspace pieces of the tensor-core decode (all device memory, carved by the caller).
@@ -42,10 +43,14 @@ cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_U
 
 // q_nope rows at qn + b*sQn_b + h*sQn_h (qk_nope = 128), q_rope rows at qr + b*sQr_b + h*sQr_h.
 // ukt / uv: the tiled weights written by tile_weights_tc; out o [B, H, 128] bf16.
+// Sequence b's cache rows are [offsets[b], offsets[b+1]) when block_table is null; with a
+// block table (paged cache, 64-token pages) sequence b has seq_lens[b] tokens and its tile j
+// is page block_table[b * bt_stride + j] (rows 64 page .. 64 page + 63).
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
                                const __nv_bfloat16* ukt, const __nv_bfloat16* uv,
                                const __nv_bfloat16* cache, long long cache_rows, const int32_t* offsets,
+                               const int32_t* seq_lens, const int32_t* block_table, int bt_stride,
                                int B, float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s);
 

@@ -155,6 +155,22 @@ mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* 
                                int32_t B, void* out, void* workspace, size_t ws_bytes,
                                mla_stream_t stream);
 
+/* mla_decode_absorbed over a PAGED latent cache: the cache is num_pages pages of 64 tokens
+ * ([num_pages, 64, d_c + d_hR] rows, the row layout of mla_decode_absorbed); sequence b has
+ * seq_lens[b] tokens (int32 [B], device) and its j-th 64-token block is page
+ * block_table[b * max_blocks + j] (int32 [B, max_blocks], device).  The result is that of
+ * mla_decode_absorbed on the same rows laid out contiguously.  The pages describe a paged
+ * cache as a layer orthogonal to MLA ["DeepSeek MLA", the PagedAttention comparison].
+ * Queries from q_nope/q_rope only; the tensor-core shape only (bf16, H = 128, d_c = 512,
+ * d_hR = 64, qk_nope = v_head = 128) and handles without W_O, else MLA_ERR_UNSUPPORTED.
+ * A sequence needing more than max_blocks pages, or a page outside [0, num_pages), latches
+ * MLA_ERR_OUT_OF_RANGE on the device.  Workspace: mla_decode_workspace_size(dims, B). */
+mla_status mla_decode_absorbed_paged(const mla_dims* dims, mla_weights w, const void* q_nope,
+                                     const void* q_rope, const void* cache, int64_t num_pages,
+                                     const int32_t* block_table, int32_t max_blocks,
+                                     const int32_t* seq_lens, int32_t B, void* out, void* workspace,
+                                     size_t ws_bytes, mla_stream_t stream);
+
 /* mla_decode_absorbed with the queries and the output in HOST memory: the call copies
  * q_nope [B,H,qk_nope] and q_rope [B,H,d_hR] (storage type, rotated) host->device into the
  * workspace, runs the same decode on the stream, and copies o [B,H,v_head] device->host.

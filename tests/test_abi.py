@@ -87,6 +87,8 @@ def test_argument_errors_return_before_any_launch():
     assert lib.mla_absorb_weights(ctypes.byref(d), None, None, None, None, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_absorbed(ctypes.byref(d), None, None, None, None, None, None, 0, None, 1, None, None, 0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_prefill_causal(ctypes.byref(d), None, None, None, None, None, None, 1, 1, None, 0, None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_decode_absorbed_paged(ctypes.byref(d), None, None, None, None, 1, None, 1, None, 1, None, None,
+                                         0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_absorbed_host(ctypes.byref(d), None, None, None, None, 1, None, 1, None, None, 0,
                                         None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_weights_destroy(None) == mla.MLA_OK

@@ -415,3 +415,40 @@ def test_decode_with_host_buffers_matches_the_oracle_and_the_device_call():
     units = [(b, h) for b in range(w.B) for h in (0, 31, 127)]
     want = oracle_decode_units(w, inp, units)
     assert_close(torch.stack([out_h[b, h] for b, h in units]), want, "bf16", "host-buffer decode")
+
+
+# -------------------------------------------------------------------- paged cache
+
+def test_paged_cache_gives_the_contiguous_result():
+    """The same rows laid out in 64-token pages (random page order, junk in the unused tail
+    of each last page, spare pages): bit-identical to the contiguous decode, which the other
+    tests hold to the oracle."""
+    lengths = [300, 1, 77, 513, 0, 64, 4096, 129]
+    w, inp = reduced_attn_inputs(lengths, seed=31)
+    dev = run_decode_attn(w, inp)
+    r = np.random.default_rng(31)
+    npg = [(L + 63) // 64 for L in lengths]
+    total_pages = sum(npg) + 5
+    perm = r.permutation(total_pages)
+    pages = (torch.from_numpy(r.standard_normal((total_pages, 64, w.row))) * 3.0).to(torch.bfloat16)
+    max_blocks = max(npg) + 2
+    table = np.zeros((w.B, max_blocks), dtype=np.int32)
+    offs = inp["offsets"].numpy()
+    k = 0
+    for b, L in enumerate(lengths):
+        for j in range(npg[b]):
+            p = int(perm[k])
+            k += 1
+            table[b, j] = p
+            n = min(64, L - 64 * j)
+            pages[p, :n] = inp["cache"][offs[b] + 64 * j: offs[b] + 64 * j + n]
+    dims = dims_of(w)
+    g = to_dev({k_: inp[k_] for k_ in ("q_nope", "q_rope", "W_UK", "W_UV")})
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B))
+    out = torch.empty(w.B, w.H, w.v_head, dtype=torch.bfloat16, device=DEV)
+    mla.mla_decode_absorbed_paged(dims, weights, pages.to(DEV), torch.from_numpy(table).to(DEV),
+                                  torch.tensor(lengths, dtype=torch.int32, device=DEV), out, ws,
+                                  q_nope=g["q_nope"], q_rope=g["q_rope"])
+    assert mla.mla_get_device_error() == (0, 0)
+    assert torch.equal(out.cpu(), dev)
