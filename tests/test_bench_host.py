@@ -1,0 +1,48 @@
+"""The benchmark's host-side arithmetic: the algorithmic bytes and flops its roofline divides
+by, and the guard that drops a stale DRAM-traffic figure."""
+import json
+import os
+
+import bench
+import workloads
+
+
+def test_decode_step_algorithmic_bytes_and_flops():
+    w = workloads.WORKLOADS["v3_decode_b32_ctx4096"]
+    a = bench.alg_step(w)
+    tokens = 32 * 4096
+    assert a["tokens"] == tokens
+    assert a["cache_bytes"] == tokens * 1152                  # (512 + 64) bf16 per token
+    # cache 151.0 MB + W_UK, W_UV 33.6 MB + queries 1.6 MB + output 1.0 MB
+    assert a["bytes"] == tokens * 1152 + 2 * 128 * 128 * 512 * 2 + 32 * 128 * 192 * 2 + 32 * 128 * 128 * 2
+    assert round(a["bytes"] / 1e6, 1) == 187.2
+    # per attended token and head: 2 x 576 (scores) + 2 x 512 (P c) flops; plus the two absorptions
+    assert a["attn_flops"] == tokens * 128 * (2 * 576 + 2 * 512)
+    assert round(a["flops"] / 1e9, 1) == 37.6
+    # the dominant kernel reads the cache and the absorbed and rotary queries once
+    assert bench.alg_kernel_bytes("tc_flash_decode", w) == tokens * 1152 + 32 * 128 * 576 * 2
+
+
+def test_layer_and_prefill_steps_count_their_weights():
+    lay = bench.alg_layer(workloads.WORKLOADS["v3_layer_b128_ctx8192"])
+    # W_Q (352 MB) and W_O (235 MB) dominate the weights; the cache holds 128 x 8193 rows
+    assert lay["bytes"] > 128 * 8193 * 1152 + 352e6 + 235e6
+    pre = bench.alg_prefill(workloads.WORKLOADS["v2_prefill_b4_s4096"])
+    assert pre["tokens"] == 4 * 4096
+    assert 7.0e12 < pre["flops"] < 8.0e12
+
+
+def test_traffic_figure_is_dropped_when_the_kernel_source_changed(tmp_path, monkeypatch):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    src = tmp_path / "k.cu"
+    src.write_text("kernel v1")
+    import hashlib
+    digest = hashlib.sha256(b"kernel v1").hexdigest()
+    (prof / "traffic.json").write_text(json.dumps({"tc_x": {"source": "k.cu", "sha256": digest,
+                                                            "bytes_per_launch": 123}}))
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.traffic_for("tc_x") == 123
+    src.write_text("kernel v2")
+    assert bench.traffic_for("tc_x") is None
+    assert bench.traffic_for("tc_other") is None
