@@ -452,3 +452,17 @@ def test_paged_cache_gives_the_contiguous_result():
                                   q_nope=g["q_nope"], q_rope=g["q_rope"])
     assert mla.mla_get_device_error() == (0, 0)
     assert torch.equal(out.cpu(), dev)
+
+
+def test_decode_large_batch_spans_several_sequence_blocks():
+    """B = 200 short ragged sequences: the q-absorb kernel runs two blocks of 128 sequences
+    and the merge kernel four blocks of 64; sampled units against the oracle."""
+    r = np.random.default_rng(47)
+    lengths = [int(x) for x in r.integers(0, 300, size=200)]
+    lengths[0], lengths[129], lengths[199] = 0, 1, 299
+    w, inp = reduced_attn_inputs(lengths, seed=47)
+    out = run_decode_attn(w, inp)
+    units = [(b, h) for b in (1, 63, 64, 127, 128, 129, 150, 199) for h in (0, 77, 127)]
+    want = oracle_decode_units(w, inp, units)
+    assert_close(torch.stack([out[b, h] for b, h in units]), want, "bf16", "decode B=200")
+    assert torch.all(out[0] == 0)
