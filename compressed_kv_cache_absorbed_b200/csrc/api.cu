@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "decode_tc.cuh"
 #include "gemm_tc.cuh"
+#include "prefill_tc.cuh"
 #include "mla.h"
 
 using mla::DevErr;
@@ -587,6 +588,13 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
         e = mla::tc::gemm_bf16_tc(H, vh, n, dc, (const bf16*)w->W_UV, (long long)vh * dc, dc, (const bf16*)cache, 0,
                                   row, ovb, err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
+        if (qk == 128 && dR == 64 && vh == 128 && dc == 512 && aligned16(out)) {
+            // 4. causal attention on the tensor cores
+            mla::ProfScope ps(s, "tc_prefill_attn");
+            return mla::tc::prefill_attn_tc((const bf16*)ws.q_buf, (const bf16*)ws.k_buf, (const bf16*)cache,
+                                            (const bf16*)ws.v_buf, B, S, H, scale_of(d), (bf16*)out, err.code,
+                                            err.detail, s);
+        }
         mla::ProfScope ps(s, "simt_prefill_attn");
         return mla::launch_prefill_attn_simt<T>((const T*)ws.q_buf, (const T*)ws.k_buf, (const T*)cache,
                                                 (const T*)ws.v_buf, B, S, H, qk, dR, dc, vh, scale_of(d),

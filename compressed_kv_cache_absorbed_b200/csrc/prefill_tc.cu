@@ -1,0 +1,314 @@
+// Causal prefill attention with K and V materialised, on the tcgen05 tensor cores, for the
+// DeepSeek-V2/V3 head shape (qk_nope = 128, d_hR = 64, v_head = 128), bf16.
+//
+// For sequence b, head h and query position t (keys t' <= t of the same sequence):
+//     s[t, t'] = scale * (q_nope[t] . k_nope[t'] + q_rope[t] . k_r[t'])     (192-long)
+//     o[t]     = sum_t' softmax_t'(s[t, :]) v[t']                              (128 wide)
+// with q = [q_nope | q_rope] from the query projection, k_nope and v materialised per head,
+// and k_r the (shared) rotary key of the cache row.
+//
+// One CTA per (block of 128 queries, head, sequence).  The query block stays in shared
+// memory; key/value blocks of 128 tokens stream through a 2-stage ring (K: two 64-column
+// boxes of k_nope and the 64 rotary columns of the cache rows; V: two 64-column boxes).
+// Per key block: S = Q K^T (M = 128, N = 128, K = 192: 12 MMAs, both operands in shared
+// memory) into TMEM, the online softmax in registers (thread = query row = TMEM lane,
+// base-2, lazy rescale), P (bf16) back to TMEM, O += P V (M = 128, N = 128, K = 128: 8 MMAs
+// with A = P from TMEM and B = V from shared memory).  The diagonal block is masked causally;
+// positions at or past the sequence end are masked too.
+// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner and MMA issuer, warps
+// 2-5 softmax and epilogue.  Every wait is bounded; a timeout latches an error and the
+// kernel drains and returns.
+#include <math.h>
+
+#include "common.cuh"
+#include "prefill_tc.cuh"
+#include "tc_common.cuh"
+
+namespace mla {
+namespace tc {
+
+namespace {
+
+constexpr int kQ = 128, kKB = 128;          // queries per CTA, keys per block
+constexpr int kBox = 128 * 128;             // one 128-row x 64-column bf16 box (16 KB)
+constexpr int kQBytes = 3 * kBox;           // Q: nope 0-63, nope 64-127, rope
+constexpr int kKBytes = 3 * kBox;           // K: the same three column groups
+constexpr int kVBytes = 2 * kBox;           // V: columns 0-63, 64-127
+constexpr int kStageBytes = kKBytes + kVBytes;
+constexpr int kPfSmem = kQBytes + 2 * kStageBytes + 1024 + 256;
+static_assert(kPfSmem <= 232448, "prefill kernel shared memory over the 227 KB limit");
+constexpr uint32_t kColS = 0, kColP = 128, kColO = 256, kPfTmem = 512;
+constexpr int kPfThreads = 192;
+constexpr float kPfRescale = 8.0f;          // log2 units
+
+__device__ __forceinline__ float ex2f_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__global__ void __launch_bounds__(kPfThreads, 1)
+prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                       const __grid_constant__ CUtensorMap tm_kr, const __grid_constant__ CUtensorMap tm_v, int S,
+                       int H, float scale_log2, __nv_bfloat16* __restrict__ out, int* err_code,
+                       long long* err_detail) {
+    extern __shared__ uint8_t pf_smem_raw[];
+    uint8_t* smem = (uint8_t*)(((uintptr_t)pf_smem_raw + 1023) & ~(uintptr_t)1023);
+    uint8_t* sQ = smem;
+    uint8_t* sKV = smem + kQBytes;   // [2] stages: K (3 boxes) then V (2 boxes)
+    uint64_t* bars = (uint64_t*)(sKV + 2 * kStageBytes);
+    uint64_t* q_full = bars;
+    uint64_t* kv_full = bars + 1;    // [2]
+    uint64_t* kv_empty = bars + 3;   // [2]
+    uint64_t* s_full = bars + 5;
+    uint64_t* s_free = bars + 6;
+    uint64_t* p_ready = bars + 7;
+    uint64_t* o_done = bars + 8;
+    uint64_t* drain = bars + 9;
+    uint32_t* tmem_slot = (uint32_t*)(bars + 10);
+    volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
+
+    // longest query blocks (most key blocks) first, so the short ones fill the tail
+    const int qb = gridDim.x - 1 - blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int q0 = qb * kQ;                      // first query position in the sequence
+    const long long tok0 = (long long)b * S;     // first token row of the sequence
+    const int nkb = qb + 1;                      // key blocks 0 .. qb (causal)
+
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(q_full, 1);
+        for (int i = 0; i < 2; ++i) {
+            ptx::mbar_init(&kv_full[i], 1);
+            ptx::mbar_init(&kv_empty[i], 1);
+        }
+        ptx::mbar_init(s_full, 1);
+        ptx::mbar_init(s_free, 128);
+        ptx::mbar_init(p_ready, 128);
+        ptx::mbar_init(o_done, 1);
+        ptx::mbar_init(drain, 1);
+        *abort_flag = 0;
+        ptx::fence_mbar_init();
+    }
+    if (warp == 1) {
+        ptx::tmem_alloc(tmem_slot, kPfTmem);
+        ptx::tmem_relinquish();
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    ptx::tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    if (threadIdx.x == 0) pdl_trigger();
+
+    auto fail = [&](int where) {
+        latch(DevErr{err_code, err_detail}, kErrTimeout, 9000000 + where);
+        *abort_flag = 1;
+    };
+
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            pdl_wait();   // q, k_nope, v and the cache come from the kernels before
+            ptx::tma_prefetch(&tm_q);
+            ptx::tma_prefetch(&tm_k);
+            ptx::tma_prefetch(&tm_kr);
+            ptx::tma_prefetch(&tm_v);
+            const int qrow = (int)(tok0 + q0);
+            ptx::mbar_expect_tx(q_full, kQBytes);
+            ptx::tma_load_3d(sQ, &tm_q, q_full, 0, h, qrow);
+            ptx::tma_load_3d(sQ + kBox, &tm_q, q_full, 64, h, qrow);
+            ptx::tma_load_3d(sQ + 2 * kBox, &tm_q, q_full, 128, h, qrow);
+            int i = 0;
+            for (; i < nkb; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !ptx::mbar_wait(&kv_empty[st], ((i >> 1) - 1) & 1, abort_flag)) {
+                    fail(1);
+                    break;
+                }
+                uint8_t* dst = sKV + st * kStageBytes;
+                const int krow = (int)(tok0 + (long long)i * kKB);
+                ptx::mbar_expect_tx(&kv_full[st], kStageBytes);
+                ptx::tma_load_3d(dst, &tm_k, &kv_full[st], 0, h, krow);
+                ptx::tma_load_3d(dst + kBox, &tm_k, &kv_full[st], 64, h, krow);
+                ptx::tma_load_2d(dst + 2 * kBox, &tm_kr, &kv_full[st], 512, krow);
+                ptx::tma_load_3d(dst + kKBytes, &tm_v, &kv_full[st], 0, h, krow);
+                ptx::tma_load_3d(dst + kKBytes + kBox, &tm_v, &kv_full[st], 64, h, krow);
+            }
+            // loads in flight complete before the CTA leaves
+            ptx::mbar_wait(q_full, 0, nullptr);
+            for (int k = (i >= 2 ? i - 2 : 0); k < i; ++k) ptx::mbar_wait(&kv_full[k & 1], (k >> 1) & 1, nullptr);
+        }
+    } else if (warp == 1) {
+        // --------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, kKB, 0, 0);
+            constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 128, 0, 1);   // B = V (MN-major)
+            bool ok = ptx::mbar_wait(q_full, 0, abort_flag);
+            const uint32_t qa = ptx::smem_u32(sQ);
+            auto issue_s = [&](int i) -> bool {
+                if (!ptx::mbar_wait(&kv_full[i & 1], (i >> 1) & 1, abort_flag)) return false;
+                if (i > 0 && !ptx::mbar_wait(s_free, (i - 1) & 1, abort_flag)) return false;
+                ptx::tc_fence_after();
+                const uint32_t ka = ptx::smem_u32(sKV + (i & 1) * kStageBytes);
+#pragma unroll
+                for (int ks = 0; ks < 12; ++ks)   // 3 column groups x 4 K-steps of 16
+                    ptx::mma_ss(tmem + kColS, ptx::desc_kmajor_sw128(qa + (ks >> 2) * kBox + (ks & 3) * 32),
+                                ptx::desc_kmajor_sw128(ka + (ks >> 2) * kBox + (ks & 3) * 32), idesc_s, ks != 0);
+                ptx::mma_commit(s_full);
+                return true;
+            };
+            if (ok) ok = issue_s(0);
+            for (int i = 0; ok && i < nkb; ++i) {
+                if (i + 1 < nkb && !issue_s(i + 1)) {
+                    ok = false;
+                    break;
+                }
+                if (!ptx::mbar_wait(p_ready, i & 1, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                ptx::tc_fence_after();
+                const uint32_t va = ptx::smem_u32(sKV + (i & 1) * kStageBytes + kKBytes);
+#pragma unroll
+                for (int k = 0; k < kKB / 16; ++k)
+                    ptx::mma_ts(tmem + kColO, tmem + kColP + 8 * k, ptx::desc_mnmajor_sw128(va + 2048 * k, kBox),
+                                idesc_o, i > 0 || k > 0);
+                ptx::mma_commit(o_done);
+                ptx::mma_commit(&kv_empty[i & 1]);
+            }
+            if (!ok) fail(2);
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait(drain, 0, nullptr)) fail(3);
+        }
+    } else {
+        // ------------------------------------------------ softmax and epilogue
+        const int sub = warp & 3;                    // TMEM lane quarter of this warp
+        const int r = sub * 32 + lane;               // query row in the block
+        const int tq = q0 + r;                       // query position
+        const uint32_t lane_addr = tmem + ((uint32_t)(sub * 32) << 16);
+        auto uwait = [&](uint64_t* bar, uint32_t parity) {
+            return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, abort_flag));
+        };
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int i = 0; i < nkb; ++i) {
+            if (!uwait(s_full, i & 1)) { ok = false; break; }
+            ptx::tc_fence_after();
+            float sc[kKB];
+#pragma unroll
+            for (int c = 0; c < kKB; c += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld32(lane_addr + kColS + c, v);
+                ptx::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 32; ++j) sc[c + j] = __uint_as_float(v[j]);
+            }
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(s_free);
+            // causal mask on the diagonal block; keys at or past the sequence end
+            const int k0 = i * kKB;
+            const int lim = min(tq, S - 1) - k0;     // last allowed key offset in this block
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < kKB; ++j) {
+                sc[j] = j <= lim ? sc[j] : -INFINITY;
+                mt = fmaxf(mt, sc[j]);
+            }
+            float alpha = 1.f;
+            const bool first = (i == 0);
+            if (mt != -INFINITY && mt * scale_log2 > m_run + kPfRescale) {
+                const float m_new = mt * scale_log2;
+                alpha = first ? 0.f : ex2f_ftz(m_run - m_new);
+                m_run = m_new;
+            }
+            // P and O are free once the O MMAs of the previous block have completed
+            if (i > 0 && !uwait(o_done, (i - 1) & 1)) { ok = false; break; }
+            ptx::tc_fence_after();
+            if (__any_sync(0xffffffffu, !first && alpha != 1.f)) {
+#pragma unroll 1
+                for (int c = 0; c < 128; c += 32) {
+                    uint32_t v[32];
+                    ptx::tmem_ld32(lane_addr + kColO + c, v);
+                    ptx::tmem_wait_ld();
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __float_as_uint(__uint_as_float(v[j]) * alpha);
+                    ptx::tmem_st32(lane_addr + kColO + c, v);
+                }
+            }
+            // P = 2^(s scale_log2 - m) as bf16 pairs, 32 keys (16 TMEM columns) at a time
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < kKB; c += 32) {
+                uint32_t pw[16];
+#pragma unroll
+                for (int j = 0; j < 32; j += 2) {
+                    const float p0 = ex2f_ftz(fmaf(sc[c + j], scale_log2, -m_run));
+                    const float p1 = ex2f_ftz(fmaf(sc[c + j + 1], scale_log2, -m_run));
+                    sum += p0 + p1;
+                    pw[j / 2] = ptx::pack_bf16(p0, p1);
+                }
+                ptx::tmem_st16(lane_addr + kColP + c / 2, pw);
+            }
+            l_run = l_run * alpha + sum;
+            ptx::tmem_wait_st();
+            ptx::tc_fence_before();
+            ptx::mbar_arrive(p_ready);
+        }
+        // epilogue: o = O / l for the queries inside the sequence
+        if (ok) ok = uwait(o_done, (nkb - 1) & 1);
+        if (ok) {
+            ptx::tc_fence_after();
+            const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+            __nv_bfloat16* dst = out + ((tok0 + tq) * H + h) * 128;
+#pragma unroll 1
+            for (int c = 0; c < 128; c += 32) {
+                uint32_t v[32];
+                ptx::tmem_ld32(lane_addr + kColO + c, v);
+                ptx::tmem_wait_ld();
+                if (tq < S) {
+#pragma unroll
+                    for (int j = 0; j < 32; j += 8)
+                        *(uint4*)(dst + c + j) = make_uint4(
+                            ptx::pack_bf16(__uint_as_float(v[j]) * inv, __uint_as_float(v[j + 1]) * inv),
+                            ptx::pack_bf16(__uint_as_float(v[j + 2]) * inv, __uint_as_float(v[j + 3]) * inv),
+                            ptx::pack_bf16(__uint_as_float(v[j + 4]) * inv, __uint_as_float(v[j + 5]) * inv),
+                            ptx::pack_bf16(__uint_as_float(v[j + 6]) * inv, __uint_as_float(v[j + 7]) * inv));
+                }
+            }
+        } else if (lane == 0) {
+            fail(4);
+        }
+    }
+    ptx::tc_fence_before();
+    __syncthreads();
+    if (warp == 1) ptx::tmem_dealloc(tmem, kPfTmem);
+}
+
+}  // namespace
+
+cudaError_t prefill_attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* k_nope, const __nv_bfloat16* cache,
+                            const __nv_bfloat16* v, int B, int S, int H, float scale, __nv_bfloat16* out,
+                            int* err_code, long long* err_detail, cudaStream_t s) {
+    if (B <= 0 || S <= 0) return cudaSuccess;
+    const uint64_t n = (uint64_t)B * S;
+    CUtensorMap mq, mk, mkr, mv;
+    const uint64_t dq[3] = {192, (uint64_t)H, n};
+    const uint64_t sq[2] = {192 * 2, (uint64_t)H * 192 * 2};
+    const uint64_t dk[3] = {128, (uint64_t)H, n};
+    const uint64_t sk[2] = {128 * 2, (uint64_t)H * 128 * 2};
+    const uint32_t box3[3] = {64, 1, 128};
+    const uint64_t dr[2] = {576, n};
+    const uint64_t sr[1] = {576 * 2};
+    const uint32_t box2[2] = {64, 128};
+    if (!make_tmap_bf16(&mq, q, 3, dq, sq, box3) || !make_tmap_bf16(&mk, k_nope, 3, dk, sk, box3) ||
+        !make_tmap_bf16(&mkr, cache, 2, dr, sr, box2) || !make_tmap_bf16(&mv, v, 3, dk, sk, box3))
+        return cudaErrorInvalidValue;
+    static const cudaError_t attr =
+        cudaFuncSetAttribute(prefill_attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPfSmem);
+    if (attr != cudaSuccess) return attr;
+    dim3 grid((S + kQ - 1) / kQ, H, B);
+    return launch_pdl(prefill_attn_tc_kernel, grid, dim3(kPfThreads), kPfSmem, s, mq, mk, mkr, mv, S, H,
+                      scale * 1.4426950408889634f, out, err_code, err_detail);
+}
+
+}  // namespace tc
+}  // namespace mla

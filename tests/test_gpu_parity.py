@@ -316,6 +316,17 @@ def test_prefill_reduced(B, S):
     assert_close(out[1, [0, 150], 3], res[3], "bf16", "prefill naive")
 
 
+def test_prefill_every_query_of_one_head():
+    """Every query position of a 3-block sequence (ragged last block) for one head, so each
+    row of the causal mask and each block boundary is checked."""
+    w = workloads.shrink(workloads.WORKLOADS["v2_prefill_b4_s4096"], B=1, ctx=300, seed=78)
+    inp = workloads.make_inputs(w)
+    out, _ = run_prefill(w, inp)
+    t_list = list(range(300))
+    res, _ = oracle_prefill(w, inp, 0, t_list, [77])
+    assert_close(out[0, t_list, 77], res[77], "bf16", "prefill every query")
+
+
 def test_prefill_full_size_sampled():
     w = workloads.WORKLOADS["v2_prefill_b4_s4096"]
     inp = workloads.make_inputs(w)
@@ -393,7 +404,9 @@ def test_v3_bf16_paths_run_the_tensor_core_kernels():
     finally:
         mla.mla_profile_enable(False)
     names = set(mla.mla_profile_report(reset=True))
-    assert {"tc_append_proj_rope", "tc_q_proj_rope", "tc_k_materialise", "tc_v_materialise"} <= names, names
+    assert {"tc_append_proj_rope", "tc_q_proj_rope", "tc_k_materialise", "tc_v_materialise",
+            "tc_prefill_attn"} <= names, names
+    assert not any(n.startswith("simt_") for n in names), names
 
 
 # ------------------------------------------------------------ host-buffer decode
