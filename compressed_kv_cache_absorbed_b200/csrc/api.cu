@@ -579,14 +579,15 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
         if (e != cudaSuccess) return e;
         // 3. K_nope[t, h] = W_UK[h] c_t and V[t, h] = W_UV[h] c_t: one B (the cache rows) for all heads
         { mla::ProfScope ps(s, "tc_k_materialise");
-        mla::tc::GemmOut okb{ws.k_buf, qk, 1, (long long)H * qk, 0};
-        e = mla::tc::gemm_bf16_tc(H, qk, n, dc, (const bf16*)w->W_UK, (long long)qk * dc, dc, (const bf16*)cache, 0,
-                                  row, okb, err.code, err.detail, s); }
+        // all heads in one product: W_UK as [H * qk, d_c] rows, K_nope[t] = [H * qk] wide
+        mla::tc::GemmOut okb{ws.k_buf, 0, 1, (long long)H * qk, 0};
+        e = mla::tc::gemm_bf16_tc(1, H * qk, n, dc, (const bf16*)w->W_UK, 0, dc, (const bf16*)cache, 0, row, okb,
+                                  err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
         { mla::ProfScope ps(s, "tc_v_materialise");
-        mla::tc::GemmOut ovb{ws.v_buf, vh, 1, (long long)H * vh, 0};
-        e = mla::tc::gemm_bf16_tc(H, vh, n, dc, (const bf16*)w->W_UV, (long long)vh * dc, dc, (const bf16*)cache, 0,
-                                  row, ovb, err.code, err.detail, s); }
+        mla::tc::GemmOut ovb{ws.v_buf, 0, 1, (long long)H * vh, 0};
+        e = mla::tc::gemm_bf16_tc(1, H * vh, n, dc, (const bf16*)w->W_UV, 0, dc, (const bf16*)cache, 0, row, ovb,
+                                  err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
         if (qk == 128 && dR == 64 && vh == 128 && dc == 512 && aligned16(out)) {
             // 4. causal attention on the tensor cores

@@ -1,11 +1,22 @@
 // Batched bf16 GEMM on the tcgen05 tensor cores.
 //
-// One 128 x BN output tile per CTA.  Warp 0 streams 128x64 A and BNx64 B tiles (128-byte
-// swizzled) into a ring of shared-memory stages with TMA; warp 1 allocates TMEM and issues
-// tcgen05.mma (M = 128, N = BN, K = 16) into a fp32 TMEM accumulator, releasing each stage
-// with tcgen05.commit; warps 2-5 read the accumulator back with tcgen05.ld (one TMEM lane
-// = one output row per thread) and store it.  Every wait is bounded: on a timeout the
-// kernel latches an error, drains the MMAs it issued, frees TMEM and returns.
+// Persistent: one CTA per SM walks the output tiles (128 x BN) in a grouped order (16
+// row-tiles by all column-tiles, so that both operands of the tiles in flight stay in L2).
+// Warp 0 streams 128x64 X and BNx64 Y tiles (128-byte swizzled) into a ring of
+// shared-memory stages with TMA, across tile boundaries; warp 1 allocates TMEM and issues
+// tcgen05.mma (M = 128, N = BN, K = 16) into one of two fp32 TMEM accumulators, releasing
+// each stage with tcgen05.commit; warps 2-5 read a finished accumulator back with
+// tcgen05.ld (one TMEM lane = one output row of the tile per thread) and store it while the
+// next tile accumulates into the other one.  Every wait is bounded: on a timeout the kernel
+// latches an error, drains the MMAs it issued and the loads in flight, frees TMEM and
+// returns.
+//
+// Two orientations of the same product C = A B^T:
+//  - weights-major (X = A, Y = B): a thread owns an output feature m and writes it for BN
+//    tokens n (a warp writes 32 consecutive features of one token at a time).  Used for
+//    few tokens, where the weights stream from HBM and more row-tiles mean more CTAs.
+//  - token-major (X = B, Y = A): a thread owns a token n and writes 32 consecutive features
+//    of it as four 16-byte stores; rotary pairs are adjacent columns of one thread.
 #include "common.cuh"
 #include "gemm_tc.cuh"
 #include "tc_common.cuh"
@@ -15,52 +26,88 @@ namespace tc {
 
 namespace {
 
-constexpr int kBM = 128, kBK = 64;
+constexpr int kBM = 128, kBK = 64, kGroupRows = 16;
+constexpr int kSwapMinTokens = 1024;   // token-major from this many tokens on
 
 template <int BN>
 struct GemmCfg {
-    static constexpr int A_BYTES = kBM * kBK * 2;
-    static constexpr int B_BYTES = BN * kBK * 2;
-    static constexpr int STAGE = A_BYTES + B_BYTES;
-    static constexpr int MAX_STAGES = (196608 / STAGE) > 8 ? 8 : (196608 / STAGE);
-    static constexpr int TMEM_COLS = BN < 32 ? 32 : BN;
-    static constexpr int smem(int stages) { return stages * STAGE + 1024 + 256; }
+    static constexpr int X_BYTES = kBM * kBK * 2;
+    static constexpr int Y_BYTES = BN * kBK * 2;
+    static constexpr int STAGE = X_BYTES + Y_BYTES;
+    static constexpr int STAGES = (196608 / STAGE) > 8 ? 8 : (196608 / STAGE);
+    static constexpr int ACC_COLS = BN < 32 ? 32 : BN;   // one accumulator; two are allocated
+    static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
 
 __device__ __forceinline__ void fail(int* code, long long* detail, volatile int* abort_flag, int where) {
-    latch(DevErr{code, detail}, kErrTimeout, (long long)where * 1000000 + blockIdx.x * 1000 + blockIdx.y);
+    latch(DevErr{code, detail}, kErrTimeout, (long long)where * 1000000 + blockIdx.x);
     *abort_flag = 1;
+}
+
+struct Tile {
+    int z, i0, j0;   // batch, first X row, first Y row
+};
+
+// tile t -> (z, X row-tile, Y row-tile): groups of kGroupRows X row-tiles, Y fastest-varying
+// across the group's columns
+__device__ __forceinline__ Tile tile_of(int t, int tiles_x, int tiles_y, int BN) {
+    const int per = tiles_x * tiles_y;
+    const int z = t / per, r = t % per;
+    const int g = r / (kGroupRows * tiles_y);
+    const int first = g * kGroupRows;
+    const int gs = min(kGroupRows, tiles_x - first);
+    const int w = r - g * kGroupRows * tiles_y;
+    return Tile{z, (first + w % gs) * kBM, (w / gs) * BN};
+}
+
+// (cos, sin) of the rotary angle of pair pi at token n
+__device__ __noinline__ double2 rope_cs(const double2* tab, int d_rope, const int32_t* pos, int pos_mod, float theta,
+                                       int n, int pi) {
+    if (tab) return tab[(long long)n * (d_rope >> 1) + pi];
+    const int p = pos ? pos[n] : n % pos_mod;
+    const double inv = pow((double)theta, -2.0 * (double)pi / (double)d_rope);
+    double sn, cs;
+    sincos((double)p * inv, &sn, &cs);
+    return make_double2(cs, sn);
 }
 
 template <int BN>
 __global__ void __launch_bounds__(192, 1)
-gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB, int M,
-                    int N, int K, int stages, GemmOut out, int chain_head, int b_bcast, int* err_code,
-                    long long* err_detail) {
+gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmY, int Mx,
+                    int Ny, int K, int Z, GemmOut out, int chain_head, int x_2d, int y_2d, int swap,
+                    int* err_code, long long* err_detail) {
     using C = GemmCfg<BN>;
+    constexpr int stages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
     uint64_t* full = (uint64_t*)(smem + stages * C::STAGE);
     uint64_t* empty = full + stages;
-    uint64_t* accum = empty + stages;
-    uint32_t* tmem_slot = (uint32_t*)(accum + 1);
+    uint64_t* acc_full = empty + stages;   // [2]
+    uint64_t* acc_empty = acc_full + 2;    // [2]
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_slot = (uint32_t*)(drain + 1);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kBM, n0 = blockIdx.x * BN, z = blockIdx.z;
     const int nk = (K + kBK - 1) / kBK;
+    const int tiles_x = (Mx + kBM - 1) / kBM, tiles_y = (Ny + BN - 1) / BN;
+    const int tiles = Z * tiles_x * tiles_y;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < stages; ++s) {
             ptx::mbar_init(&full[s], 1);
             ptx::mbar_init(&empty[s], 1);
         }
-        ptx::mbar_init(accum, 1);
+        for (int b = 0; b < 2; ++b) {
+            ptx::mbar_init(&acc_full[b], 1);
+            ptx::mbar_init(&acc_empty[b], 128);
+        }
+        ptx::mbar_init(drain, 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == 1) {
-        ptx::tmem_alloc(tmem_slot, C::TMEM_COLS);
+        ptx::tmem_alloc(tmem_slot, 2 * C::ACC_COLS);
         ptx::tmem_relinquish();
     }
     ptx::tc_fence_before();
@@ -77,97 +124,176 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 
     if (warp == 0) {
         if (lane == 0) {
-            ptx::tma_prefetch(&tmA);
-            ptx::tma_prefetch(&tmB);
-            // A (the weights) of the first stages does not depend on earlier kernels: start it
-            // before waiting for them; B and the output do.
-            const int pre = nk < stages ? nk : stages;
-            for (int kb = 0; kb < pre; ++kb) {
-                ptx::mbar_expect_tx(&full[kb], C::STAGE);
-                ptx::tma_load_3d(smem + kb * C::STAGE, &tmA, &full[kb], kb * kBK, m0, z);
+            ptx::tma_prefetch(&tmX);
+            ptx::tma_prefetch(&tmY);
+            auto load_x = [&](uint8_t* st, uint64_t* bar, int kb, const Tile& tl) {
+                if (x_2d)
+                    ptx::tma_load_2d(st, &tmX, bar, kb * kBK, tl.i0);
+                else
+                    ptx::tma_load_3d(st, &tmX, bar, kb * kBK, tl.i0, tl.z);
+            };
+            auto load_y = [&](uint8_t* st, uint64_t* bar, int kb, const Tile& tl) {
+                if (y_2d)
+                    ptx::tma_load_2d(st + C::X_BYTES, &tmY, bar, kb * kBK, tl.j0);
+                else
+                    ptx::tma_load_3d(st + C::X_BYTES, &tmY, bar, kb * kBK, tl.j0, tl.z);
+            };
+            // The weights (X weights-major, Y token-major) of the first stages do not depend
+            // on earlier kernels: start them before waiting for those; the activations do.
+            int pre = 0;
+            if ((int)blockIdx.x < tiles) {
+                const Tile tl = tile_of(blockIdx.x, tiles_x, tiles_y, BN);
+                pre = nk < stages ? nk : stages;
+                for (int kb = 0; kb < pre; ++kb) {
+                    ptx::mbar_expect_tx(&full[kb], C::STAGE);
+                    if (swap)
+                        load_y(smem + kb * C::STAGE, &full[kb], kb, tl);
+                    else
+                        load_x(smem + kb * C::STAGE, &full[kb], kb, tl);
+                }
             }
             pdl_wait();
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % stages;
-                const uint32_t ph = (kb / stages) & 1;
-                uint8_t* a = smem + s * C::STAGE;
-                if (kb >= pre) {
-                    if (!ptx::mbar_wait(&empty[s], ph ^ 1, abort_flag)) {
-                        fail(err_code, err_detail, abort_flag, 1);
-                        break;
+            int it = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x) {
+                const Tile tl = tile_of(t, tiles_x, tiles_y, BN);
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % stages;
+                    uint8_t* st = smem + s * C::STAGE;
+                    if (it >= pre) {
+                        if (it >= stages && !ptx::mbar_wait(&empty[s], ((it / stages) & 1) ^ 1, abort_flag)) {
+                            fail(err_code, err_detail, abort_flag, 1);
+                            ok = false;
+                            break;
+                        }
+                        ptx::mbar_expect_tx(&full[s], C::STAGE);
+                        if (swap)
+                            load_y(st, &full[s], kb, tl);
+                        else
+                            load_x(st, &full[s], kb, tl);
                     }
-                    ptx::mbar_expect_tx(&full[s], C::STAGE);
-                    ptx::tma_load_3d(a, &tmA, &full[s], kb * kBK, m0, z);
+                    if (swap)
+                        load_x(st, &full[s], kb, tl);
+                    else
+                        load_y(st, &full[s], kb, tl);
                 }
-                if (b_bcast)
-                    ptx::tma_load_2d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0);
-                else
-                    ptx::tma_load_3d(a + C::A_BYTES, &tmB, &full[s], kb * kBK, n0, z);
             }
+            // the loads in flight land before the CTA leaves
+            for (int k = (it > stages ? it - stages : 0); k < it; ++k)
+                ptx::mbar_wait(&full[k % stages], (k / stages) & 1, nullptr);
         }
     } else if (warp == 1) {
         if (lane == 0) {
             constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN, 0, 0);
-            for (int kb = 0; kb < nk; ++kb) {
-                const int s = kb % stages;
-                const uint32_t ph = (kb / stages) & 1;
-                if (!ptx::mbar_wait(&full[s], ph, abort_flag)) {
-                    fail(err_code, err_detail, abort_flag, 2);
+            int it = 0, lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
+                const int buf = lt & 1;
+                if (lt >= 2 && !ptx::mbar_wait(&acc_empty[buf], ((lt >> 1) - 1) & 1, abort_flag)) {
+                    ok = false;
                     break;
                 }
                 ptx::tc_fence_after();
-                const uint32_t a = ptx::smem_u32(smem + s * C::STAGE);
-                const uint32_t b = a + C::A_BYTES;
+                const uint32_t d = tmem + buf * C::ACC_COLS;
+                for (int kb = 0; kb < nk; ++kb, ++it) {
+                    const int s = it % stages;
+                    if (!ptx::mbar_wait(&full[s], (it / stages) & 1, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    ptx::tc_fence_after();
+                    const uint32_t a = ptx::smem_u32(smem + s * C::STAGE);
+                    const uint32_t b = a + C::X_BYTES;
 #pragma unroll
-                for (int k = 0; k < kBK / 16; ++k)
-                    ptx::mma_ss(tmem, ptx::desc_kmajor_sw128(a + 32 * k), ptx::desc_kmajor_sw128(b + 32 * k),
-                                idesc, (kb | k) != 0);
-                ptx::mma_commit(&empty[s]);
+                    for (int k = 0; k < kBK / 16; ++k)
+                        ptx::mma_ss(d, ptx::desc_kmajor_sw128(a + 32 * k), ptx::desc_kmajor_sw128(b + 32 * k), idesc,
+                                    (kb | k) != 0);
+                    ptx::mma_commit(&empty[s]);
+                }
+                if (ok) ptx::mma_commit(&acc_full[buf]);
             }
+            if (!ok) fail(err_code, err_detail, abort_flag, 2);
             // completes once every MMA issued above has finished (also after an abort)
-            ptx::mma_commit(accum);
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait(drain, 0, nullptr)) fail(err_code, err_detail, abort_flag, 3);
         }
     } else {
         const int sub = warp & 3;
         pdl_wait();   // the output may still be read by an earlier kernel
-        const bool ok = ptx::mbar_wait(accum, 0, nullptr);
-        if (!ok) fail(err_code, err_detail, abort_flag, 3);
-        ptx::tc_fence_after();
-        const int row = m0 + sub * 32 + lane;
-        const int within = out.period > 0 ? row % out.period : -1;
-        const bool rope_row = out.period > 0 && within >= out.rope_start;
-        if (ok && !*abort_flag && nk > 0) {
+        int lt = 0;
+        bool ok = true;
+        for (int t = blockIdx.x; t < tiles; t += gridDim.x, ++lt) {
+            const int buf = lt & 1;
+            ok = __all_sync(0xffffffffu, ptx::mbar_wait(&acc_full[buf], (lt >> 1) & 1, abort_flag));
+            if (!ok) break;
+            ptx::tc_fence_after();
+            const Tile tl = tile_of(t, tiles_x, tiles_y, BN);
+            const uint32_t taddr = tmem + ((uint32_t)(sub * 32) << 16) + buf * C::ACC_COLS;
+            const int xr = tl.i0 + sub * 32 + lane;   // this thread's X row
+            char* base = (char*)out.C;
 #pragma unroll 1
             for (int c0 = 0; c0 < BN; c0 += 32) {
                 uint32_t r[32];
-                ptx::tmem_ld32(tmem + ((uint32_t)(sub * 32) << 16) + c0, r);
+                ptx::tmem_ld32(taddr + c0, r);
                 ptx::tmem_wait_ld();
-                char* base = (char*)out.C;
+                if (c0 + 32 >= BN) {   // the accumulator may be reused from here on
+                    ptx::tc_fence_before();
+                    ptx::mbar_arrive(&acc_empty[buf]);
+                }
+                if (*abort_flag) continue;
+                if (swap) {
+                    // token xr, features f0 .. f0 + 31 (Ny % 32 == 0: all or none in range)
+                    const int f0 = tl.j0 + c0;
+                    if (xr >= Mx || f0 >= Ny) continue;
+                    long long orow = xr;
+                    if (out.slot) {
+                        orow = out.slot[xr];
+                        if (orow < 0 || orow >= out.cap) {
+                            latch(DevErr{err_code, err_detail}, kErrOutOfRange, xr);
+                            continue;
+                        }
+                    }
+                    float v[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r[j]);
+                    if (out.period > 0) {
+#pragma unroll
+                        for (int j = 0; j < 32; j += 2) {
+                            const int within = (f0 + j) % out.period;
+                            if (within < out.rope_start) continue;
+                            const double2 t = rope_cs(out.rope_tab, out.d_rope, out.pos, out.pos_mod, out.theta, xr, (within - out.rope_start) >> 1);
+                            const double ve = v[j], vo = v[j + 1];
+                            v[j] = (float)(ve * t.x - vo * t.y);
+                            v[j + 1] = (float)(ve * t.y + vo * t.x);
+                        }
+                    }
+                    uint4* dst = (uint4*)((__nv_bfloat16*)base + (long long)tl.z * out.sz + f0 + orow * out.sn);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(ptx::pack_bf16(v[8 * q], v[8 * q + 1]), ptx::pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                            ptx::pack_bf16(v[8 * q + 4], v[8 * q + 5]),
+                                            ptx::pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                    continue;
+                }
+                // weights-major: feature row xr, tokens n0 + c0 .. + 31
+                const int row = xr;
+                const int within = out.period > 0 ? row % out.period : -1;
+                const bool rope_row = out.period > 0 && within >= out.rope_start;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
-                    const int n = n0 + c0 + j;   // the same for the whole warp
-                    if (n >= N) continue;
+                    const int n = tl.j0 + c0 + j;   // the same for the whole warp
+                    if (n >= Ny) continue;
                     float v = __uint_as_float(r[j]);
                     if (out.period > 0) {
                         // rows m and m ^ 1 are adjacent lanes: the pair (even, odd) is rotated
                         const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
                         if (rope_row) {
-                            const int pi = (within - out.rope_start) >> 1;
-                            double cs, sn;
-                            if (out.rope_tab) {
-                                const double2 t = out.rope_tab[(long long)n * (out.d_rope >> 1) + pi];
-                                cs = t.x;
-                                sn = t.y;
-                            } else {
-                                const int p = out.pos ? out.pos[n] : n % out.pos_mod;
-                                const double inv = pow((double)out.theta, -2.0 * (double)pi / (double)out.d_rope);
-                                sincos((double)p * inv, &sn, &cs);
-                            }
-                            v = (row & 1) ? (float)((double)partner * sn + (double)v * cs)
-                                          : (float)((double)v * cs - (double)partner * sn);
+                            const double2 t = rope_cs(out.rope_tab, out.d_rope, out.pos, out.pos_mod, out.theta, n, (within - out.rope_start) >> 1);
+                            v = (row & 1) ? (float)((double)partner * t.y + (double)v * t.x)
+                                          : (float)((double)v * t.x - (double)partner * t.y);
                         }
                     }
-                    if (row >= M) continue;
+                    if (row >= Mx) continue;
                     long long orow = n;
                     if (out.slot) {
                         orow = out.slot[n];
@@ -176,7 +302,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                             continue;
                         }
                     }
-                    const long long idx = (long long)z * out.sz + (long long)row * out.sm + orow * out.sn;
+                    const long long idx = (long long)tl.z * out.sz + (long long)row * out.sm + orow * out.sn;
                     if (out.f32)
                         ((float*)base)[idx] = v;
                     else
@@ -184,28 +310,30 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 }
             }
         }
+        if (!ok && lane == 0) fail(err_code, err_detail, abort_flag, 4);
     }
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == 1) ptx::tmem_dealloc(tmem, C::TMEM_COLS);
+    if (warp == 1) ptx::tmem_dealloc(tmem, 2 * C::ACC_COLS);
 }
 
 template <int BN>
-cudaError_t launch(int Z, int M, int N, int K, const CUtensorMap& ma, const CUtensorMap& mb, const GemmOut& out,
-                   bool chain_head, bool b_bcast, int* err_code, long long* err_detail, cudaStream_t s) {
+cudaError_t launch(int Z, int Mx, int Ny, int K, const CUtensorMap& mx, const CUtensorMap& my, const GemmOut& out,
+                   bool chain_head, bool x_2d, bool y_2d, bool swap, int sms, int* err_code,
+                   long long* err_detail, cudaStream_t s) {
     using C = GemmCfg<BN>;
     static bool attr_set = false;   // the attribute is per function; set it once
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             C::smem(C::MAX_STAGES));
+        cudaError_t e =
+            cudaFuncSetAttribute(gemm_bf16_tc_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
-    const int nk = (K + kBK - 1) / kBK;
-    const int stages = nk < C::MAX_STAGES ? (nk < 2 ? 2 : nk) : C::MAX_STAGES;
-    dim3 grid((N + BN - 1) / BN, (M + kBM - 1) / kBM, Z);
-    return launch_pdl(gemm_bf16_tc_kernel<BN>, grid, dim3(192), C::smem(stages), s, ma, mb, M, N, K, stages, out,
-                      (int)chain_head, (int)b_bcast, err_code, err_detail);
+    const long long tiles = (long long)Z * ((Mx + kBM - 1) / kBM) * ((Ny + BN - 1) / BN);
+    if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const int grid = (int)(tiles < sms ? tiles : sms);
+    return launch_pdl(gemm_bf16_tc_kernel<BN>, dim3(grid), dim3(192), C::SMEM, s, mx, my, Mx, Ny, K, Z, out,
+                      (int)chain_head, (int)x_2d, (int)y_2d, (int)swap, err_code, err_detail);
 }
 
 __global__ void __launch_bounds__(256)
@@ -236,18 +364,25 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
                          int* err_code, long long* err_detail, cudaStream_t s, bool chain_head) {
     if (Z <= 0 || M <= 0 || N <= 0 || K <= 0) return cudaSuccess;
-    // the narrowest tile that covers N, narrowed further while the grid has fewer CTAs than a
-    // quarter of the SMs (very skinny weight-streaming GEMMs: A is then re-read from L2)
     static int sms = 0;
     if (sms == 0) {
         int dev = 0;
         cudaGetDevice(&dev);
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) sms = 148;
     }
-    int BN = N <= 32 ? 32 : N <= 64 ? 64 : N <= 128 ? 128 : 256;
-    const long long mtiles = (long long)Z * ((M + 127) / 128);
-    while (BN > 32 && mtiles * ((N + BN - 1) / BN) < sms / 4) BN >>= 1;
+    // token-major for many tokens when the output rows take 16-byte stores
+    const bool swap = N >= kSwapMinTokens && !out.f32 && out.sm == 1 && M % 32 == 0 && out.sz % 8 == 0 &&
+                      out.sn % 8 == 0 && ((uintptr_t)out.C & 15) == 0 &&
+                      (out.period == 0 || (out.period % 2 == 0 && out.rope_start % 2 == 0));
+    const int Mx = swap ? N : M, Ny = swap ? M : N;   // MMA rows (128-tiles) and columns (BN-tiles)
+    // the narrowest tile that covers Ny, narrowed further while there are fewer tiles than a
+    // quarter of the SMs (very skinny weight-streaming GEMMs: the weights are then re-read
+    // from L2)
+    int BN = Ny <= 32 ? 32 : Ny <= 64 ? 64 : Ny <= 128 ? 128 : 256;
+    const long long xtiles = (long long)Z * ((Mx + 127) / 128);
+    while (BN > 32 && xtiles * ((Ny + BN - 1) / BN) < sms / 4) BN >>= 1;
     const bool b_bcast = sBz == 0;   // one B for every z: a 2-D map
+    const bool a_bcast = sAz == 0 && Z > 1;
     if (Z == 1) {
         sAz = (long long)M * sAm;
         sBz = (long long)N * sBn;
@@ -255,17 +390,23 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     CUtensorMap ma, mb;
     const uint64_t da[3] = {(uint64_t)K, (uint64_t)M, (uint64_t)Z};
     const uint64_t sa[2] = {(uint64_t)sAm * 2, (uint64_t)sAz * 2};
-    const uint32_t ba[3] = {(uint32_t)kBK, (uint32_t)kBM, 1};
     const uint64_t db[3] = {(uint64_t)K, (uint64_t)N, (uint64_t)Z};
     const uint64_t sb[2] = {(uint64_t)sBn * 2, (uint64_t)sBz * 2};
-    const uint32_t bb[3] = {(uint32_t)kBK, (uint32_t)BN, 1};
-    if (!make_tmap_bf16(&ma, A, 3, da, sa, ba) || !make_tmap_bf16(&mb, B, b_bcast ? 2 : 3, db, sb, bb))
+    const uint32_t bx[3] = {(uint32_t)kBK, (uint32_t)kBM, 1};   // the 128-row operand
+    const uint32_t by[3] = {(uint32_t)kBK, (uint32_t)BN, 1};    // the BN-row operand
+    if (!make_tmap_bf16(&ma, A, a_bcast ? 2 : 3, da, sa, swap ? by : bx) ||
+        !make_tmap_bf16(&mb, B, b_bcast ? 2 : 3, db, sb, swap ? bx : by))
         return cudaErrorInvalidValue;
+    const CUtensorMap& mx = swap ? mb : ma;
+    const CUtensorMap& my = swap ? ma : mb;
+    const bool x_2d = swap ? b_bcast : a_bcast, y_2d = swap ? a_bcast : b_bcast;
     switch (BN) {
-        case 32: return launch<32>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
-        case 64: return launch<64>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
-        case 128: return launch<128>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
-        default: return launch<256>(Z, M, N, K, ma, mb, out, chain_head, b_bcast, err_code, err_detail, s);
+        case 32: return launch<32>(Z, Mx, Ny, K, mx, my, out, chain_head, x_2d, y_2d, swap, sms, err_code, err_detail, s);
+        case 64: return launch<64>(Z, Mx, Ny, K, mx, my, out, chain_head, x_2d, y_2d, swap, sms, err_code, err_detail, s);
+        case 128:
+            return launch<128>(Z, Mx, Ny, K, mx, my, out, chain_head, x_2d, y_2d, swap, sms, err_code, err_detail, s);
+        default:
+            return launch<256>(Z, Mx, Ny, K, mx, my, out, chain_head, x_2d, y_2d, swap, sms, err_code, err_detail, s);
     }
 }
 

@@ -61,8 +61,10 @@ def check_rows(gpu_rows: torch.Tensor, want64: np.ndarray, dtype: str, what: str
 
 
 @pytest.mark.parametrize("name,n", [("tiny_fp32_layer", 37), ("v3_layer_b128_ctx8192", 128),
-                                    ("v2_prefill_b4_s4096", 200)])
+                                    ("v2_prefill_b4_s4096", 200), ("v2_prefill_b4_s4096", 1300)])
 def test_append_rows_and_layout(name, n):
+    """n = 1300 takes the token-major GEMM orientation (a thread per token, 16-byte row
+    stores, rotary pairs inside one thread); the others the weights-major one."""
     w = workloads.WORKLOADS[name]
     d = workloads.make_weights(w)
     dims = dims_of(w)
@@ -314,6 +316,20 @@ def test_prefill_reduced(B, S):
         check_rows(cache[b * S:(b + 1) * S], rows, "bf16", "prefill cache")
     res, _ = oracle_prefill(w, inp, 1, [0, 150], [3], absorbed=False)
     assert_close(out[1, [0, 150], 3], res[3], "bf16", "prefill naive")
+
+
+def test_prefill_token_major_projections():
+    """1100 tokens: the query, K and V projections run token-major; 9 query blocks with a
+    ragged last one."""
+    w = workloads.shrink(workloads.WORKLOADS["v2_prefill_b4_s4096"], B=1, ctx=1100, seed=79)
+    inp = workloads.make_inputs(w)
+    out, cache = run_prefill(w, inp)
+    t_list = [0, 1, 127, 128, 500, 1023, 1024, 1098, 1099]
+    heads = [0, 33, 127]
+    res, rows = oracle_prefill(w, inp, 0, t_list, heads)
+    for h in heads:
+        assert_close(out[0, t_list, h], res[h], "bf16", f"prefill token-major h={h}")
+    check_rows(cache[:1100], rows, "bf16", "prefill cache token-major")
 
 
 def test_prefill_every_query_of_one_head():
