@@ -53,6 +53,8 @@ def _declare(lib):
     lib.oracle_attend_probs.argtypes = att[:-1]
     lib.oracle_decode.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, _D, _P, _P, _P, _P, _P, _P,
                                   _I32, _P, _P, _P, _P]
+    lib.oracle_decode_multi.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, _I32, _D, _P, _P, _P, _P, _P,
+                                        _P, _I32, _P, _P, _P, _P]
     lib.oracle_out_proj.argtypes = [_I32, _I32, _I32, _P, _P, _P]
     lib.oracle_prefill_head.argtypes = [_I32, _I32, _I32, _I32, _I32, _I32, _D, _P, _P, _P, _P, _P,
                                         _I32, _P, _P]
@@ -190,6 +192,37 @@ def decode(q_nope, q_rope, rows, offsets, W_UK, W_UV, scale: float,
     if units is None:
         return o.reshape(B, H, v_head), lse.reshape(B, H)
     return o, lse
+
+
+def decode_multi(q_nope, q_rope, rows, offsets, W_UK, W_UV, scale: float,
+                 units: Optional[Sequence[Tuple[int, int, int]]] = None, absorbed: bool = False,
+                 lib=None) -> np.ndarray:
+    """Multi-token decode per (b, t, h) unit: new token t of sequence b (the last q_len rows
+    of the sequence are the new tokens) attends to the sequence's rows up to its own.
+
+    rows: [total, d_c+d_hR]; offsets: [B+1]; q_nope [B,q_len,H,qk_nope]; q_rope [B,q_len,H,d_hR].
+    Returns o: [B,q_len,H,v_head] when units is None, else [len(units), v_head].
+    """
+    qn, qr, rows, wk, wv = f64(q_nope), f64(q_rope), f64(rows), f64(W_UK), f64(W_UV)
+    B, q_len, H, qk_nope = qn.shape
+    d_hR = qr.shape[3]
+    d_c = wk.shape[2]
+    v_head = wv.shape[1]
+    offs = _i64(offsets)
+    if units is None:
+        units = [(b, t, h) for b in range(B) for t in range(q_len) for h in range(H)]
+    ub = _i32([u[0] for u in units])
+    ut = _i32([u[1] for u in units])
+    uh = _i32([u[2] for u in units])
+    n = len(ub)
+    o = np.empty((n, v_head))
+    (lib or load()).oracle_decode_multi(int(absorbed), H, q_len, d_c, d_hR, qk_nope, v_head, float(scale),
+                                        _p(offs), _p(qn), _p(qr), _p(rows), _p(wk), _p(wv), n, _p(ub), _p(ut),
+                                        _p(uh), _p(o))
+    if n == B * q_len * H and list(units) == [(b, t, h) for b in range(B) for t in range(q_len)
+                                              for h in range(H)]:
+        return o.reshape(B, q_len, H, v_head)
+    return o
 
 
 def out_proj(o, W_O, lib=None) -> np.ndarray:

@@ -270,6 +270,41 @@ void oracle_decode(int absorbed, int H, int d_c, int d_hR, int qk_nope, int v_he
     }
 }
 
+/* ------------------------------------------------- multi-token decode [L4][L1] */
+
+/* Several new tokens per sequence in one step: the verification of draft tokens in
+ * speculative decoding, which [L4] ("Concepte cheie": the MTP module) names as a use of
+ * multi-token prediction.  The pages give no formula; the reading taken is the causal rule
+ * of attention within the sequence ([L1] "La compresion de MLA": each token attends to the
+ * tokens before it and itself).  Sequence b owns rows [offsets[b], offsets[b+1]); its last
+ * q_len rows are the new tokens.  New token t (0 <= t < q_len) sits at position
+ * L_b - q_len + t and attends to rows 0 .. L_b - q_len + t of its sequence.
+ * Units are (b, t, h).  q_nope: [B, q_len, H, qk_nope]; q_rope: [B, q_len, H, d_hR];
+ * o: [n_units, v_head].  A token with no rows (L_b - q_len + t < 0) gives o = 0. */
+void oracle_decode_multi(int absorbed, int H, int q_len, int d_c, int d_hR, int qk_nope, int v_head,
+                         double scale, const int64_t* offsets, const double* q_nope,
+                         const double* q_rope, const double* rows, const double* W_UK,
+                         const double* W_UV, int n_units, const int32_t* unit_b,
+                         const int32_t* unit_t, const int32_t* unit_h, double* o) {
+    int rw = d_c + d_hR;
+    for (int u = 0; u < n_units; ++u) {
+        int b = unit_b[u], t = unit_t[u], h = unit_h[u];
+        int64_t t0 = offsets[b];
+        int64_t T = offsets[b + 1] - offsets[b] - (q_len - 1 - t);   /* keys up to the token itself */
+        if (T < 0) T = 0;
+        size_t q = ((size_t)b * q_len + t) * H + h;
+        const double* wk = W_UK + (size_t)h * qk_nope * d_c;
+        const double* wv = W_UV + (size_t)h * v_head * d_c;
+        double* ou = o + (size_t)u * v_head;
+        if (absorbed)
+            oracle_attend_absorbed((int)T, d_c, d_hR, qk_nope, v_head, scale, q_nope + q * qk_nope,
+                                   q_rope + q * d_hR, rows + (size_t)t0 * rw, wk, wv, ou, NULL, NULL);
+        else
+            oracle_attend_naive((int)T, d_c, d_hR, qk_nope, v_head, scale, q_nope + q * qk_nope,
+                                q_rope + q * d_hR, rows + (size_t)t0 * rw, wk, wv, ou, NULL, NULL);
+    }
+}
+
 /* ----------------------------------------------------- output projection [L1][L2] */
 
 /* out[i] = W_O concat_h o[i, h, :].  o: [n, H*v_head]; W_O: [d_model, H*v_head]. */

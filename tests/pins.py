@@ -270,7 +270,51 @@ def pin_prefill(lib):
         _close(o, ref, 1e-12, "prefill vs causal sdpa")
 
 
+def pin_decode_multi(lib):
+    """Multi-token decode: token t of the q_len new ones attends to the keys up to itself.
+    Checked against torch attention with an explicit boolean mask, against the causal
+    prefill of the same sequence, and q_len = 1 against the one-token decode."""
+    r = _rs(20)
+    B, q_len, H, d_c, d_hR, qk, v = 3, 3, 2, 16, 8, 8, 12
+    lens = [7, 3, 2]                     # 3 = q_len: the first new token sees one key; 2 < q_len
+    offs = np.concatenate([[0], np.cumsum(lens)])
+    rows = r.standard_normal((offs[-1], d_c + d_hR))
+    qn, qr = r.standard_normal((B, q_len, H, qk)), r.standard_normal((B, q_len, H, d_hR))
+    WUK, WUV = r.standard_normal((H, qk, d_c)) / 4, r.standard_normal((H, v, d_c)) / 4
+    for absorbed in (False, True):
+        o = oracle.decode_multi(qn, qr, rows, offs, WUK, WUV, 0.3, absorbed=absorbed, lib=lib)
+        for b in range(B):
+            L = lens[b]
+            rr = rows[offs[b]:offs[b + 1]]
+            c = rr[:, :d_c]
+            for h in range(H):
+                K = np.concatenate([c @ WUK[h].T, rr[:, d_c:]], 1)
+                V = c @ WUV[h].T
+                for t in range(q_len):
+                    n_keys = L - q_len + t + 1
+                    if n_keys <= 0:
+                        assert np.all(o[b, t, h] == 0), "a token with no keys gives 0"
+                        continue
+                    mask = torch.from_numpy(np.arange(L) < n_keys)[None, None, None]
+                    q = torch.from_numpy(np.concatenate([qn[b, t, h], qr[b, t, h]]))[None, None, None]
+                    ref = torch.nn.functional.scaled_dot_product_attention(
+                        q, torch.from_numpy(K)[None, None], torch.from_numpy(V)[None, None], attn_mask=mask,
+                        scale=0.3)[0, 0, 0].numpy()
+                    _close(o[b, t, h], ref, 1e-12, f"multi b={b} t={t} h={h}")
+    # the new tokens' outputs are the causal prefill's outputs at their positions
+    b, h, L = 0, 1, lens[0]
+    QN, QR = r.standard_normal((L, qk)), r.standard_normal((L, d_hR))
+    QN[L - q_len:], QR[L - q_len:] = qn[b, :, h], qr[b, :, h]
+    pre = oracle.prefill_head(QN, QR, rows[:L], WUK[h], WUV[h], 0.3, list(range(L - q_len, L)), False, lib)
+    o = oracle.decode_multi(qn, qr, rows, offs, WUK, WUV, 0.3, absorbed=True, lib=lib)
+    _close(o[b, :, h], pre, 1e-12, "multi vs causal prefill")
+    # one new token: the one-token decode
+    o1 = oracle.decode_multi(qn[:, :1], qr[:, :1], rows, offs, WUK, WUV, 0.3, lib=lib)
+    d1, _ = oracle.decode(qn[:, 0], qr[:, 0], rows, offs, WUK, WUV, 0.3, lib=lib)
+    _close(o1[:, 0], d1, 1e-13, "q_len = 1")
+
+
 ALL_PINS = [pin_page_figures, pin_round_bf16, pin_rope, pin_latent_rows, pin_query,
             pin_decode_vs_library_attention, pin_decode_textbook_reduction, pin_decode_score_split,
             pin_decode_special_cases, pin_naive_equals_absorbed, pin_decode_batch_driver,
-            pin_out_proj, pin_prefill]
+            pin_out_proj, pin_prefill, pin_decode_multi]

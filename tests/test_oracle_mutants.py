@@ -26,6 +26,9 @@ MUTANTS = {
                              "oracle_rope(d_hR, kr, (double)(pos[i] + 1), theta, row + d_c);"),
     "bf16_truncates": ("double r = rint(ldexp(m, 8));", "double r = floor(ldexp(m, 8));"),
     "causal_excludes_self": ("oracle_attend_naive(t + 1, d_c", "oracle_attend_naive(t, d_c"),
+    "multi_window_off_by_one": ("- (q_len - 1 - t);   /* keys up to the token itself */",
+                                "- (q_len - t);   /* keys up to the token itself */"),
+    "multi_query_index": ("size_t q = ((size_t)b * q_len + t) * H + h;", "size_t q = ((size_t)t * q_len + b) * H + h;"),
     "mla_row_without_rope": ("return (d_c + d_hR) * layers;", "return d_c * layers;"),
     "out_proj_transposed": ("acc += W_O[(size_t)j * Hv + k] * o[(size_t)i * Hv + k];",
                             "acc += W_O[(size_t)(k % d_model) * Hv + j % Hv] * o[(size_t)i * Hv + k];"),
