@@ -56,6 +56,9 @@ SIGNATURES = {
                                          _P]),
     "mla_decode_absorbed_paged": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, ctypes.c_int32,
                                        _P, _P, ctypes.c_size_t, _P]),
+    "mla_decode_absorbed_paged_multi": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P,
+                                             ctypes.c_int32, ctypes.c_int32, _P, _P, ctypes.c_size_t, _P]),
+    "mla_decode_multi_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "mla_decode_absorbed_host": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
                                       ctypes.c_size_t, _P]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
@@ -193,6 +196,24 @@ def mla_decode_absorbed_paged(dims, weights: MLAWeights, cache_pages, block_tabl
                                           _ptr(cache_pages), cache_pages.shape[0], _ptr(block_table), max_blocks,
                                           _ptr(seq_lens), B, _ptr(out), _ptr(ws), ws.numel(), _stream(stream)),
            "mla_decode_absorbed_paged")
+
+
+def mla_decode_multi_workspace_size(dims, B: int, q_len: int, max_blocks: int) -> int:
+    return _lib.mla_decode_multi_workspace_size(ctypes.byref(dims), B, q_len, max_blocks)
+
+
+def mla_decode_absorbed_paged_multi(dims, weights: MLAWeights, cache_pages, block_table, seq_lens, out, ws,
+                                    q_nope, q_rope, stream=None) -> None:
+    """Multi-token decode over a paged cache: q_nope [B, q_len, H, qk_nope], q_rope
+    [B, q_len, H, d_hR], out [B, q_len, H, v_head]; the q_len new tokens are the last
+    q_len of each sequence's seq_lens[b] tokens (already appended to the pages)."""
+    B, max_blocks = block_table.shape
+    q_len = q_nope.shape[1]
+    _check(_lib.mla_decode_absorbed_paged_multi(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
+                                                _ptr(cache_pages), cache_pages.shape[0], _ptr(block_table),
+                                                max_blocks, _ptr(seq_lens), B, q_len, _ptr(out), _ptr(ws),
+                                                ws.numel(), _stream(stream)),
+           "mla_decode_absorbed_paged_multi")
 
 
 def mla_decode_absorbed_host(dims, weights: MLAWeights, cache, offsets, q_nope_host, q_rope_host, out_host, ws,

@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "decode_tc.cuh"
 #include "gemm_tc.cuh"
+#include "multi.cuh"
 #include "prefill_tc.cuh"
 #include "mla.h"
 
@@ -523,6 +524,74 @@ extern "C" mla_status mla_decode_absorbed_paged(const mla_dims* d, mla_weights w
         (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, (const bf16*)cache, rows, nullptr, seq_lens,
         block_table, max_blocks, B, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged");
+}
+
+// ---------------------------------------------------------- multi-token decode
+
+// The decode workspace for B * q_len sequences, then the per-token block table and lengths.
+struct MultiWs {
+    DecodeWs dec;
+    int32_t* vbt;    // [B * q_len, max_blocks]
+    int32_t* vlen;   // [B * q_len]
+    size_t bytes;
+};
+
+static MultiWs carve_multi(const mla_dims* d, int B, int q_len, int max_blocks, void* base) {
+    MultiWs m{};
+    m.dec = carve_decode(d, B * q_len, base, true);
+    const size_t head = (m.dec.bytes + 255) & ~(size_t)255;
+    Carve c(base ? (char*)base + head : nullptr);
+    m.vbt = (int32_t*)c.take((size_t)B * q_len * max_blocks * sizeof(int32_t));
+    m.vlen = (int32_t*)c.take((size_t)B * q_len * sizeof(int32_t));
+    m.bytes = head + c.used;
+    return m;
+}
+
+static bool multi_sizes_ok(int32_t B, int32_t q_len, int32_t max_blocks) {
+    return B >= 0 && q_len >= 1 && max_blocks >= 1 && (long long)B * q_len <= 0x7FFFFFFFLL &&
+           (long long)B * q_len * max_blocks <= 0x7FFFFFFFLL;
+}
+
+extern "C" size_t mla_decode_multi_workspace_size(const mla_dims* d, int32_t B, int32_t q_len,
+                                                  int32_t max_blocks) {
+    if (dims_supported(d) != MLA_OK || !tc_decode_ok(d) || !multi_sizes_ok(B, q_len, max_blocks)) return 0;
+    return carve_multi(d, B, q_len, max_blocks, nullptr).bytes;
+}
+
+extern "C" mla_status mla_decode_absorbed_paged_multi(const mla_dims* d, mla_weights w, const void* q_nope,
+                                                      const void* q_rope, const void* cache, int64_t num_pages,
+                                                      const int32_t* block_table, int32_t max_blocks,
+                                                      const int32_t* seq_lens, int32_t B, int32_t q_len,
+                                                      void* out, void* workspace, size_t ws_bytes,
+                                                      mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0 || q_len < 1) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if (!tc_decode_ok(d) || w->W_O) return MLA_ERR_UNSUPPORTED;
+    if (B == 0) return MLA_OK;
+    if (!q_nope || !q_rope || !cache || !block_table || !seq_lens || !out || max_blocks <= 0 || num_pages <= 0)
+        return MLA_ERR_INVALID_ARG;
+    if (!multi_sizes_ok(B, q_len, max_blocks)) return MLA_ERR_UNSUPPORTED;
+    const long long rows = (long long)num_pages * mla::tc::kPageTokens;
+    if (rows > 0x7FFFFFFFLL) return MLA_ERR_UNSUPPORTED;
+    MultiWs ws = carve_multi(d, B, q_len, max_blocks, workspace);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    cudaError_t e;
+    {
+        mla::ProfScope ps(s, "multi_token_views");
+        e = mla::expand_multi_token(block_table, seq_lens, B, q_len, max_blocks, ws.vbt, ws.vlen, s);
+    }
+    if (e != cudaSuccess) return cuda_fail(e, "mla_decode_absorbed_paged_multi");
+    const long long H = d->H;
+    e = mla::tc::decode_absorbed_tc((const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope,
+                                    H * d->d_hR, d->d_hR, (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
+                                    (const bf16*)cache, rows, nullptr, ws.vlen, ws.vbt, max_blocks, B * q_len,
+                                    scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code, err.detail, s);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged_multi");
 }
 
 // ----------------------------------------------------------------------- prefill

@@ -171,6 +171,36 @@ mla_status mla_decode_absorbed_paged(const mla_dims* dims, mla_weights w, const 
                                      const int32_t* seq_lens, int32_t B, void* out, void* workspace,
                                      size_t ws_bytes, mla_stream_t stream);
 
+/* Multi-token decode over a PAGED latent cache: q_len >= 1 new tokens per sequence in one
+ * call (the verification of draft tokens in speculative decoding; the DeepSeek pages name
+ * the multi-token-prediction module's use for it ["Multi-head Latent Attention (MLA) si
+ * arhitectura DeepSeekMoE", "Concepte cheie"]).  The new tokens' cache rows must already be
+ * appended: sequence b holds seq_lens[b] tokens (int32 [B], device), the last q_len of them
+ * the new ones, in the pages of block_table (int32 [B, max_blocks], device), laid out as for
+ * mla_decode_absorbed_paged.  New token t (0 <= t < q_len) of sequence b sits at position
+ * seq_lens[b] - q_len + t and attends to the sequence's first seq_lens[b] - q_len + t + 1
+ * tokens: causal inside the window, the rule of causal attention ["02 - Multi-Latent
+ * Attention (MLA)", "La compresion de MLA"].
+ *   q_nope [B, q_len, H, qk_nope], q_rope [B, q_len, H, d_hR] (rotated at the tokens'
+ *   positions), out [B, q_len, H, v_head]: device, storage type, contiguous.
+ * The result for token (b, t) is that of mla_decode_absorbed_paged on a sequence of
+ * seq_lens[b] - q_len + t + 1 tokens; a token with no key (seq_lens[b] < q_len - t) gets
+ * zeros.  Tensor-core shape only and handles without W_O, else MLA_ERR_UNSUPPORTED; a page
+ * outside [0, num_pages) or more than max_blocks blocks latch MLA_ERR_OUT_OF_RANGE on the
+ * device.  Each new token streams its own keys: the cache bytes read are q_len times those
+ * of one decode step.
+ * Workspace: device, >= mla_decode_multi_workspace_size(dims, B, q_len, max_blocks) bytes,
+ * 256-byte aligned, contents on entry do not matter. */
+mla_status mla_decode_absorbed_paged_multi(const mla_dims* dims, mla_weights w, const void* q_nope,
+                                           const void* q_rope, const void* cache, int64_t num_pages,
+                                           const int32_t* block_table, int32_t max_blocks,
+                                           const int32_t* seq_lens, int32_t B, int32_t q_len, void* out,
+                                           void* workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* Workspace bytes of mla_decode_absorbed_paged_multi; 0 for shapes it does not support or
+ * sizes out of range (q_len < 1, max_blocks < 1, B * q_len * max_blocks >= 2^31). */
+size_t mla_decode_multi_workspace_size(const mla_dims* dims, int32_t B, int32_t q_len, int32_t max_blocks);
+
 /* mla_decode_absorbed with the queries and the output in HOST memory: the call copies
  * q_nope [B,H,qk_nope] and q_rope [B,H,d_hR] (storage type, rotated) host->device into the
  * workspace, runs the same decode on the stream, and copies o [B,H,v_head] device->host.

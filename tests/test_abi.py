@@ -64,6 +64,15 @@ def test_workspace_sizes_are_positive_and_monotone():
     a, b = mla.mla_decode_workspace_size(d, 8), mla.mla_decode_workspace_size(d, 64)
     assert 0 < a < b
     assert mla.mla_decode_workspace_size(v3(H=0), 8) == 0
+    # multi-token decode: the decode workspace of B * q_len sequences plus the per-token
+    # block table; invalid sizes give 0
+    m1, m4 = mla.mla_decode_multi_workspace_size(d, 8, 1, 64), mla.mla_decode_multi_workspace_size(d, 8, 4, 64)
+    assert mla.mla_decode_workspace_size(d, 8) < m1 < m4
+    assert m4 >= mla.mla_decode_workspace_size(d, 32) + 32 * 64 * 4
+    assert mla.mla_decode_multi_workspace_size(d, 8, 0, 64) == 0
+    assert mla.mla_decode_multi_workspace_size(d, 8, 2, 0) == 0
+    assert mla.mla_decode_multi_workspace_size(d, 1 << 20, 1 << 12, 64) == 0
+    assert mla.mla_decode_multi_workspace_size(v3(H=64), 8, 2, 64) == 0   # tensor-core shape only
     p = mla.mla_prefill_workspace_size(v3(d_model=5120), 4, 4096)
     # q (192) + K_nope (128) + V (128) per token and head, bf16
     assert p >= 4 * 4096 * 128 * (192 + 128 + 128) * 2
@@ -91,4 +100,9 @@ def test_argument_errors_return_before_any_launch():
                                          0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_absorbed_host(ctypes.byref(d), None, None, None, None, 1, None, 1, None, None, 0,
                                         None) == mla.MLA_ERR_INVALID_ARG
+    multi = lambda B, q_len: lib.mla_decode_absorbed_paged_multi(ctypes.byref(d), None, None, None, None, 1, None,
+                                                                 1, None, B, q_len, None, None, 0, None)
+    assert multi(1, 2) == mla.MLA_ERR_INVALID_ARG      # no weights handle
+    assert multi(1, 0) == mla.MLA_ERR_INVALID_ARG      # q_len < 1
+    assert multi(-1, 2) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_weights_destroy(None) == mla.MLA_OK

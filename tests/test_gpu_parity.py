@@ -483,6 +483,51 @@ def test_paged_cache_gives_the_contiguous_result():
     assert torch.equal(out.cpu(), dev)
 
 
+# ------------------------------------------------------------ multi-token decode
+
+def test_multi_token_decode_over_pages_matches_the_oracle():
+    """q_len = 3 new tokens per sequence over a paged cache (random page order, spare
+    pages): token t of sequence b attends to the keys up to its own position.  Sequences of
+    3 and 2 tokens give new tokens with 1, 2, 3 and 0, 1, 2 keys (no key: zeros)."""
+    q_len = 3
+    lengths = [300, 3, 2, 513, 64, 130]
+    w, inp = reduced_attn_inputs(lengths, seed=53)
+    r = np.random.default_rng(53)
+    qn = torch.from_numpy(r.standard_normal((w.B, q_len, w.H, w.qk_nope))).to(torch.bfloat16)
+    qr = torch.from_numpy(r.standard_normal((w.B, q_len, w.H, w.d_hR))).to(torch.bfloat16)
+    npg = [(L + 63) // 64 for L in lengths]
+    total_pages = sum(npg) + 3
+    perm = r.permutation(total_pages)
+    pages = torch.zeros(total_pages, 64, w.row, dtype=torch.bfloat16)
+    max_blocks = max(npg) + 1
+    table = np.zeros((w.B, max_blocks), dtype=np.int32)
+    offs = inp["offsets"].numpy()
+    k = 0
+    for b, L in enumerate(lengths):
+        for j in range(npg[b]):
+            p = int(perm[k])
+            k += 1
+            table[b, j] = p
+            n = min(64, L - 64 * j)
+            pages[p, :n] = inp["cache"][offs[b] + 64 * j: offs[b] + 64 * j + n]
+    dims = dims_of(w)
+    g = to_dev({k_: inp[k_] for k_ in ("W_UK", "W_UV")})
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    ws = mla.workspace(mla.mla_decode_multi_workspace_size(dims, w.B, q_len, max_blocks))
+    out = torch.empty(w.B, q_len, w.H, w.v_head, dtype=torch.bfloat16, device=DEV)
+    mla.mla_decode_absorbed_paged_multi(dims, weights, pages.to(DEV), torch.from_numpy(table).to(DEV),
+                                        torch.tensor(lengths, dtype=torch.int32, device=DEV), out, ws,
+                                        q_nope=qn.to(DEV), q_rope=qr.to(DEV))
+    assert mla.mla_get_device_error() == (0, 0)
+    out = out.cpu()
+    assert torch.all(out[2, 0] == 0), "a new token with no key decodes to zeros"
+    units = [(b, t, h) for b in range(w.B) for t in range(q_len) for h in (0, 45, 127)
+             if lengths[b] - q_len + t + 1 > 0]
+    want = oracle.decode_multi(qn, qr, inp["cache"], inp["offsets"], inp["W_UK"], inp["W_UV"], w.scale,
+                               units=units, absorbed=True)
+    assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", "multi-token decode")
+
+
 def test_decode_large_batch_spans_several_sequence_blocks():
     """B = 200 short ragged sequences: the q-absorb kernel runs two blocks of 128 sequences
     and the merge kernel four blocks of 64; sampled units against the oracle."""
