@@ -55,6 +55,46 @@ def alg_step(w: workloads.Workload) -> dict:
             "attn_flops": flops_attn, "tokens": tokens}
 
 
+def alg_multi(w: workloads.Workload) -> dict:
+    """Bytes and flops of one multi-token decode step: each sequence's L + q_len rows read
+    once, new token t attending to the first L + t + 1 of them."""
+    L = workloads.lengths(w)
+    rows = int((L + w.q_len).sum())
+    e = 2
+    cache = rows * w.row * e
+    weights = 2 * w.H * w.qk_nope * w.d_c * e
+    n = w.B * w.q_len
+    q = n * w.H * (w.qk_nope + w.d_hR) * e
+    out = n * w.H * w.v_head * e
+    attended = int(sum(int(l) + t + 1 for l in L for t in range(w.q_len)))
+    flops_attn = attended * w.H * (2 * w.row + 2 * w.d_c)
+    flops_proj = 2 * n * w.H * w.qk_nope * w.d_c * 2
+    return {"bytes": cache + weights + q + out, "cache_bytes": cache, "flops": flops_attn + flops_proj,
+            "attn_flops": flops_attn, "tokens": rows}
+
+
+def paged_layout(w, inp, seed):
+    """The contiguous rows of `inp` laid out in 64-token pages of a shuffled page pool:
+    (pages [n_pages, 64, row], block_table int32 [B, max_blocks], seq_lens int32 [B])."""
+    offs = inp["offsets"].numpy().astype(np.int64)
+    L = offs[1:] - offs[:-1]
+    npg = (L + 63) // 64
+    max_blocks = max(int(npg.max()), 1)
+    total = int(npg.sum())
+    perm = np.random.default_rng(seed).permutation(total)
+    pages = torch.zeros(total, 64, w.row, dtype=inp["cache"].dtype)
+    table = np.zeros((w.B, max_blocks), dtype=np.int32)
+    k = 0
+    for b in range(w.B):
+        for j in range(int(npg[b])):
+            p = int(perm[k])
+            k += 1
+            table[b, j] = p
+            n = int(min(64, L[b] - 64 * j))
+            pages[p, :n] = inp["cache"][offs[b] + 64 * j: offs[b] + 64 * j + n]
+    return pages, torch.from_numpy(table), torch.from_numpy(L.astype(np.int32))
+
+
 def alg_layer(w: workloads.Workload) -> dict:
     """Bytes and flops of one full decode-layer step: append the new token, project the
     query, absorbed attention over L + 1 rows, W_UV, W_O."""
@@ -268,7 +308,8 @@ def run_reference(args, w):
 def config_of(w, world):
     return {"workload": w.name, "B_per_gpu": w.B, "ctx": w.ctx, "H": w.H, "d_c": w.d_c, "d_hR": w.d_hR,
             "qk_nope": w.qk_nope, "v_head": w.v_head, "global_batch": w.B * world,
-            "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write, outside the step events)"}
+            "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write, outside the step events)",
+            **({"q_len": w.q_len} if w.kind == "decode_multi" else {})}
 
 
 def build_step(w, inp, dev, mla):
@@ -286,6 +327,19 @@ def build_step(w, inp, dev, mla):
                                     q_rope=g["q_rope"])
         h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
         return g, dims, weights, out, step, h2d, alg_step(w), w.B
+    if w.kind == "decode_multi":
+        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+        out = torch.empty(w.B, w.q_len, w.H, w.v_head, dtype=dt, device=dev)
+        pages, table, lens = paged_layout(w, inp, w.seed)
+        pages, table, lens = pages.to(dev), table.to(dev), lens.to(dev)
+        del g["cache"]   # the pages hold the rows
+        ws = mla.workspace(mla.mla_decode_multi_workspace_size(dims, w.B, w.q_len, table.shape[1]), dev)
+
+        def step():
+            mla.mla_decode_absorbed_paged_multi(dims, weights, pages, table, lens, out, ws, q_nope=g["q_nope"],
+                                                q_rope=g["q_rope"])
+        h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
+        return g, dims, weights, out, step, h2d, alg_multi(w), w.B * w.q_len
     if w.kind == "decode_layer":
         weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"])
         out = torch.empty(w.B, w.d_model, dtype=dt, device=dev)
@@ -439,8 +493,9 @@ def run_ours(args, w0):
                         "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak,
                         "traffic": None, "dominant_kernel": dom, "dominant_launch_us": launch_s * 1e6,
                         "peak_source": f"{pk_kind} " + ("bf16_tflops" if bound == "tensor" else "hbm_gbs")}
-            metric = ("MLA decode-layer tokens/s (append + q proj + absorbed attention + W_UV + W_O)"
-                      if w.kind == "decode_layer" else "MLA causal prefill tokens/s (K/V materialised)")
+            metric = {"decode_layer": "MLA decode-layer tokens/s (append + q proj + absorbed attention + W_UV + W_O)",
+                      "decode_multi": "MLA multi-token decode tokens/s (q_len new tokens per sequence, paged cache)",
+                      "prefill": "MLA causal prefill tokens/s (K/V materialised)"}[w.kind]
             unit = "tokens/s"
         line = {
             "metric": metric, "value": world * units / step_s, "unit": unit, "n_gpus": world,

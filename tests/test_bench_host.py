@@ -3,6 +3,8 @@ by, and the guard that drops a stale DRAM-traffic figure."""
 import json
 import os
 
+import torch
+
 import bench
 import workloads
 
@@ -30,6 +32,31 @@ def test_layer_and_prefill_steps_count_their_weights():
     pre = bench.alg_prefill(workloads.WORKLOADS["v2_prefill_b4_s4096"])
     assert pre["tokens"] == 4 * 4096
     assert 7.0e12 < pre["flops"] < 8.0e12
+
+
+def test_multi_token_step_counts_the_window():
+    w = workloads.WORKLOADS["v3_mtp_b32_ctx4096_q2"]
+    a = bench.alg_multi(w)
+    rows = 32 * (4096 + 2)
+    assert a["tokens"] == rows and a["cache_bytes"] == rows * 1152
+    # new token t attends to 4096 + t + 1 rows
+    assert a["attn_flops"] == 32 * (4097 + 4098) * 128 * (2 * 576 + 2 * 512)
+    inp = workloads.make_inputs(workloads.shrink(w, B=3, ctx=100, q_len=3))
+    assert tuple(inp["q_nope"].shape) == (3, 3, 128, 128) and tuple(inp["q_rope"].shape) == (3, 3, 128, 64)
+    assert inp["offsets"].tolist() == [0, 103, 206, 309]
+
+
+def test_paged_layout_keeps_every_row():
+    w = workloads.shrink(workloads.WORKLOADS["v3_mtp_b32_ctx4096_q2"], B=3, ctx=100, q_len=2)
+    inp = workloads.make_inputs(w)
+    pages, table, lens = bench.paged_layout(w, inp, 5)
+    assert lens.tolist() == [102, 102, 102] and tuple(table.shape) == (3, 2)
+    assert sorted(table.flatten().tolist()) == list(range(6))
+    offs = inp["offsets"].tolist()
+    for b in range(3):
+        for t in (0, 63, 64, 101):
+            assert bytes(pages[table[b, t // 64], t % 64].view(-1).view(torch.int16).numpy()) == \
+                bytes(inp["cache"][offs[b] + t].view(torch.int16).numpy())
 
 
 def test_traffic_figure_is_dropped_when_the_kernel_source_changed(tmp_path, monkeypatch):

@@ -1,4 +1,4 @@
-"""The five synthetic MLA workloads, with their shapes, seeds and input recipes.
+"""The six synthetic MLA workloads, with their shapes, seeds and input recipes.
 
 Shapes follow DeepSeek-V2/V3 layers: latent width d_c = 512 (kv_lora_rank), decoupled
 RoPE key width d_hR = 64 (qk_rope_head_dim), 128 heads of 128 content dims.  No
@@ -27,7 +27,7 @@ TENSOR_IDS = {
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "decode_layer" | "decode_attn" | "prefill"
+    kind: str                 # "decode_layer" | "decode_attn" | "decode_multi" | "prefill"
     B: int
     H: int
     d_model: int              # 0 when the workload starts from given queries
@@ -42,6 +42,7 @@ class Workload:
     history: str = ""         # decode_layer: "hidden" (cache built by appending) | "synthetic"
     rope_theta: float = 10000.0
     cache_std: float = 0.5    # synthetic cache rows ~ cache_std * N(0, 1)
+    q_len: int = 1            # decode_multi: new tokens per sequence (appended after the ctx rows)
 
     @property
     def row(self) -> int:
@@ -78,11 +79,16 @@ WORKLOADS: Dict[str, Workload] = {
     "v2_prefill_b4_s4096": Workload("v2_prefill_b4_s4096", "prefill", B=4, H=128, d_model=5120,
                                     d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
                                     seed=_seed(5), ctx=4096),
+    # multi-token decode (speculative verification): 2 new tokens per sequence over 4096
+    # cached tokens, paged cache
+    "v3_mtp_b32_ctx4096_q2": Workload("v3_mtp_b32_ctx4096_q2", "decode_multi", B=32, H=128, d_model=0,
+                                      d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
+                                      seed=_seed(6), ctx=4096, q_len=2),
 }
 
 # the order the workloads are listed in (smallest first)
-ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_ragged_b64", "v3_layer_b128_ctx8192",
-         "v2_prefill_b4_s4096"]
+ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_mtp_b32_ctx4096_q2", "v3_ragged_b64",
+         "v3_layer_b128_ctx8192", "v2_prefill_b4_s4096"]
 
 
 def shrink(w: Workload, **over) -> Workload:
@@ -134,6 +140,9 @@ def make_inputs(w: Workload) -> Dict[str, torch.Tensor]:
 
     decode_attn : cache [sum L, row], offsets int32 [B+1], q_nope [B,H,qk_nope],
                   q_rope [B,H,d_hR] (already rotated), W_UK, W_UV.
+    decode_multi: cache [sum (L + q_len), row] (the new tokens' rows last in each sequence),
+                  offsets int32 [B+1], q_nope [B,q_len,H,qk_nope], q_rope [B,q_len,H,d_hR],
+                  W_UK, W_UV.
     decode_layer: weights, h_new [B, d_model] (the token being decoded, at position L),
                   offsets int32 [B+1] over a cache of capacity L+1 per sequence, and either
                   h_hist [B, L, d_model] (cache built by appending at positions 0..L-1) or
@@ -148,6 +157,12 @@ def make_inputs(w: Workload) -> Dict[str, torch.Tensor]:
         d["cache"] = _tensor(w, "cache", (int(offs[-1]), w.row), w.cache_std)
         d["q_nope"] = _tensor(w, "q_nope", (w.B, w.H, w.qk_nope), 1.0)
         d["q_rope"] = _tensor(w, "q_rope", (w.B, w.H, w.d_hR), 1.0)
+    elif w.kind == "decode_multi":
+        offs = np.concatenate([[0], np.cumsum(L + w.q_len)]).astype(np.int32)
+        d["offsets"] = torch.from_numpy(offs)
+        d["cache"] = _tensor(w, "cache", (int(offs[-1]), w.row), w.cache_std)
+        d["q_nope"] = _tensor(w, "q_nope", (w.B, w.q_len, w.H, w.qk_nope), 1.0)
+        d["q_rope"] = _tensor(w, "q_rope", (w.B, w.q_len, w.H, w.d_hR), 1.0)
     elif w.kind == "decode_layer":
         cap = L + 1
         offs = np.concatenate([[0], np.cumsum(cap)]).astype(np.int32)
