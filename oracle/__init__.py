@@ -44,6 +44,9 @@ def _declare(lib):
     lib.oracle_round_bf16.restype = ctypes.c_uint16
     lib.oracle_round_bf16.argtypes = [_D]
     lib.oracle_round_bf16_array.argtypes = [_I64, _P, _P]
+    lib.oracle_round_e4m3.restype = _D
+    lib.oracle_round_e4m3.argtypes = [_D]
+    lib.oracle_quantize_latent_fp8.argtypes = [_I32, _I32, _I32, _P, _P, _P]
     lib.oracle_rope.argtypes = [_I32, _P, _D, _D, _P]
     lib.oracle_latent_rows.argtypes = [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _D, _P]
     lib.oracle_query.argtypes = [_I32, _I32, _I32, _I32, _I32, _P, _P, _P, _D, _P, _P]
@@ -109,6 +112,23 @@ def bf16_value(bits: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------- RoPE
+
+def round_e4m3(x, lib=None) -> np.ndarray:
+    """Nearest FP8 E4M3 value (ties to even, saturating at 448) of each element, as float64."""
+    x = f64(x)
+    fn = (lib or load()).oracle_round_e4m3
+    return np.array([fn(float(v)) for v in x.reshape(-1)]).reshape(x.shape)
+
+
+def quantize_latent_fp8(rows, d_c: int, lib=None) -> Tuple[np.ndarray, np.ndarray]:
+    """Per-token FP8 E4M3 latent: (dequantised rows [n, d_c + d_hR], scales [n])."""
+    rows = f64(rows)
+    n, rw = rows.shape
+    deq = np.empty_like(rows)
+    scales = np.empty(n)
+    (lib or load()).oracle_quantize_latent_fp8(n, d_c, rw - d_c, _p(rows), _p(deq), _p(scales))
+    return deq, scales
+
 
 def rope(x, pos: float, theta: float = 10000.0, lib=None) -> np.ndarray:
     a = f64(x)

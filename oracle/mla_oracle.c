@@ -71,6 +71,45 @@ void oracle_round_bf16_array(int64_t n, const double* x, uint16_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_round_bf16(x[i]);
 }
 
+/* float64 -> the value of the nearest FP8 E4M3 number (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, no infinities, largest finite 448, subnormals down to 2^-9), ties to even.
+ * Magnitudes above 448 saturate to 448 (the per-token scale below never produces them). */
+double oracle_round_e4m3(double x) {
+    double a = fabs(x);
+    if (isnan(x)) return x;
+    if (a == 0.0) return x;
+    int e;
+    frexp(a, &e);                          /* a = m * 2^e, m in [0.5, 1): exponent e - 1 */
+    int ue = e - 1 < -6 ? -6 : e - 1;      /* below 2^-6 the quantum stays 2^-9 */
+    double q = ldexp(1.0, ue - 3);         /* 3 mantissa bits */
+    double r = rint(a / q) * q;            /* rint: ties to even in the default mode */
+    if (r > 448.0) r = 448.0;
+    return signbit(x) ? -r : r;
+}
+
+/* -------------------------------------------------- FP8 latent cache [L1][L4] */
+
+/* A quantised latent cache, which [L1] ("Lo que esta fase NO cubre": quantised KV cache as
+ * another compression) and [L4] ("Exemplul 1": the engine's real cache format, e.g. FP8)
+ * name without a format.  Reading: each token's latent c (d_c values) is stored as FP8 E4M3
+ * codes with one scale per token, s = max_i |c_i| / 448 (s = 1 for an all-zero c), code_i =
+ * e4m3(c_i / s); the decoupled RoPE key stays as it is.  The attention then runs on the
+ * dequantised row [code * s | k_r].  rows, deq: [n, d_c + d_hR]; scales: [n]. */
+void oracle_quantize_latent_fp8(int n, int d_c, int d_hR, const double* rows, double* deq,
+                                double* scales) {
+    int rw = d_c + d_hR;
+    for (int t = 0; t < n; ++t) {
+        const double* r = rows + (size_t)t * rw;
+        double* o = deq + (size_t)t * rw;
+        double amax = 0.0;
+        for (int i = 0; i < d_c; ++i) amax = fmax(amax, fabs(r[i]));
+        double sc = amax > 0.0 ? amax / 448.0 : 1.0;
+        for (int i = 0; i < d_c; ++i) o[i] = oracle_round_e4m3(r[i] / sc) * sc;
+        for (int i = 0; i < d_hR; ++i) o[d_c + i] = r[d_c + i];
+        scales[t] = sc;
+    }
+}
+
 /* ------------------------------------------------------------------- RoPE [L1][L2] */
 
 /* out = x rotated: for i < d/2, angle = pos * theta^(-2i/d),

@@ -270,6 +270,51 @@ def pin_prefill(lib):
         _close(o, ref, 1e-12, "prefill vs causal sdpa")
 
 
+def pin_e4m3(lib):
+    """FP8 E4M3 rounding against the format's definition and torch's float8_e4m3fn cast."""
+    table = [(1.0625, 1.0), (1.1875, 1.25), (2.0 ** -10, 0.0), (3 * 2.0 ** -10, 2.0 ** -8),
+             (5 * 2.0 ** -11, 2.0 ** -9), (448.0, 448.0), (464.0, 448.0), (1e6, 448.0), (-0.1, -0.1015625),
+             (0.0, 0.0), (240.0, 240.0), (17.0, 16.0), (19.0, 20.0), (2.0 ** -6 * 1.0625, 2.0 ** -6)]
+    for x, want in table:
+        assert oracle.round_e4m3(np.array([x]), lib)[0] == want, (x, want)
+    r = _rs(21)
+    # float32-representable inputs (torch's cast may pass through float32) over the whole range
+    x = (r.standard_normal(20000) * np.exp2(r.uniform(-12, 8.7, 20000))).astype(np.float32)
+    x = np.clip(x, -448, 448).astype(np.float64)
+    got = oracle.round_e4m3(x, lib)
+    ref = torch.from_numpy(x).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(got, ref), f"{int((got != ref).sum())} values differ from torch's e4m3 cast"
+    big = np.abs(x) >= 2.0 ** -6
+    assert np.all(np.abs(got - x)[big] <= 2.0 ** -4 * np.abs(x[big]))       # half an ulp, 3-bit mantissa
+    assert np.all(np.abs(got - x)[~big] <= 2.0 ** -10)                        # half the subnormal quantum
+    assert np.array_equal(oracle.round_e4m3(got, lib), got)                    # representable values stay
+
+
+def pin_fp8_latent(lib):
+    """Per-token FP8 latent: the largest |c| of a token is code 448 and comes back exactly;
+    every value within the format's error; the rotary key untouched; a zero token stays zero."""
+    r = _rs(22)
+    d_c, d_hR = 64, 8
+    rows = r.standard_normal((9, d_c + d_hR)) * np.exp2(r.uniform(-8, 8, (9, 1)))
+    rows[4, :d_c] = 0.0
+    deq, sc = oracle.quantize_latent_fp8(rows, d_c, lib)
+    for t in range(9):
+        c, q = rows[t, :d_c], deq[t, :d_c]
+        assert np.array_equal(deq[t, d_c:], rows[t, d_c:]), "k_r is not quantised"
+        if t == 4:
+            assert sc[t] == 1.0 and np.all(q == 0)
+            continue
+        amax = np.max(np.abs(c))
+        assert abs(sc[t] - amax / 448) <= 1e-15 * sc[t]
+        codes = q / sc[t]
+        assert abs(np.max(np.abs(codes)) - 448.0) <= 1e-12, "the largest element is code 448"
+        _close(oracle.round_e4m3(codes, lib), codes, 1e-12, "codes are e4m3 values")
+        assert np.all(np.abs(q - c) <= 2.0 ** -4 * np.abs(c) + 2.0 ** -10 * sc[t] * (1 + 1e-12))
+    # scaling a token by a power of two scales its codes' scale and nothing else
+    deq2, sc2 = oracle.quantize_latent_fp8(rows * 8.0, d_c, lib)
+    assert np.array_equal(deq2[:, :d_c], deq[:, :d_c] * 8.0) and np.array_equal(sc2[[0, 1, 2, 3, 5]], sc[[0, 1, 2, 3, 5]] * 8)
+
+
 def pin_decode_multi(lib):
     """Multi-token decode: token t of the q_len new ones attends to the keys up to itself.
     Checked against torch attention with an explicit boolean mask, against the causal
@@ -317,4 +362,4 @@ def pin_decode_multi(lib):
 ALL_PINS = [pin_page_figures, pin_round_bf16, pin_rope, pin_latent_rows, pin_query,
             pin_decode_vs_library_attention, pin_decode_textbook_reduction, pin_decode_score_split,
             pin_decode_special_cases, pin_naive_equals_absorbed, pin_decode_batch_driver,
-            pin_out_proj, pin_prefill, pin_decode_multi]
+            pin_out_proj, pin_prefill, pin_decode_multi, pin_e4m3, pin_fp8_latent]

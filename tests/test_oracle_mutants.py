@@ -29,6 +29,10 @@ MUTANTS = {
     "multi_window_off_by_one": ("- (q_len - 1 - t);   /* keys up to the token itself */",
                                 "- (q_len - t);   /* keys up to the token itself */"),
     "multi_query_index": ("size_t q = ((size_t)b * q_len + t) * H + h;", "size_t q = ((size_t)t * q_len + b) * H + h;"),
+    "e4m3_truncates": ("double r = rint(a / q) * q;", "double r = floor(a / q) * q;"),
+    "e4m3_two_mantissa_bits": ("double q = ldexp(1.0, ue - 3);", "double q = ldexp(1.0, ue - 2);"),
+    "e4m3_subnormal_quantum": ("int ue = e - 1 < -6 ? -6 : e - 1;", "int ue = e - 1 < -7 ? -7 : e - 1;"),
+    "fp8_scale_to_240": ("double sc = amax > 0.0 ? amax / 448.0 : 1.0;", "double sc = amax > 0.0 ? amax / 240.0 : 1.0;"),
     "mla_row_without_rope": ("return (d_c + d_hR) * layers;", "return d_c * layers;"),
     "out_proj_transposed": ("acc += W_O[(size_t)j * Hv + k] * o[(size_t)i * Hv + k];",
                             "acc += W_O[(size_t)(k % d_model) * Hv + j % Hv] * o[(size_t)i * Hv + k];"),
