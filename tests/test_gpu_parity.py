@@ -301,12 +301,14 @@ def oracle_prefill(w, inp, b, t_list, heads, absorbed=True):
     return res, rows
 
 
-@pytest.mark.parametrize("B,S", [(2, 200)])
+@pytest.mark.parametrize("B,S", [(2, 200), (2, 1), (1, 128), (3, 257)])
 def test_prefill_reduced(B, S):
+    """Several query blocks with a ragged last one; one token (one query, one key); exactly
+    one block; one query alone in the last block."""
     w = workloads.shrink(workloads.WORKLOADS["v2_prefill_b4_s4096"], B=B, ctx=S, seed=77)
     inp = workloads.make_inputs(w)
     out, cache = run_prefill(w, inp)
-    t_list = [0, 1, 63, 64, 65, 127, 128, 150, 191, 192, 199]
+    t_list = sorted({t for t in (0, 1, 63, 64, 65, 127, 128, 150, 191, 192, 199, 255, 256) if t < S} | {S - 1})
     heads = [0, 5, 127]
     for b in range(B):
         res, rows = oracle_prefill(w, inp, b, t_list, heads)
@@ -314,8 +316,9 @@ def test_prefill_reduced(B, S):
             assert_close(out[b, t_list, h], res[h], "bf16", f"prefill b={b} h={h}")
         assert len(rows) == S
         check_rows(cache[b * S:(b + 1) * S], rows, "bf16", "prefill cache")
-    res, _ = oracle_prefill(w, inp, 1, [0, 150], [3], absorbed=False)
-    assert_close(out[1, [0, 150], 3], res[3], "bf16", "prefill naive")
+    tn = sorted({0, min(150, S - 1)})
+    res, _ = oracle_prefill(w, inp, B - 1, tn, [3], absorbed=False)
+    assert_close(out[B - 1, tn, 3], res[3], "bf16", "prefill naive")
 
 
 def test_prefill_token_major_projections():
