@@ -531,6 +531,46 @@ def test_multi_token_decode_over_pages_matches_the_oracle():
     assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", "multi-token decode")
 
 
+def test_chunked_prefill_over_an_existing_cache():
+    """Absorbed chunked prefill: a chunk of 100 new tokens per sequence attends to a cached
+    prefix (300 and 77 tokens) and causally to itself, K and V never materialised: the
+    multi-token call with q_len = the chunk (200 per-token sequences).  Sampled tokens of
+    the chunk against the oracle, whose multi-token decode is pinned to its causal prefill."""
+    chunk, prefix = 100, [300, 77]
+    lengths = [p + chunk for p in prefix]
+    w, inp = reduced_attn_inputs(lengths, seed=59)
+    r = np.random.default_rng(59)
+    qn = torch.from_numpy(r.standard_normal((w.B, chunk, w.H, w.qk_nope))).to(torch.bfloat16)
+    qr = torch.from_numpy(r.standard_normal((w.B, chunk, w.H, w.d_hR))).to(torch.bfloat16)
+    npg = [(L + 63) // 64 for L in lengths]
+    pages = torch.zeros(sum(npg), 64, w.row, dtype=torch.bfloat16)
+    table = np.zeros((w.B, max(npg)), dtype=np.int32)
+    offs = inp["offsets"].numpy()
+    perm = r.permutation(sum(npg))
+    k = 0
+    for b, L in enumerate(lengths):
+        for j in range(npg[b]):
+            p = int(perm[k])
+            k += 1
+            table[b, j] = p
+            n = min(64, L - 64 * j)
+            pages[p, :n] = inp["cache"][offs[b] + 64 * j: offs[b] + 64 * j + n]
+    dims = dims_of(w)
+    g = to_dev({k_: inp[k_] for k_ in ("W_UK", "W_UV")})
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+    ws = mla.workspace(mla.mla_decode_multi_workspace_size(dims, w.B, chunk, table.shape[1]))
+    out = torch.empty(w.B, chunk, w.H, w.v_head, dtype=torch.bfloat16, device=DEV)
+    mla.mla_decode_absorbed_paged_multi(dims, weights, pages.to(DEV), torch.from_numpy(table).to(DEV),
+                                        torch.tensor(lengths, dtype=torch.int32, device=DEV), out, ws,
+                                        q_nope=qn.to(DEV), q_rope=qr.to(DEV))
+    assert mla.mla_get_device_error() == (0, 0)
+    out = out.cpu()
+    units = [(b, t, h) for b in range(w.B) for t in (0, 1, 63, 64, 99) for h in (0, 64, 127)]
+    want = oracle.decode_multi(qn, qr, inp["cache"], inp["offsets"], inp["W_UK"], inp["W_UV"], w.scale,
+                               units=units, absorbed=True)
+    assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", "chunked prefill")
+
+
 def test_decode_large_batch_spans_several_sequence_blocks():
     """B = 200 short ragged sequences: the q-absorb kernel runs two blocks of 128 sequences
     and the merge kernel four blocks of 64; sampled units against the oracle."""
