@@ -133,6 +133,13 @@ def alg_kernel_bytes(name: str, w: workloads.Workload) -> int:
     return cache + w.B * w.H * (w.d_c * 4 + w.d_hR * 2)
 
 
+def alg_kernel_flops(name: str, w: workloads.Workload) -> int:
+    """Algorithmic flops of one launch of the attention kernel: per attended token and head,
+    2 x (d_c + d_hR) for the score and 2 x d_c for P c."""
+    tokens = int(workloads.lengths(w).sum())
+    return tokens * w.H * (2 * w.row + 2 * w.d_c)
+
+
 def peaks() -> tuple:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -483,6 +490,15 @@ def run_ours(args, w0):
                         "unit": "GB/s", "frac": achieved / pk["hbm_gbs"], "traffic": traffic_for(dom),
                         "alg_bytes_per_launch": kbytes, "launch_us": launch_s * 1e6,
                         "peak_source": f"{pk_kind} hbm_gbs"}
+            # the absorbed decode sits next to the ridge point: report the tensor side too
+            kflops = alg_kernel_flops(dom, w)
+            tf = kflops / launch_s / 1e12
+            roofline["tensor_side"] = {
+                "alg_flops_per_launch": kflops, "achieved_tflops": tf, "peak": pk["bf16_tflops"],
+                "frac": tf / pk["bf16_tflops"], "peak_sustained": pk["bf16_tflops_sustained"],
+                "frac_sustained": tf / pk["bf16_tflops_sustained"],
+                "intensity_flop_per_byte": kflops / kbytes,
+                "ridge_flop_per_byte": pk["bf16_tflops"] * 1e12 / (pk["hbm_gbs"] * 1e9)}
             metric, unit = METRIC, "tokens/s"
         else:
             # whole-step roofline: these steps chain several kernels of different bounds

@@ -23,6 +23,11 @@ def test_decode_step_algorithmic_bytes_and_flops():
     assert round(a["flops"] / 1e9, 1) == 37.6
     # the dominant kernel reads the cache and the absorbed and rotary queries once
     assert bench.alg_kernel_bytes("tc_flash_decode", w) == tokens * 1152 + 32 * 128 * 576 * 2
+    # 2176 flops per attended token and head: 242 flop per cache byte, next to the measured
+    # ridge of about 249 flop/B (1628.3 TFLOP/s over 6535.1 GB/s)
+    f = bench.alg_kernel_flops("tc_flash_decode", w)
+    assert f == tokens * 128 * 2176
+    assert 240 < f / (tokens * 1152) < 243
 
 
 def test_layer_and_prefill_steps_count_their_weights():
