@@ -34,7 +34,10 @@ cudaError_t rope_table(const int32_t* pos, int pos_mod, int N, int d_rope, float
 
 // C[z][m][n] = sum_k A[z][m][k] * B[z][n][k] for z < Z, m < M, n < N.
 // A rows are K-contiguous with element strides (sAz, sAm); B rows likewise (sBz, sBn);
-// sBz = 0 shares one B among all z.
+// sBz = 0 shares one B among all z, and sAz = 0 (Z > 1) one A.  From 1024 tokens (N) on,
+// with bf16 output, unit m stride and 16-byte aligned rows, the tile is computed token-major
+// (a thread per token, 16-byte stores); otherwise weights-major.  The grid is persistent:
+// min(tiles, SMs) CTAs.
 // Row strides must be multiples of 8 elements (16 bytes) and the bases 16-byte aligned.
 // The launch uses programmatic dependent launch.  A (read before waiting for the previous
 // kernel) must not be written by it.  chain_head: wait for all earlier work before letting
