@@ -250,36 +250,66 @@ def rank_workload(w: workloads.Workload, rank: int) -> workloads.Workload:
 
 # ------------------------------------------------------------------ CPU oracle
 
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except (AttributeError, OSError):
+        return os.cpu_count() or 1
+
+
 def time_oracle_units(w: workloads.Workload, inp: dict, budget_s: float, min_units: int = 2,
-                      max_units: int = 10 ** 6, tokens: int = 0):
-    """Run the float64 naive oracle on (b, h) units until `budget_s` is spent.  With
-    tokens > 0 each unit attends over only its first `tokens` rows; the naive cost is
-    linear in the rows attended, so the step time scales by (rows of the unit / tokens)."""
+                      max_units: int = 10 ** 6, tokens: int = 0, threads: int = 1):
+    """Run the float64 naive oracle on seeded (b, h) units until `budget_s` of wall time is
+    spent, on `threads` host threads (the oracle's C routine runs outside the interpreter
+    lock, one unit per thread at a time).  With tokens > 0 each unit attends over only its
+    first `tokens` rows; the naive cost is linear in the rows attended, so a unit's time
+    scales by (rows of the unit / tokens).  Throughput = units done / wall time, scaled to
+    the full step of B x H units."""
     import oracle
+    from concurrent.futures import ThreadPoolExecutor
     offs = inp["offsets"].numpy().astype(np.int64)
     rng = np.random.default_rng(0)
+    units = [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(min(max_units, 1 << 16))]
     lib = oracle.load()
-    done, t_spent, scale_sum = 0, 0.0, 0.0
-    while done < max_units and (done < min_units or t_spent < budget_s):
-        b, h = int(rng.integers(w.B)), int(rng.integers(w.H))
-        T = int(offs[b + 1] - offs[b])
-        n = T if tokens <= 0 else max(1, min(T, tokens))
-        rows = inp["cache"][offs[b]:offs[b] + n]
-        t = time.perf_counter()
-        oracle.attend(inp["q_nope"][b, h], inp["q_rope"][b, h], rows, inp["W_UK"][h], inp["W_UV"][h],
-                      w.scale, absorbed=False, lib=lib)
-        dt = time.perf_counter() - t
-        t_spent += dt
-        scale_sum += dt * T / n
-        done += 1
-    per_unit = scale_sum / done
-    step_s = per_unit * w.B * w.H
+    lock = threading.Lock()
+    state = {"next": 0, "done": 0, "scaled": 0.0, "busy": 0.0}
+    t_start = time.perf_counter()
+
+    def worker():
+        while True:
+            with lock:
+                i = state["next"]
+                over = time.perf_counter() - t_start >= budget_s and i >= min_units
+                if i >= len(units) or i >= max_units or over:
+                    return
+                state["next"] = i + 1
+            b, h = units[i]
+            T = int(offs[b + 1] - offs[b])
+            n = T if tokens <= 0 else max(1, min(T, tokens))
+            rows = inp["cache"][offs[b]:offs[b] + n]
+            t = time.perf_counter()
+            oracle.attend(inp["q_nope"][b, h], inp["q_rope"][b, h], rows, inp["W_UK"][h], inp["W_UV"][h],
+                          w.scale, absorbed=False, lib=lib)
+            dt = time.perf_counter() - t
+            with lock:
+                state["done"] += 1
+                state["scaled"] += T / n
+                state["busy"] += dt
+
+    with ThreadPoolExecutor(max_workers=threads) as ex:
+        for f in [ex.submit(worker) for _ in range(threads)]:
+            f.result()
+    wall = time.perf_counter() - t_start
+    done = state["done"]
+    # full-row units per second of wall time, over all threads
+    rate = state["scaled"] / wall
+    step_s = w.B * w.H / rate
     what = "all rows" if tokens <= 0 else f"its first {tokens} rows (time scaled to all rows)"
-    return {"value": w.B / step_s, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"{done} (sequence, head) units of {w.name}, each over {what}, through the naive "
-                      f"float64 oracle (K and V materialised), {t_spent:.1f} s single-threaded; the full "
-                      f"step ({w.B * w.H} units) extrapolated as {per_unit * 1e3:.1f} ms x {w.B * w.H}",
-            "step_s_extrapolated": step_s}
+    return {"value": w.B / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{done} seeded (sequence, head) units of {w.name}, each over {what}, through the naive "
+                      f"float64 oracle (K and V materialised) on {threads} host thread(s) for {wall:.1f} s; "
+                      f"the full step ({w.B * w.H} units) extrapolated from the units per second",
+            "step_s_extrapolated": step_s, "unit_s_mean": state["busy"] / max(done, 1)}
 
 
 # ------------------------------------------------------------------------ arms
@@ -294,18 +324,22 @@ def run_reference(args, w):
     oracle.load()
     # calibrate: rows per second of the naive oracle, then size each step's sample so the
     # whole run (warm-up + timed) takes about args.reference_seconds
+    cores = host_cores()
     cal = time_oracle_units(w, inp, 0.0, min_units=2, max_units=2, tokens=256)
-    rows_per_s = 256.0 / (cal["step_s_extrapolated"] / (w.B * w.H) * 256.0 / w.ctx) if w.ctx else 1e5
+    rows_per_s = 256.0 / cal["unit_s_mean"]   # rows per second of one thread
     per_step = args.reference_seconds / (args.steps + args.warmup)
+    # each step is one unit per host thread, over the first `tokens` rows of its sequence
     tokens = int(max(16, min(w.ctx or 10 ** 9, per_step * rows_per_s)))
-    time_oracle_units(w, inp, 0.0, min_units=args.warmup, max_units=args.warmup, tokens=tokens)
-    r = time_oracle_units(w, inp, 0.0, min_units=args.steps, max_units=args.steps, tokens=tokens)
+    time_oracle_units(w, inp, 0.0, min_units=cores * args.warmup, max_units=cores * args.warmup, tokens=tokens,
+                      threads=cores)
+    r = time_oracle_units(w, inp, 0.0, min_units=cores * args.steps, max_units=cores * args.steps, tokens=tokens,
+                          threads=cores)
     line = {"impl": "reference", "metric": METRIC, "value": r["value"], "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": r["step_s_extrapolated"] * 1e3, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": config_of(w, world),
-            "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": r["value"], "unit": "tokens/s", "cores": r["cores"], "kind": "oracle",
                              "sample": r["sample"]},
             "e2e": {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -422,17 +456,21 @@ def run_ours(args, w0):
         if profile:
             mla.mla_profile_enable(False)
             prof = mla.mla_profile_report(reset=True)
-        return float(np.mean([a_.elapsed_time(b_) for a_, b_ in ev])), prof, t0, t1
+        return [a_.elapsed_time(b_) for a_, b_ in ev], prof, t0, t1
 
     # timed region: per-step CUDA events, the L2 flush between them (outside the events);
-    # the library's kernels chain with programmatic dependent launch
-    ms_local, _, t0, t1 = timed_pass(False)
-    ms = max_over_ranks(ms_local)
+    # the library's kernels chain with programmatic dependent launch.  The step time is the
+    # median of the per-step events (p10 / p90 reported beside it), max over ranks.
+    step_ms, _, t0, t1 = timed_pass(False)
+    ms = max_over_ranks(float(np.median(step_ms)))
+    pct = {"p10": max_over_ranks(float(np.percentile(step_ms, 10))),
+           "p90": max_over_ranks(float(np.percentile(step_ms, 90))),
+           "mean": max_over_ranks(float(np.mean(step_ms)))}
     # second timed pass: CUDA events around every library launch on its stream give each
     # kernel's live launch duration (events between launches stop the kernels from
     # overlapping, so this pass is slower than the first)
-    ms_prof_local, prof, _, _ = timed_pass(True)
-    ms_prof = max_over_ranks(ms_prof_local)
+    prof_ms, prof, _, _ = timed_pass(True)
+    ms_prof = max_over_ranks(float(np.median(prof_ms)))
     clk = clocks.summary(t0, t1) if clocks else None
     if clocks:
         clocks.stop()
@@ -465,15 +503,23 @@ def run_ours(args, w0):
         if j >= 0:
             ev3[j][1].record(stream)
     torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(float(np.mean([a_.elapsed_time(b_) for a_, b_ in ev3])))
+    e2e_all = [a_.elapsed_time(b_) for a_, b_ in ev3]
+    e2e_ms = max_over_ranks(float(np.median(e2e_all)))
+    e2e_pct = {"p10": max_over_ranks(float(np.percentile(e2e_all, 10))),
+               "p90": max_over_ranks(float(np.percentile(e2e_all, 90)))}
     st, det = mla.mla_get_device_error()
     if st != 0:
         raise RuntimeError(f"device error {st} ({det})")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kind == "decode_attn":
-        cpu = time_oracle_units(w, inp, args.cpu_seconds)
-        cpu.pop("step_s_extrapolated", None)
+        cores = host_cores()
+        one = time_oracle_units(w, inp, args.cpu_seconds / 4)
+        cpu = time_oracle_units(w, inp, args.cpu_seconds, min_units=cores, threads=cores)
+        cpu["single_core"] = {"value": one["value"], "unit": "tokens/s", "sample": one["sample"]}
+        cpu["nproc"] = cores
+        for k in ("step_s_extrapolated", "unit_s_mean"):
+            cpu.pop(k, None)
 
     if rank == 0:
         pk, pk_kind = peaks()
@@ -515,7 +561,9 @@ def run_ours(args, w0):
             unit = "tokens/s"
         line = {
             "metric": metric, "value": world * units / step_s, "unit": unit, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+            "ms_per_step_stats": {"stat": "median of the per-step CUDA events", **pct},
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
             "config": config_of(w, world),
             "step_roofline": {"alg_bytes": a["bytes"], "alg_flops": a["flops"], "roofline_us": roof_s * 1e6,
@@ -527,6 +575,7 @@ def run_ours(args, w0):
             "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": unit,
                     "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for _, v in h2d)),
                     "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms,
+                    "ms_p10": e2e_pct["p10"], "ms_p90": e2e_pct["p90"],
                     "api": "mla_decode_absorbed_host" if w.kind == "decode_attn" else "device call + torch copies",
                     "note": "latent cache and weights stay resident in HBM (decode state)"},
             "gpu_launches": int(round(launches_per_step * args.steps)),

@@ -61,6 +61,8 @@ SIGNATURES = {
     "mla_decode_multi_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "mla_decode_absorbed_host": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
                                       ctypes.c_size_t, _P]),
+    "mla_set_wait_limit": (_S, [ctypes.c_uint32]),
+    "mla_test_starve_projection": (_S, [ctypes.c_int32]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
     "mla_profile_report": (ctypes.c_int32, [ctypes.c_char_p, ctypes.c_size_t, ctypes.c_int32]),
 }
@@ -239,6 +241,16 @@ def mla_get_device_error(stream=None):
     d = ctypes.c_int64(0)
     st = _lib.mla_get_device_error(_stream(stream), ctypes.byref(d))
     return int(st), int(d.value)
+
+
+def mla_set_wait_limit(polls: int) -> None:
+    """Polls each bounded device wait makes before giving up (0 = the default); a test hook."""
+    _check(_lib.mla_set_wait_limit(int(polls)), "mla_set_wait_limit")
+
+
+def mla_test_starve_projection(on: bool) -> None:
+    """While on, the projection GEMM's loader issues no loads so its waits run out (test hook)."""
+    _check(_lib.mla_test_starve_projection(1 if on else 0), "mla_test_starve_projection")
 
 
 def mla_profile_enable(on: bool = True) -> None:

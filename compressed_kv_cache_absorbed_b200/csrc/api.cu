@@ -634,6 +634,10 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
     const bool tc_proj = tc_proj_ok(d) && aligned16(h) && aligned16(w->W_Q) && aligned16(cache) &&
                          aligned16(w->W_UK) && aligned16(w->W_UV);
     if (tc_proj) {
+        // The tensor-core attention reads the content parts of q and K and all of V as fp16
+        // (more precise than bf16 for these magnitudes, same MMA rate); the rotary columns stay
+        // bf16, as the cache's k_r is.  Other shapes keep every intermediate in bf16.
+        const bool tc_attn = qk == 128 && dR == 64 && vh == 128 && dc == 512 && aligned16(out);
         // 2. queries with RoPE at t = i % S
         { mla::ProfScope ps(s, "tc_q_proj_rope");
         e = mla::tc::rope_table(nullptr, S, n, dR, theta_of(d), ws.rope_tab, s);
@@ -643,6 +647,7 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
         oq.rope_start = qk;
         oq.d_rope = dR;
         oq.rope_tab = ws.rope_tab;
+        oq.f16 = tc_attn;
         e = mla::tc::gemm_bf16_tc(1, H * qh, n, d->d_model, (const bf16*)w->W_Q, 0, d->d_model, (const bf16*)h, 0,
                                   d->d_model, oq, err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
@@ -650,20 +655,21 @@ static cudaError_t prefill_impl(const mla_dims* d, mla_weights w, const void* h,
         { mla::ProfScope ps(s, "tc_k_materialise");
         // all heads in one product: W_UK as [H * qk, d_c] rows, K_nope[t] = [H * qk] wide
         mla::tc::GemmOut okb{ws.k_buf, 0, 1, (long long)H * qk, 0};
+        okb.f16 = tc_attn;
         e = mla::tc::gemm_bf16_tc(1, H * qk, n, dc, (const bf16*)w->W_UK, 0, dc, (const bf16*)cache, 0, row, okb,
                                   err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
         { mla::ProfScope ps(s, "tc_v_materialise");
         mla::tc::GemmOut ovb{ws.v_buf, 0, 1, (long long)H * vh, 0};
+        ovb.f16 = tc_attn;
         e = mla::tc::gemm_bf16_tc(1, H * vh, n, dc, (const bf16*)w->W_UV, 0, dc, (const bf16*)cache, 0, row, ovb,
                                   err.code, err.detail, s); }
         if (e != cudaSuccess) return e;
-        if (qk == 128 && dR == 64 && vh == 128 && dc == 512 && aligned16(out)) {
+        if (tc_attn) {
             // 4. causal attention on the tensor cores
             mla::ProfScope ps(s, "tc_prefill_attn");
-            return mla::tc::prefill_attn_tc((const bf16*)ws.q_buf, (const bf16*)ws.k_buf, (const bf16*)cache,
-                                            (const bf16*)ws.v_buf, B, S, H, scale_of(d), (bf16*)out, err.code,
-                                            err.detail, s);
+            return mla::tc::prefill_attn_tc(ws.q_buf, ws.k_buf, (const bf16*)cache, ws.v_buf, B, S, H, scale_of(d),
+                                            (bf16*)out, err.code, err.detail, s);
         }
         mla::ProfScope ps(s, "simt_prefill_attn");
         return mla::launch_prefill_attn_simt<T>((const T*)ws.q_buf, (const T*)ws.k_buf, (const T*)cache,
@@ -715,6 +721,19 @@ extern "C" mla_status mla_prefill_causal(const mla_dims* d, mla_weights w, const
 }
 
 // ------------------------------------------------------------------- diagnostics
+
+extern "C" mla_status mla_set_wait_limit(uint32_t polls) {
+    const uint32_t p = polls ? polls : 1u << 22;
+    MLA_CUDA(mla::tc::set_wait_limit_decode(p));
+    MLA_CUDA(mla::tc::set_wait_limit_gemm(p));
+    MLA_CUDA(mla::tc::set_wait_limit_prefill(p));
+    return MLA_OK;
+}
+
+extern "C" mla_status mla_test_starve_projection(int32_t on) {
+    MLA_CUDA(mla::tc::set_starve_gemm(on ? 1 : 0));
+    return MLA_OK;
+}
 
 extern "C" mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail) {
     MLA_CUDA(cudaStreamSynchronize((cudaStream_t)stream));

@@ -113,12 +113,29 @@ struct Seg {
 // Where the cache rows of a sequence live: rows [offsets[b], offsets[b+1]) of the cache, or,
 // with a block table (paged cache), seq_lens[b] tokens in 64-token pages, tile j of sequence
 // b in page block_table[b * bt_stride + j] (cache rows 64 page .. 64 page + 63).
+//
+// A sequence whose rows are not inside the cache (decreasing or negative offsets, rows past
+// cache_rows, more tokens than its block-table row has pages for) is invalid: raw_len
+// returns -1 for it, the planner latches MLA_ERR_OUT_OF_RANGE, and every role of both
+// kernels sees it as empty (len = 0), so its output is zero and no CTA has to abort.
 struct SeqSrc {
     const int32_t* offsets;
     const int32_t* seq_lens;
     const int32_t* block_table;
     int bt_stride;
-    __device__ int len(int b) const { return block_table ? seq_lens[b] : offsets[b + 1] - offsets[b]; }
+    long long cache_rows;
+    __device__ int raw_len(int b) const {
+        if (block_table) {
+            const int L = seq_lens[b];
+            return (L < 0 || (long long)L > (long long)bt_stride * 64) ? -1 : L;
+        }
+        const long long r0 = offsets[b], r1 = offsets[b + 1];
+        return (r0 < 0 || r1 < r0 || r1 > cache_rows) ? -1 : (int)(r1 - r0);
+    }
+    __device__ int len(int b) const {
+        const int L = raw_len(b);
+        return L > 0 ? L : 0;
+    }
     __device__ long long row0(int b) const { return block_table ? 0 : offsets[b]; }
 };
 
@@ -177,7 +194,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     }
     // this thread's sequence length for the planning below, requested before the set-up
     // so that the load overlaps it
-    const int len0 = threadIdx.x < B ? src.len(threadIdx.x) : 0;
+    const int len0 = threadIdx.x < B ? src.raw_len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
     uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
@@ -257,8 +274,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     {
         int mine = 0;
         for (int b = threadIdx.x; b < B; b += kThreads) {
-            const int L = b == (int)threadIdx.x ? len0 : src.len(b);
-            if (L < 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
+            const int L = b == (int)threadIdx.x ? len0 : src.raw_len(b);
+            if (L < 0 && blockIdx.x == 0) latch(DevErr{err_code, err_detail}, kErrOutOfRange, b);
             mine += cost_of_tiles(tiles_of_len(L));
         }
 #pragma unroll
@@ -319,12 +336,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             const uint64_t stream_policy = ptx::policy_evict_first();
             uint32_t g = 0;
             while (!*abort_flag && it.next(sg)) {
-                if (src.block_table ? sg.L > src.bt_stride * kT                 // more pages than the table row
-                                    : sg.row0 + (long long)sg.L > cache_rows) {  // sequence beyond the cache
-                    latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
-                    *abort_flag = 1;
-                    break;
-                }
                 for (int j = sg.j0; j < sg.j1; ++j, ++g) {
                     const int s = g % kStages;
                     const uint32_t n = g / kStages;
@@ -336,12 +347,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     long long row_l = sg.row0 + (long long)j * kT;
                     if (src.block_table) {
                         const long long page = src.block_table[(long long)sg.b * src.bt_stride + j];
-                        if (page < 0 || (page + 1) * kT > cache_rows) {   // page outside the cache
+                        if (page < 0 || (page + 1) * kT > cache_rows) {
+                            // a page outside the cache: latch the error and load a tile that
+                            // lies wholly past the tensor's last row, which TMA fills with
+                            // zeros, so every role still sees the tile it expects
                             latch(DevErr{err_code, err_detail}, kErrOutOfRange, sg.b);
-                            *abort_flag = 1;
-                            break;
+                            row_l = cache_rows;
+                        } else {
+                            row_l = page * kT;
                         }
-                        row_l = page * kT;
                     }
                     const int row = (int)row_l;
                     ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
@@ -389,7 +403,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             uint32_t s_g = 0;
             bool o_have = !*abort_flag && it.next(sg);
             int o_j = o_have ? sg.j0 : 0;
-            uint32_t idle = 0;
+            // the issuer polls its barriers without blocking: allow 16 polls per wait poll
+            const uint64_t idle_limit = (uint64_t)ptx::g_wait_limit << 4;
+            uint64_t idle = 0;
             while (o_have) {
                 // ---- O of tile g
                 if (g < s_g && ptx::mbar_test(&p_ready[g & 1], (g >> 1) & 1)) {
@@ -442,7 +458,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         continue;
                     }
                 }
-                if (++idle > (ptx::kWaitLimit << 4) || *abort_flag) {
+                if (++idle > idle_limit || *abort_flag) {
                     ok = false;
                     break;
                 }
@@ -1102,6 +1118,8 @@ int max_clusters(int num_sms) {
 
 }  // namespace
 
+cudaError_t set_wait_limit_decode(uint32_t polls) { return ptx::set_wait_limit_of_this_file(polls); }
+
 cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
                             __nv_bfloat16* uv, cudaStream_t s) {
     tile_weights_kernel<<<1184, 256, 0, s>>>(W_UKT, W_UV, ukt, uv);
@@ -1144,7 +1162,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     cudaError_t e;
     if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
     if (block_table && (!seq_lens || bt_stride <= 0)) return cudaErrorInvalidValue;
-    const SeqSrc seqs{offsets, seq_lens, block_table, bt_stride};
+    const SeqSrc seqs{offsets, seq_lens, block_table, bt_stride, cache_rows};
     const int P = max_clusters(num_sms);
     {
         // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]

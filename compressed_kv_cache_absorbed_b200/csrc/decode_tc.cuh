@@ -54,5 +54,8 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
                                int B, float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s);
 
+// Sets the polls a bounded wait of this file's kernels makes before giving up (current device).
+cudaError_t set_wait_limit_decode(uint32_t polls);
+
 }  // namespace tc
 }  // namespace mla

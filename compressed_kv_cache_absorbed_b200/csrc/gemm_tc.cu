@@ -39,6 +39,18 @@ struct GemmCfg {
     static constexpr int SMEM = STAGES * STAGE + 1024 + 256;
 };
 
+// Test hook for the failure-detection path (set only by mla_test_starve_projection): when
+// nonzero the loader warp issues no loads, so the MMA issuer's and the epilogue's bounded
+// waits run out and latch a timeout while no copy and no MMA is in flight.
+__device__ int g_starve_loads = 0;
+
+// fp16 store of an fp32 value, saturated to the finite range
+__device__ __forceinline__ __half to_half_sat(float v) { return __float2half_rn(fminf(fmaxf(v, -65504.f), 65504.f)); }
+__device__ __forceinline__ uint32_t pack_half_sat(float lo, float hi) {
+    __half2 h = __halves2half2(to_half_sat(lo), to_half_sat(hi));
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
 __device__ __forceinline__ void fail(int* code, long long* detail, volatile int* abort_flag, int where) {
     latch(DevErr{code, detail}, kErrTimeout, (long long)where * 1000000 + blockIdx.x);
     *abort_flag = 1;
@@ -123,7 +135,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
     }
 
     if (warp == 0) {
-        if (lane == 0) {
+        if (lane == 0 && !g_starve_loads) {
             ptx::tma_prefetch(&tmX);
             ptx::tma_prefetch(&tmY);
             auto load_x = [&](uint8_t* st, uint64_t* bar, int kb, const Tile& tl) {
@@ -268,17 +280,28 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         }
                     }
                     uint4* dst = (uint4*)((__nv_bfloat16*)base + (long long)tl.z * out.sz + f0 + orow * out.sn);
+                    // 32 columns from a multiple of 32: all fp16 or all bf16 (rope_start % 32 == 0)
+                    const bool half_out = out.f16 && (out.period == 0 || f0 % out.period < out.rope_start);
+                    if (half_out) {
 #pragma unroll
-                    for (int q = 0; q < 4; ++q)
-                        dst[q] = make_uint4(ptx::pack_bf16(v[8 * q], v[8 * q + 1]), ptx::pack_bf16(v[8 * q + 2], v[8 * q + 3]),
-                                            ptx::pack_bf16(v[8 * q + 4], v[8 * q + 5]),
-                                            ptx::pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(pack_half_sat(v[8 * q], v[8 * q + 1]), pack_half_sat(v[8 * q + 2], v[8 * q + 3]),
+                                                pack_half_sat(v[8 * q + 4], v[8 * q + 5]),
+                                                pack_half_sat(v[8 * q + 6], v[8 * q + 7]));
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            dst[q] = make_uint4(ptx::pack_bf16(v[8 * q], v[8 * q + 1]), ptx::pack_bf16(v[8 * q + 2], v[8 * q + 3]),
+                                                ptx::pack_bf16(v[8 * q + 4], v[8 * q + 5]),
+                                                ptx::pack_bf16(v[8 * q + 6], v[8 * q + 7]));
+                    }
                     continue;
                 }
                 // weights-major: feature row xr, tokens n0 + c0 .. + 31
                 const int row = xr;
                 const int within = out.period > 0 ? row % out.period : -1;
                 const bool rope_row = out.period > 0 && within >= out.rope_start;
+                const bool half_row = out.f16 && !rope_row;
 #pragma unroll
                 for (int j = 0; j < 32; ++j) {
                     const int n = tl.j0 + c0 + j;   // the same for the whole warp
@@ -305,6 +328,8 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     const long long idx = (long long)tl.z * out.sz + (long long)row * out.sm + orow * out.sn;
                     if (out.f32)
                         ((float*)base)[idx] = v;
+                    else if (half_row)
+                        ((__half*)base)[idx] = to_half_sat(v);
                     else
                         ((__nv_bfloat16*)base)[idx] = __float2bfloat16_rn(v);
                 }
@@ -351,6 +376,10 @@ rope_table_kernel(const int32_t* __restrict__ pos, int pos_mod, int N, int half,
 
 }  // namespace
 
+cudaError_t set_wait_limit_gemm(uint32_t polls) { return ptx::set_wait_limit_of_this_file(polls); }
+
+cudaError_t set_starve_gemm(int on) { return cudaMemcpyToSymbol(g_starve_loads, &on, sizeof on); }
+
 cudaError_t rope_table(const int32_t* pos, int pos_mod, int N, int d_rope, float theta, double2* tab,
                        cudaStream_t s) {
     if (N <= 0) return cudaSuccess;
@@ -373,7 +402,8 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     // token-major for many tokens when the output rows take 16-byte stores
     const bool swap = N >= kSwapMinTokens && !out.f32 && out.sm == 1 && M % 32 == 0 && out.sz % 8 == 0 &&
                       out.sn % 8 == 0 && ((uintptr_t)out.C & 15) == 0 &&
-                      (out.period == 0 || (out.period % 2 == 0 && out.rope_start % 2 == 0));
+                      (out.period == 0 || (out.period % 2 == 0 && out.rope_start % 2 == 0)) &&
+                      (!out.f16 || out.period == 0 || (out.period % 32 == 0 && out.rope_start % 32 == 0));
     const int Mx = swap ? N : M, Ny = swap ? M : N;   // MMA rows (128-tiles) and columns (BN-tiles)
     // the narrowest tile that covers Ny, narrowed further while there are fewer tiles than a
     // quarter of the SMs (very skinny weight-streaming GEMMs: the weights are then re-read

@@ -15,10 +15,14 @@ namespace tc {
 // index within the rotary block, pos(n) = pos ? pos[n] : n % pos_mod; with rope_tab set the
 // (cos, sin) of that angle are read from rope_tab[n * d_rope / 2 + i] instead of computed.
 // Rotation is done in double precision and the result rounded once.
+// f16 (with f32 == 0) stores fp16 instead of bf16: every column, or with period > 0 only the
+// columns m with (m % period) < rope_start (the rotary columns stay bf16).  fp16 stores
+// saturate at +-65504.
 struct GemmOut {
     void* C;
     long long sz, sm, sn;
     int f32;
+    int f16 = 0;
     const int64_t* slot = nullptr;
     long long cap = 0;
     int period = 0, rope_start = 0, d_rope = 0;
@@ -45,6 +49,14 @@ cudaError_t rope_table(const int32_t* pos, int pos_mod, int N, int d_rope, float
 cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, long long sAz, long long sAm,
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
                          int* err_code, long long* err_detail, cudaStream_t s, bool chain_head = false);
+
+// Sets the polls a bounded wait of the GEMM kernel makes before giving up (current device).
+cudaError_t set_wait_limit_gemm(uint32_t polls);
+
+// Failure-detection test hook: while on, the GEMM's loader issues no loads, so its MMA and
+// epilogue waits run out and the launch latches a timeout with nothing in flight
+// (current device).
+cudaError_t set_starve_gemm(int on);
 
 }  // namespace tc
 }  // namespace mla

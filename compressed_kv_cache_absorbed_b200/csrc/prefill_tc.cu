@@ -1,5 +1,6 @@
 // Causal prefill attention with K and V materialised, on the tcgen05 tensor cores, for the
-// DeepSeek-V2/V3 head shape (qk_nope = 128, d_hR = 64, v_head = 128), bf16.
+// DeepSeek-V2/V3 head shape (qk_nope = 128, d_hR = 64, v_head = 128): bf16 cache and output,
+// the materialised content parts of q and K, and V, in fp16 (see prefill_tc.cuh), P in fp16.
 //
 // For sequence b, head h and query position t (keys t' <= t of the same sequence):
 //     s[t, t'] = scale * (q_nope[t] . k_nope[t'] + q_rope[t] . k_r[t'])     (192-long)
@@ -12,7 +13,7 @@
 // (K: two 64-column boxes of k_nope and the 64 rotary columns of the cache rows; V: two
 // 64-column boxes), each with its own ring.  Per key block: S = Q K^T (M = 128, N = 128, K = 192: 12 MMAs, both
 // operands in shared memory) into TMEM, the online softmax in registers (base-2, lazy
-// rescale), P (bf16) back to TMEM in one of two buffers, O += P V (M = 128, N = 128,
+// rescale), P (fp16) back to TMEM in one of two buffers, O += P V (M = 128, N = 128,
 // K = 128: 8 MMAs with A = P from TMEM and B = V from shared memory).  The diagonal block is
 // masked causally; positions at or past the sequence end are masked too.  K and V have
 // rings of their own: a K stage is refilled as soon as its Q K^T product completes, and K
@@ -35,7 +36,7 @@ namespace tc {
 namespace {
 
 constexpr int kQ = 128, kKB = 128;          // queries per CTA, keys per block
-constexpr int kBox = 128 * 128;             // one 128-row x 64-column bf16 box (16 KB)
+constexpr int kBox = 128 * 128;             // one 128-row x 64-column box of 2-byte values (16 KB)
 constexpr int kQBytes = 3 * kBox;           // Q: nope 0-63, nope 64-127, rope
 constexpr int kKBytes = 3 * kBox;           // K: the same three column groups
 constexpr int kVBytes = 2 * kBox;           // V: columns 0-63, 64-127
@@ -172,8 +173,10 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
     } else if (warp == 1) {
         // --------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, kKB, 0, 0);
-            constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 128, 0, 1);   // B = V (MN-major)
+            // content columns (q_nope, k_nope) and P, V are fp16; the rotary columns bf16
+            constexpr uint32_t idesc_s_nope = ptx::idesc_f16_f32(128, kKB, 0, 0);
+            constexpr uint32_t idesc_s_rope = ptx::idesc_bf16_f32(128, kKB, 0, 0);
+            constexpr uint32_t idesc_o = ptx::idesc_f16_f32(128, 128, 0, 1);   // B = V (MN-major)
             bool ok = ptx::mbar_wait(q_full, 0, abort_flag);
             const uint32_t qa = ptx::smem_u32(sQ);
             auto issue_s = [&](int i) -> bool {
@@ -184,7 +187,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 #pragma unroll
                 for (int ks = 0; ks < 12; ++ks)   // 3 column groups x 4 K-steps of 16
                     ptx::mma_ss(tmem + kColS, ptx::desc_kmajor_sw128(qa + (ks >> 2) * kBox + (ks & 3) * 32),
-                                ptx::desc_kmajor_sw128(ka + (ks >> 2) * kBox + (ks & 3) * 32), idesc_s, ks != 0);
+                                ptx::desc_kmajor_sw128(ka + (ks >> 2) * kBox + (ks & 3) * 32),
+                                ks < 8 ? idesc_s_nope : idesc_s_rope, ks != 0);
                 ptx::mma_commit(s_full);
                 ptx::mma_commit(&k_empty[i & 1]);
                 return true;
@@ -298,7 +302,8 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                 }
                 ptx::tc_fence_after();
             }
-            // P = 2^(s scale_log2 - m) as bf16 pairs, 32 keys (16 TMEM columns) at a time
+            // P = 2^(s scale_log2 - m) as fp16 pairs (p <= 2^8 under the lazy rescale), 32
+            // keys (16 TMEM columns) at a time
             float sum = 0.f;
 #pragma unroll
             for (int c = 0; c < 64; c += 32) {
@@ -308,7 +313,7 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
                     const float p0 = ex2f_ftz(fmaf(sc[c + j], scale_log2, -m_run));
                     const float p1 = ex2f_ftz(fmaf(sc[c + j + 1], scale_log2, -m_run));
                     sum += p0 + p1;
-                    pw[j / 2] = ptx::pack_bf16(p0, p1);
+                    pw[j / 2] = ptx::pack_f16(p0, p1);
                 }
                 ptx::tmem_st16(lane_addr + kColP + par * 64 + hf * 32 + c / 2, pw);
             }
@@ -355,8 +360,10 @@ prefill_attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_co
 
 }  // namespace
 
-cudaError_t prefill_attn_tc(const __nv_bfloat16* q, const __nv_bfloat16* k_nope, const __nv_bfloat16* cache,
-                            const __nv_bfloat16* v, int B, int S, int H, float scale, __nv_bfloat16* out,
+cudaError_t set_wait_limit_prefill(uint32_t polls) { return ptx::set_wait_limit_of_this_file(polls); }
+
+cudaError_t prefill_attn_tc(const void* q, const void* k_nope, const __nv_bfloat16* cache,
+                            const void* v, int B, int S, int H, float scale, __nv_bfloat16* out,
                             int* err_code, long long* err_detail, cudaStream_t s) {
     if (B <= 0 || S <= 0) return cudaSuccess;
     const uint64_t n = (uint64_t)B * S;

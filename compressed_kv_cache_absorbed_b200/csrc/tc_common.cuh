@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -90,23 +91,34 @@ __device__ __forceinline__ bool mbar_try_cluster(uint64_t* bar, uint32_t parity)
     return ok != 0;
 }
 
-// A wait that gives up: spins at most `limit` polls (each try_wait itself blocks for a
+// A wait that gives up: polls at most g_wait_limit times (each try_wait itself blocks for a
 // hardware-defined interval), then returns false so the caller can record a timeout and
-// leave instead of hanging the GPU.
-constexpr uint32_t kWaitLimit = 1u << 22;
+// leave instead of hanging the GPU.  The limit is a device variable so that a test can
+// shorten it (mla_set_wait_limit); every file that includes this header has its own copy,
+// which set_wait_limit_of_this_file() sets on the current device.
+constexpr uint32_t kDefaultWaitLimit = 1u << 22;
+static __device__ uint32_t g_wait_limit = kDefaultWaitLimit;
+
+static inline cudaError_t set_wait_limit_of_this_file(uint32_t polls) {
+    return cudaMemcpyToSymbol(g_wait_limit, &polls, sizeof polls);
+}
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;   // the common case reads no limit
+    const uint32_t limit = g_wait_limit;
+    for (uint32_t i = 1; i < limit; ++i) {
         if (abort_flag && *abort_flag) return false;
+        if (mbar_try(bar, parity)) return true;
     }
     return false;
 }
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity,
                                                   const volatile int* abort_flag) {
-    for (uint32_t i = 0; i < kWaitLimit; ++i) {
-        if (mbar_try_cluster(bar, parity)) return true;
+    if (mbar_try_cluster(bar, parity)) return true;
+    const uint32_t limit = g_wait_limit;
+    for (uint32_t i = 1; i < limit; ++i) {
         if (abort_flag && *abort_flag) return false;
+        if (mbar_try_cluster(bar, parity)) return true;
     }
     return false;
 }
@@ -292,9 +304,18 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn_maj
     return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) |
            ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// The same for fp16 x fp16 -> fp32 (A and B formats 0 = f16).
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N, int a_mn_major, int b_mn_major) {
+    return (1u << 4) | ((uint32_t)a_mn_major << 15) | ((uint32_t)b_mn_major << 16) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
 

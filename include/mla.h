@@ -23,8 +23,8 @@
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
  *   - Argument errors are detected on the host and returned before anything is launched;
  *     outputs are then untouched.  Errors found on the device (a slot outside the cache,
- *     decreasing offsets) skip the offending work and latch a device error word that
- *     mla_get_device_error() reads.  No call traps, aborts or throws.
+ *     decreasing offsets, a sequence past the cache) skip the offending work and latch a
+ *     device error word that mla_get_device_error() reads.  No call traps, aborts or throws.
  *   - The caller owns every tensor (cache, inputs, outputs, workspace).  The only
  *     library-owned object is an mla_weights handle (device memory it allocates once).
  *   - Storage type: all float tensors of one call share `dims->dtype` (fp32 or bf16);
@@ -141,14 +141,16 @@ size_t mla_decode_workspace_size(const mla_dims* dims, int32_t B);
  *     o[b,h]      = W_UV[h] o_lat[b,h]                            (v_head)
  *     out[b]      = W_O concat_h o[b,h]        (only when the handle holds W_O)
  * Sequence b attends over cache rows [offsets[b], offsets[b+1]) (int32 [B+1], ragged) of a
- * cache of cache_rows rows (1 <= cache_rows < 2^31); a sequence reaching past cache_rows
- * latches MLA_ERR_OUT_OF_RANGE.
+ * cache of cache_rows rows (1 <= cache_rows < 2^31).  A sequence whose rows are not inside
+ * the cache (offsets[b] < 0, offsets[b+1] < offsets[b] or offsets[b+1] > cache_rows) latches
+ * MLA_ERR_OUT_OF_RANGE on the device and decodes to zeros; the other sequences of the call
+ * are computed as usual.
  * An empty sequence gives o = 0.  The query comes either from (q_nope [B,H,qk_nope],
  * q_rope [B,H,d_hR], q_rope already rotated) or, when both are NULL, from the hidden
  * state h [B, d_model] through the handle's W_Q with RoPE at q_pos int32 [B].
  * out is [B, H, v_head], or [B, d_model] when the handle holds W_O.
  * workspace: device, >= mla_decode_workspace_size(dims, B) bytes, 256-byte aligned;
- * its contents on entry do not matter.  Decreasing offsets latch MLA_ERR_OUT_OF_RANGE. */
+ * its contents on entry do not matter. */
 mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* q_nope,
                                const void* q_rope, const void* h, const int32_t* q_pos,
                                const void* cache, int64_t cache_rows, const int32_t* offsets,
@@ -163,8 +165,10 @@ mla_status mla_decode_absorbed(const mla_dims* dims, mla_weights w, const void* 
  * cache as a layer orthogonal to MLA ["DeepSeek MLA", the PagedAttention comparison].
  * Queries from q_nope/q_rope only; the tensor-core shape only (bf16, H = 128, d_c = 512,
  * d_hR = 64, qk_nope = v_head = 128) and handles without W_O, else MLA_ERR_UNSUPPORTED.
- * A sequence needing more than max_blocks pages, or a page outside [0, num_pages), latches
- * MLA_ERR_OUT_OF_RANGE on the device.  Workspace: mla_decode_workspace_size(dims, B). */
+ * A sequence needing more than max_blocks pages (or with seq_lens[b] < 0) latches
+ * MLA_ERR_OUT_OF_RANGE on the device and decodes to zeros; a page outside [0, num_pages)
+ * latches the same error and its tile is read as zeros (that sequence's output is then
+ * meaningless; the others are unaffected).  Workspace: mla_decode_workspace_size(dims, B). */
 mla_status mla_decode_absorbed_paged(const mla_dims* dims, mla_weights w, const void* q_nope,
                                      const void* q_rope, const void* cache, int64_t num_pages,
                                      const int32_t* block_table, int32_t max_blocks,
@@ -187,7 +191,7 @@ mla_status mla_decode_absorbed_paged(const mla_dims* dims, mla_weights w, const 
  * seq_lens[b] - q_len + t + 1 tokens; a token with no key (seq_lens[b] < q_len - t) gets
  * zeros.  Tensor-core shape only and handles without W_O, else MLA_ERR_UNSUPPORTED; a page
  * outside [0, num_pages) or more than max_blocks blocks latch MLA_ERR_OUT_OF_RANGE on the
- * device.  Each new token streams its own keys: the cache bytes read are q_len times those
+ * device, as for mla_decode_absorbed_paged.  Each new token streams its own keys: the cache bytes read are q_len times those
  * of one decode step.
  * Workspace: device, >= mla_decode_multi_workspace_size(dims, B, q_len, max_blocks) bytes,
  * 256-byte aligned, contents on entry do not matter. */
@@ -267,6 +271,23 @@ mla_status mla_prefill_causal(const mla_dims* dims, mla_weights w, const void* h
  * latched code (MLA_ERR_OUT_OF_RANGE, MLA_ERR_DEVICE_TIMEOUT); *detail (nullable)
  * receives a kernel-specific detail value. */
 mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail);
+
+/* Failure-detection test hooks.  Leave both at their defaults outside tests.
+ *
+ * mla_set_wait_limit: on the current device, the number of polls each bounded wait in the
+ * library's tensor-core kernels (a kernel waiting for its own loads, MMAs or sibling warps)
+ * makes before it gives up, latches MLA_ERR_DEVICE_TIMEOUT, drains what it issued, frees its
+ * tensor memory and returns.  0 restores the default (2^22 polls, seconds).  Synchronous
+ * (cudaMemcpyToSymbol); call it with no library kernel running.
+ *
+ * mla_test_starve_projection: while on != 0, the loader warp of the tensor-core projection
+ * GEMM (the kernel behind mla_append_cache on bf16, the query projection and W_O) issues no
+ * loads, so its MMA and epilogue waits run out: such a call writes no output and latches
+ * MLA_ERR_DEVICE_TIMEOUT, with no copy and no MMA in flight, and the next call works.  It is
+ * how the timeout path is tested without faulting or hanging the GPU.  Current device,
+ * synchronous. */
+mla_status mla_set_wait_limit(uint32_t polls);
+mla_status mla_test_starve_projection(int32_t on);
 
 /* Per-kernel device timing of this library's own launches (a diagnostic, off by default).
  * While enabled, each launch is bracketed by two CUDA events recorded on its stream. */

@@ -10,3 +10,15 @@ for p in (ROOT, HERE):
 
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a CUDA device (B200, sm_100a)")
+
+
+def pytest_terminal_summary(terminalreporter):
+    """The parity margins: the largest err/limit ratios of the comparisons that ran."""
+    from helpers import RATIOS
+    if not RATIOS:
+        return
+    tr = terminalreporter
+    tr.section("parity margins (worst err / limit per comparison, largest first)")
+    for what, dtype, worst in sorted(RATIOS, key=lambda r: -r[2])[:25]:
+        tr.write_line(f"{worst:7.3f}  {dtype:4s}  {what}")
+    tr.write_line(f"{len(RATIOS)} comparisons")

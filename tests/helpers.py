@@ -2,9 +2,7 @@
 
 Tolerances (written once, used everywhere):
   fp32 storage:  |x - y| <= 1e-5 |y| + 1e-5 RMS(y), elementwise
-  bf16 storage:  |x - y| <= 2e-2 RMS(y) + 2^-8 |y|, elementwise: the first term is the
-                 2e-2 x RMS bound, the second the rounding of the bf16 output itself (half a
-                 bf16 ulp is at most 2^-8 |y|), which no implementation storing bf16 avoids
+  bf16 storage:  max |x - y| <= 2e-2 RMS(y)
   RMS(y) is taken per output vector: one head's v_head outputs for one query, or one
   token's d_model outputs after W_O (a t = 0 prefill row is ~N(0,1) while late rows are
   averages ~10x smaller, so one RMS over all rows would sit below the bf16 rounding of the
@@ -23,7 +21,6 @@ import torch
 
 FP32_REL = 1e-5
 BF16_RMS = 2e-2
-BF16_OUT_ROUND = 2.0 ** -8
 CACHE_ABS_RMS = 2.0 ** -16
 CACHE_EXACT_FRAC = 0.99
 
@@ -37,6 +34,11 @@ def np64(t) -> np.ndarray:
 def rms(y) -> float:
     y = np64(y)
     return float(np.sqrt(np.mean(y * y))) if y.size else 0.0
+
+
+# (what, dtype, worst err/limit) of every comparison made in this process; the session summary
+# prints the closest ones (conftest.py)
+RATIOS: list = []
 
 
 def assert_close(x, y, dtype: str, what: str = "") -> dict:
@@ -53,9 +55,10 @@ def assert_close(x, y, dtype: str, what: str = "") -> dict:
     if dtype == "f32":
         lim = FP32_REL * np.abs(y2) + FP32_REL * r
     else:
-        lim = BF16_RMS * r + BF16_OUT_ROUND * np.abs(y2)
+        lim = np.broadcast_to(BF16_RMS * r, err.shape)
     bad = err > lim
     worst = float(np.max(err / np.maximum(lim, 1e-300)))
+    RATIOS.append((what, dtype, worst))
     assert not bad.any(), (f"{what}: {int(bad.sum())} of {err.size} elements over the {dtype} tolerance; "
                            f"worst err/limit {worst:.3f}, max err {err.max():.3e}")
     return {"max_err": float(err.max()), "worst_ratio": worst}

@@ -78,3 +78,17 @@ def test_traffic_figure_is_dropped_when_the_kernel_source_changed(tmp_path, monk
     src.write_text("kernel v2")
     assert bench.traffic_for("tc_x") is None
     assert bench.traffic_for("tc_other") is None
+
+
+def test_cpu_baseline_runs_the_oracle_on_several_threads():
+    """The CPU baseline's host logic: a fixed number of seeded units spread over two threads,
+    each through the oracle, throughput scaled from the units to the full step."""
+    w = workloads.shrink(workloads.WORKLOADS["v3_decode_b32_ctx4096"], B=2, ctx=64)
+    inp = workloads.make_inputs(w)
+    r = bench.time_oracle_units(w, inp, 0.0, min_units=6, max_units=6, threads=2)
+    assert r["cores"] == 2 and r["kind"] == "oracle" and r["value"] > 0
+    assert r["sample"].startswith("6 seeded (sequence, head) units")
+    # a unit over its first 16 rows counts as 64 / 16 of a full unit
+    s = bench.time_oracle_units(w, inp, 0.0, min_units=3, max_units=3, tokens=16)
+    assert s["cores"] == 1 and "first 16 rows" in s["sample"]
+    assert bench.host_cores() >= 1
