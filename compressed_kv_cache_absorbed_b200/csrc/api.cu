@@ -414,8 +414,8 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (tc_path) {
         e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
                                         (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                        (const bf16*)cache, cache_rows, offsets, nullptr, nullptr, 0, B, scale_of(d),
-                                        (bf16*)o_dst,
+                                        (const bf16*)cache, cache_rows, offsets, nullptr, nullptr, 0, B, 1, true,
+                                        scale_of(d), (bf16*)o_dst,
                                         ws.tc, num_sms(), err.code, err.detail, s);
     } else {
         e = decode_simt<T>(d, w, qn, sQn_b, sQn_h, qr, sQr_b, sQr_h, (const T*)cache, cache_rows, offsets, B,
@@ -522,7 +522,7 @@ extern "C" mla_status mla_decode_absorbed_paged(const mla_dims* d, mla_weights w
     cudaError_t e = mla::tc::decode_absorbed_tc(
         (const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope, H * d->d_hR, d->d_hR,
         (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, (const bf16*)cache, rows, nullptr, seq_lens,
-        block_table, max_blocks, B, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, s);
+        block_table, max_blocks, B, 1, true, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged");
 }
 
@@ -545,6 +545,12 @@ static MultiWs carve_multi(const mla_dims* d, int B, int q_len, int max_blocks, 
     m.vlen = (int32_t*)c.take((size_t)B * q_len * sizeof(int32_t));
     m.bytes = head + c.used;
     return m;
+}
+
+// Sibling clusters for a few new tokens per sequence, while at least two cost ranges remain;
+// longer chunks expand into per-token sequences.
+static bool multi_siblings(int q_len) {
+    return q_len <= 8 && mla::tc::decode_clusters(num_sms()) / q_len >= 2;
 }
 
 static bool multi_sizes_ok(int32_t B, int32_t q_len, int32_t max_blocks) {
@@ -581,16 +587,31 @@ extern "C" mla_status mla_decode_absorbed_paged_multi(const mla_dims* d, mla_wei
     if ((st = dev_err(&err)) != MLA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     cudaError_t e;
+    const long long H = d->H;
+    if (multi_siblings(q_len)) {
+        // a few new tokens per sequence (draft verification): the q_len queries of a sequence
+        // run on sibling clusters that walk the same tiles together, so each cache tile
+        // streams from HBM once
+        e = mla::tc::decode_absorbed_tc((const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope,
+                                        H * d->d_hR, d->d_hR, (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
+                                        (const bf16*)cache, rows, nullptr, seq_lens, block_table, max_blocks, B,
+                                        q_len, false, scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code,
+                                        err.detail, s);
+        return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged_multi");
+    }
+    // a long chunk of new tokens (chunked prefill): every token becomes a query sequence of
+    // its own on its parent's pages, cut at its own row; consecutive tokens of a sequence run
+    // on neighbouring clusters at the same time, and the prefix stays in L2 (loads without the
+    // evict-first hint)
     {
         mla::ProfScope ps(s, "multi_token_views");
         e = mla::expand_multi_token(block_table, seq_lens, B, q_len, max_blocks, ws.vbt, ws.vlen, s);
     }
     if (e != cudaSuccess) return cuda_fail(e, "mla_decode_absorbed_paged_multi");
-    const long long H = d->H;
     e = mla::tc::decode_absorbed_tc((const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope,
                                     H * d->d_hR, d->d_hR, (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                    (const bf16*)cache, rows, nullptr, ws.vlen, ws.vbt, max_blocks, B * q_len,
-                                    scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code, err.detail, s);
+                                    (const bf16*)cache, rows, nullptr, ws.vlen, ws.vbt, max_blocks, B * q_len, 1,
+                                    false, scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code, err.detail, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged_multi");
 }
 

@@ -105,8 +105,10 @@ __device__ __forceinline__ float ex2_ftz(float x) {
     return y;
 }
 
+// A piece of work: tiles [j0, j1) of parent sequence b (whose rows start at row0 or sit in
+// b's pages) for query v, which attends to the first L of b's rows.
 struct Seg {
-    int b, j0, j1, L, slot;
+    int b, v, j0, j1, L, slot;
     long long row0;
 };
 
@@ -141,16 +143,26 @@ struct SeqSrc {
 
 // Walks the pieces of sequences in this cluster's cost range [lo, hi), in sequence order,
 // starting from the sequence whose cost region holds lo (cost start cs).  The same walk runs
-// in every role of both CTAs.  Partial slots: a piece that starts at its sequence's first
-// tile takes slot b; the one piece of a cluster that continues a sequence begun in an
-// earlier cluster takes slot B + cluster.  So B + clusters slots suffice.
+// in every role of both CTAs.
+//
+// Sibling queries.  With Q > 1, each sequence b carries Q queries (the last Q rows of b are
+// new tokens; query v = b Q + t attends to the first len(b) - (Q - 1 - t) rows).  The
+// clusters form groups of Q siblings: cluster c takes cost range c / Q of the sequences and
+// query t = c % Q, so the Q siblings walk the same tiles at the same time and the cache
+// streams from HBM once while L2 serves the other Q - 1 reads.  Costs are counted on the
+// sequences, so all siblings get the same ranges; a sibling whose query ends earlier skips
+// the tiles past its end.
+//
+// Partial slots: a piece that starts at its query's first tile takes slot v; the one piece
+// of a cluster that continues a query begun in an earlier range takes slot B Q + cluster.
+// So B Q + clusters slots suffice.
 struct SegIter {
     SeqSrc src;
     int B, lo, hi, cluster, b, cs;
+    int Q, t;
     __device__ bool next(Seg& s) {
         while (b < B && cs < hi) {
-            const int Lraw = src.len(b);
-            const int L = Lraw > 0 ? Lraw : 0;
+            const int L = src.len(b);
             const long long r0 = src.row0(b);
             const int n = tiles_of_len(L);
             const int f = cs + kPieceCost;   // cost position of tile 0
@@ -158,15 +170,18 @@ struct SegIter {
             ++b;
             cs += cost_of_tiles(n);
             if (n == 0) continue;
+            const int Lt = L - (Q - 1 - t);    // rows this query attends to
+            const int nt = tiles_of_len(Lt);
             const int j0 = lo > f ? lo - f : 0;
-            const int j1 = hi - f < n ? hi - f : n;
+            const int j1 = hi - f < nt ? hi - f : nt;
             if (j0 < j1) {
                 s.b = bb;
+                s.v = bb * Q + t;
                 s.j0 = j0;
                 s.j1 = j1;
                 s.row0 = r0;
-                s.L = L;
-                s.slot = j0 == 0 ? bb : B + cluster;
+                s.L = Lt;
+                s.slot = j0 == 0 ? s.v : B * Q + cluster;
                 return true;
             }
         }
@@ -183,7 +198,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_rope,
                  const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
-                 const SeqSrc src, int B, long long cache_rows,
+                 const SeqSrc src, int B, int Q, int stream_once, long long cache_rows,
                  float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
@@ -290,8 +305,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         for (int i = 0; i < kWarps; ++i) total += plan_wsum[i];
         __syncthreads();
     }
-    const int per = total > 0 ? (total + P - 1) / P : 1;
-    const int lo = cluster * per, hi = min(total, lo + per);
+    // Q sibling clusters per cost range (one per query of a sequence); clusters past the
+    // last full group of Q have no range
+    const int R = P / Q, range = cluster / Q, tok = cluster % Q;
+    const int per = total > 0 ? (total + R - 1) / R : 1;
+    const int lo = range < R ? range * per : total, hi = min(total, lo + per);
     if (lo < total) {
         int carry = 0;
         for (int c0 = 0; c0 < B; c0 += kThreads) {
@@ -324,7 +342,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             __syncthreads();
         }
     }
-    SegIter it{src, B, lo, hi, cluster, plan_first[0], plan_first[1]};
+    SegIter it{src, B, lo, hi, cluster, plan_first[0], plan_first[1], Q, tok};
     Seg sg;
 
     if (warp == 0) {
@@ -332,8 +350,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         if (lane == 0) {
             ptx::tma_prefetch(&tm_cache);
             ptx::tma_prefetch(&tm_rope);
-            // the cache is streamed once: let L2 drop it first, keeping the partials and weights
-            const uint64_t stream_policy = ptx::policy_evict_first();
+            // a cache read once is let go from L2 first, keeping the partials and weights; with
+            // sibling queries (or other calls' queries) reading the same tiles it is kept
+            const uint64_t stream_policy = stream_once ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             uint32_t g = 0;
             while (!*abort_flag && it.next(sg)) {
                 for (int j = sg.j0; j < sg.j1; ++j, ++g) {
@@ -491,10 +510,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         uint32_t g = 0;
         if (sender) {
             // ------------------------------------------------------- score senders
-            // Q_r of sequence b: 256 latent columns of this head -> TMEM, 32 rotary columns -> smem
-            auto load_q = [&](int b) {
-                const uint4* ql = (const uint4*)(q_lat + ((long long)b * 128 + h) * 512 + 256 * rank);
-                const uint4* qr = (const uint4*)(q_rope + b * sQr_b + h * sQr_h + 32 * rank);
+            // Q_r of query v: 256 latent columns of this head -> TMEM, 32 rotary columns -> smem
+            auto load_q = [&](int v) {
+                const uint4* ql = (const uint4*)(q_lat + ((long long)v * 128 + h) * 512 + 256 * rank);
+                const uint4* qr = (const uint4*)(q_rope + v * sQr_b + h * sQr_h + 32 * rank);
 #pragma unroll
                 for (int c = 0; c < 4; ++c) {
                     uint32_t r[32];
@@ -514,7 +533,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                 ptx::mbar_arrive(q_ready);
             };
             pdl_wait();   // q_lat is written by the previous kernel of this call
-            if (have) load_q(cur.b);
+            if (have) load_q(cur.v);
             while (have) {
                 const uint32_t b = g & 1, u = g >> 1;
                 // partial scores: TMEM -> registers -> bf16 pairs
@@ -558,7 +577,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     have = it.next(cur);
                     if (have) {
                         j = cur.j0;
-                        load_q(cur.b);   // the S of this piece's last tile is already read
+                        load_q(cur.v);   // the S of this piece's last tile is already read
                     }
                 }
             }
@@ -724,9 +743,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 }
 
 // ------------------------------------------------------------- merge + W_UV
-// o[b,h,:] = W_UV[h] o_lat[b,h,:],  o_lat[b,h,c] = sum_p 2^(m_p - M) O_p[h,c] / sum_p 2^(m_p - M) l_p
-// over the pieces p of sequence b (M = max_p m_p; an empty sequence gives o = 0).
-// One CTA per (head h, block of BN sequences).  Thread 0 starts the bulk loads of the tiled
+// o[v,h,:] = W_UV[h] o_lat[v,h,:],  o_lat[v,h,c] = sum_p 2^(m_p - M) O_p[h,c] / sum_p 2^(m_p - M) l_p
+// over the pieces p of query v (M = max_p m_p; a query with no row gives o = 0); query v is
+// query v % Q of sequence v / Q.  One CTA per (head h, block of BN queries).  Thread 0 starts the bulk loads of the tiled
 // W_UV[h] (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
 // then merge the partials of their rows (warp per row, lane per 16 columns) straight into
 // the B operand in shared memory (K-major, 128-byte swizzle, as TMA would lay it out);
@@ -739,7 +758,7 @@ constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
 template <int BN>
 __global__ void __launch_bounds__(kMergeThreads, 1)
-merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B,
+merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B, int Q,
                  const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
@@ -768,9 +787,9 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         ptx::tmem_relinquish();
     }
     if (threadIdx.x == 0) pdl_trigger();
-    // The split of the decode kernel (same cost model, same cluster count), recomputed from
-    // the offsets before waiting for that kernel: cost positions of the first and one past
-    // the last tile of this CTA's sequences.
+    // The split of the decode kernel (same cost model, same cluster count, same sibling
+    // groups), recomputed from the sequence lengths before waiting for that kernel: cost
+    // positions of the first and one past the last tile of this CTA's queries.
     __shared__ int s_wsum[kMergeThreads / 32];
     __shared__ int s_pos[2][BN];
     constexpr int kW = kMergeThreads / 32;
@@ -786,10 +805,12 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         for (int i = 0; i < kW; ++i) total += s_wsum[i];
         __syncthreads();
     }
-    const int per = total > 0 ? (total + P - 1) / P : 1;
+    const int R = P / Q;
+    const int per = total > 0 ? (total + R - 1) / R : 1;
+    const int NV = B * Q;   // queries
     {
         int carry = 0;
-        for (int c0 = 0; c0 < B && c0 < n0 + BN; c0 += kMergeThreads) {
+        for (int c0 = 0; c0 < B && c0 * Q < n0 + BN; c0 += kMergeThreads) {
             const int b = c0 + (int)threadIdx.x;
             const int nt = b < B ? tiles_of_len(src.len(b)) : 0;
             const int cb = cost_of_tiles(nt);
@@ -809,9 +830,19 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
                 chunk += v;
             }
             const int cs = before + incl - cb;
-            if (b < B && b >= n0 && b < n0 + BN) {
-                s_pos[0][b - n0] = cs + kPieceCost;
-                s_pos[1][b - n0] = cs + kPieceCost + nt;
+            if (b < B && nt > 0) {
+                for (int t = 0; t < Q; ++t) {
+                    const int v = b * Q + t;
+                    if (v >= n0 && v < n0 + BN) {
+                        s_pos[0][v - n0] = cs + kPieceCost;
+                        s_pos[1][v - n0] = cs + kPieceCost + tiles_of_len(src.len(b) - (Q - 1 - t));
+                    }
+                }
+            } else if (b < B) {
+                for (int t = 0; t < Q; ++t) {
+                    const int v = b * Q + t;
+                    if (v >= n0 && v < n0 + BN) s_pos[0][v - n0] = s_pos[1][v - n0] = 0;
+                }
             }
             carry += chunk;
             __syncthreads();
@@ -823,23 +854,24 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
     int t0r[kRowsPerWarp], t1r[kRowsPerWarp];
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int b = n0 + warp + kW * i;
-        t0r[i] = b < B ? s_pos[0][warp + kW * i] : 0;
-        t1r[i] = b < B ? s_pos[1][warp + kW * i] : 0;
+        const int v = n0 + warp + kW * i;
+        t0r[i] = v < NV ? s_pos[0][warp + kW * i] : 0;
+        t1r[i] = v < NV ? s_pos[1][warp + kW * i] : 0;
     }
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int r = warp + kW * i, b = n0 + r;
+        const int r = warp + kW * i, v = n0 + r, tq = v % Q;
         const int t0 = t0r[i], t1 = t1r[i];
         float acc[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) acc[k] = 0.f;
         if (t1 > t0) {
-            // piece 0 (from cluster t0 / per) is in slot b; piece p > 0 continues the
-            // sequence in cluster t0 / per + p and is in slot B + t0 / per + p
+            // piece 0 (from range t0 / per) is in slot v; piece p > 0 continues the query in
+            // range t0 / per + p, i.e. in sibling cluster (t0 / per + p) Q + tq, and is in slot
+            // NV + that cluster
             const int cfirst = t0 / per;
             const int np = (t1 - 1) / per - cfirst + 1;
-            auto slot_of = [&](int p) -> long long { return p == 0 ? b : B + cfirst + p; };
+            auto slot_of = [&](int p) -> long long { return p == 0 ? v : NV + (long long)(cfirst + p) * Q + tq; };
             // (m, l) of up to 32 pieces (lane p) and the first 4 pieces' partial rows are
             // requested together; the weights need the maximum, the loads do not
             float2 ml = lane < np ? *(const float2*)(part_ml + (slot_of(lane) * 128 + h) * 2)
@@ -945,8 +977,8 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         }
         ptx::named_barrier_sync(1, 128);   // the four epilogue warps
         for (int i = threadIdx.x; i < BN * 16; i += 128) {
-            const int b = n0 + (i >> 4);
-            if (b < B) ((uint4*)(o + b * sO_b + h * sO_h))[i & 15] = ((const uint4*)sA)[i];
+            const int v = n0 + (i >> 4);
+            if (v < NV) ((uint4*)(o + v * sO_b + h * sO_h))[i & 15] = ((const uint4*)sA)[i];
         }
     }
     (void)ok;
@@ -1118,6 +1150,8 @@ int max_clusters(int num_sms) {
 
 }  // namespace
 
+int decode_clusters(int num_sms) { return max_clusters(num_sms); }
+
 cudaError_t set_wait_limit_decode(uint32_t polls) { return ptx::set_wait_limit_of_this_file(polls); }
 
 cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
@@ -1155,7 +1189,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
                                long long sQr_b, long long sQr_h, const __nv_bfloat16* ukt,
                                const __nv_bfloat16* uv, const __nv_bfloat16* cache, long long cache_rows,
                                const int32_t* offsets, const int32_t* seq_lens, const int32_t* block_table,
-                               int bt_stride, int B, float scale, __nv_bfloat16* o, const DecodeWs& ws,
+                               int bt_stride, int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms,
                                int* err_code, long long* err_detail, cudaStream_t s) {
     if (B <= 0) return cudaSuccess;
@@ -1164,18 +1198,20 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     if (block_table && (!seq_lens || bt_stride <= 0)) return cudaErrorInvalidValue;
     const SeqSrc seqs{offsets, seq_lens, block_table, bt_stride, cache_rows};
     const int P = max_clusters(num_sms);
+    if (Q < 1 || Q > P) return cudaErrorInvalidValue;
+    const int NV = B * Q;   // queries
     {
-        // q_lat[b,h,:] = W_UK[h]^T q_nope[b,h,:]
+        // q_lat[v,h,:] = W_UK[h]^T q_nope[v,h,:]
         ProfScope ps(s, "tc_q_absorb");
         CUtensorMap mq;
-        const int BN = B <= 32 ? 32 : B <= 64 ? 64 : 128;
-        const uint64_t dq[3] = {128, (uint64_t)B, 128};
+        const int BN = NV <= 32 ? 32 : NV <= 64 ? 64 : 128;
+        const uint64_t dq[3] = {128, (uint64_t)NV, 128};
         const uint64_t sq[2] = {(uint64_t)sQn_b * 2, (uint64_t)sQn_h * 2};
         const uint32_t bq[3] = {64, (uint32_t)BN, 1};
         if (!make_tmap_bf16(&mq, qn, 3, dq, sq, bq)) return cudaErrorInvalidValue;
-        e = BN == 32   ? launch_absorb<32>(ukt, mq, B, ws.q_lat, err_code, err_detail, s)
-            : BN == 64 ? launch_absorb<64>(ukt, mq, B, ws.q_lat, err_code, err_detail, s)
-                       : launch_absorb<128>(ukt, mq, B, ws.q_lat, err_code, err_detail, s);
+        e = BN == 32   ? launch_absorb<32>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s)
+            : BN == 64 ? launch_absorb<64>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s)
+                       : launch_absorb<128>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s);
         if (e != cudaSuccess) return e;
     }
     {
@@ -1191,25 +1227,26 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
         if (attr != cudaSuccess) return attr;
         if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
-                            seqs, B, (long long)cache_rows, scale * 1.4426950408889634f,
+                            seqs, B, Q, (int)(stream_once ? 1 : 0), (long long)cache_rows,
+                            scale * 1.4426950408889634f,
                             ws.part_o, ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code,
                             err_detail)) != cudaSuccess)
             return e;
     }
     {
-        // merge of the pieces fused with o[b,h,:] = W_UV[h] o_lat[b,h,:]
+        // merge of the pieces fused with o[v,h,:] = W_UV[h] o_lat[v,h,:]
         ProfScope ps(s, "tc_merge_w_uv");
-        if (B <= 32) {
+        if (NV <= 32) {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
             if (attr != cudaSuccess) return attr;
             e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                           seqs, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+                           seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         } else {
             static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
             if (attr != cudaSuccess) return attr;
-            e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (B + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                           uv, seqs, P, B, (const float*)ws.part_o, (const float*)ws.part_ml, o,
+            e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
+                           uv, seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o,
                            128LL * 128, 128LL, err_code, err_detail);
         }
     }

@@ -41,18 +41,26 @@ constexpr size_t kTiledWeightBytes = (size_t)kH * kDc * 128 * 2;
 cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
                             __nv_bfloat16* uv, cudaStream_t s);
 
-// q_nope rows at qn + b*sQn_b + h*sQn_h (qk_nope = 128), q_rope rows at qr + b*sQr_b + h*sQr_h.
-// ukt / uv: the tiled weights written by tile_weights_tc; out o [B, H, 128] bf16.
+// Q queries per sequence (Q = 1: decode; Q > 1: the last Q rows of each sequence are new
+// tokens and query v = b Q + t attends to the first len(b) - (Q - 1 - t) rows).
+// q_nope rows at qn + v*sQn_b + h*sQn_h (qk_nope = 128), q_rope rows at qr + v*sQr_b + h*sQr_h.
+// ukt / uv: the tiled weights written by tile_weights_tc; out o [B * Q, H, 128] bf16.
 // Sequence b's cache rows are [offsets[b], offsets[b+1]) when block_table is null; with a
 // block table (paged cache, 64-token pages) sequence b has seq_lens[b] tokens and its tile j
 // is page block_table[b * bt_stride + j] (rows 64 page .. 64 page + 63).
+// stream_once: the call reads each cache tile once (loads carry an L2 evict-first hint);
+// pass false when other queries of the call read the same tiles.  1 <= Q <= the cluster
+// count; the workspace is that of B * Q queries.
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
                                const __nv_bfloat16* ukt, const __nv_bfloat16* uv,
                                const __nv_bfloat16* cache, long long cache_rows, const int32_t* offsets,
                                const int32_t* seq_lens, const int32_t* block_table, int bt_stride,
-                               int B, float scale, __nv_bfloat16* o, const DecodeWs& ws, int num_sms,
-                               int* err_code, long long* err_detail, cudaStream_t s);
+                               int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
+                               int num_sms, int* err_code, long long* err_detail, cudaStream_t s);
+
+// Clusters of the decode kernel on this device (sibling groups are formed from these).
+int decode_clusters(int num_sms);
 
 // Sets the polls a bounded wait of this file's kernels makes before giving up (current device).
 cudaError_t set_wait_limit_decode(uint32_t polls);

@@ -1,8 +1,8 @@
-// Multi-token decode over a paged latent cache: per-token views of the pages (the
-// verification step of speculative decoding, several draft tokens per sequence; the
-// DeepSeek pages name the multi-token-prediction module's use for it).  Each new token
+// Multi-token decode over a paged latent cache, for long chunks of new tokens (an absorbed
+// chunked prefill over a cached prefix): per-token views of the pages.  Each new token
 // becomes a sequence of its own that shares its parent's pages and stops at the token's own
-// row, so the paged absorbed decode runs on them unchanged.
+// row, so the paged absorbed decode runs on them unchanged.  (A few new tokens per sequence,
+// as in draft verification, run on sibling clusters instead, without these views.)
 #include "multi.cuh"
 
 namespace mla {

@@ -191,8 +191,12 @@ mla_status mla_decode_absorbed_paged(const mla_dims* dims, mla_weights w, const 
  * seq_lens[b] - q_len + t + 1 tokens; a token with no key (seq_lens[b] < q_len - t) gets
  * zeros.  Tensor-core shape only and handles without W_O, else MLA_ERR_UNSUPPORTED; a page
  * outside [0, num_pages) or more than max_blocks blocks latch MLA_ERR_OUT_OF_RANGE on the
- * device, as for mla_decode_absorbed_paged.  Each new token streams its own keys: the cache bytes read are q_len times those
- * of one decode step.
+ * device, as for mla_decode_absorbed_paged.
+ * Up to 8 new tokens per sequence run on sibling groups of clusters that walk the same cache
+ * tiles at the same time, so the cache streams from HBM once per call (the siblings' reads
+ * are served by L2); longer chunks (chunked prefill) make every new token a query sequence
+ * of its own, and the prefix tiles, read by neighbouring clusters at the same time, are
+ * served from L2 after their first read.
  * Workspace: device, >= mla_decode_multi_workspace_size(dims, B, q_len, max_blocks) bytes,
  * 256-byte aligned, contents on entry do not matter. */
 mla_status mla_decode_absorbed_paged_multi(const mla_dims* dims, mla_weights w, const void* q_nope,
@@ -235,7 +239,10 @@ mla_status mla_decode_absorbed_host(const mla_dims* dims, mla_weights w, const v
  *     MLA_NOALLOC_SCRATCH_BYTES returns MLA_ERR_WORKSPACE before launching anything
  *     (compare the two to know in advance whether a batch fits).
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
- *     with that device current; make that first call before any stream capture.
+ *     with that device current; make that first call before any stream capture.  The
+ *     address is kept for the life of the process: a cudaDeviceReset in the same process
+ *     destroys the array with the rest of the library's device state, and the library must
+ *     not be called on that device afterwards.
  *   - All calls share the one array and it keeps the previous call's contents (nothing
  *     in it needs to start at zero).  Calls that overlap on the GPU (other streams,
  *     other host threads, without ordering between them) race on it and give wrong

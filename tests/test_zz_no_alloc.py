@@ -32,6 +32,13 @@ def test_noalloc_matches_the_workspace_entry_point(lengths):
     ws = mla.workspace(mla.mla_decode_workspace_size(dims, B))
     mla.mla_decode_absorbed(dims, weights, g["cache"], g["offsets"], ref, ws, q_nope=g["q_nope"],
                             q_rope=g["q_rope"])
+    # a larger, different batch first, so that its data is what the checked calls find left
+    # in the shared scratch
+    wb, ib = reduced_attn_inputs([2000] * 24, seed=29)
+    gb = {k: v.cuda() for k, v in ib.items()}
+    ob = torch.empty(wb.B, wb.H, wb.v_head, dtype=torch.bfloat16, device="cuda")
+    mla.mla_decode_absorbed_noalloc(dims, weights, gb["cache"], gb["offsets"], ob, q_nope=gb["q_nope"],
+                                    q_rope=gb["q_rope"])
     outs = []
     for _ in range(2):   # the second call finds the first call's data in the scratch
         o = torch.full((B, w.H, w.v_head), float("nan"), dtype=torch.bfloat16, device="cuda")
