@@ -55,6 +55,18 @@ def alg_step(w: workloads.Workload) -> dict:
             "attn_flops": flops_attn, "tokens": tokens}
 
 
+FP8_ROW_BYTES = 656   # E4M3 codes (512) + bf16 rotary key (128) + fp32 scale (4) + padding (12)
+
+
+def alg_step_fp8(w: workloads.Workload) -> dict:
+    """alg_step over FP8 cache rows: 656 bytes per token instead of 1152."""
+    a = alg_step(w)
+    cache = a["tokens"] * FP8_ROW_BYTES
+    a["bytes"] += cache - a["cache_bytes"]
+    a["cache_bytes"] = cache
+    return a
+
+
 def alg_multi(w: workloads.Workload) -> dict:
     """Bytes and flops of one multi-token decode step: each sequence's L + q_len rows read
     once, new token t attending to the first L + t + 1 of them."""
@@ -125,9 +137,9 @@ def alg_prefill(w: workloads.Workload) -> dict:
 
 def alg_kernel_bytes(name: str, w: workloads.Workload) -> int:
     """Algorithmic bytes of one launch of the kernel that dominates the step: the cache rows
-    it attends over (1152 B per token) plus the queries it reads."""
+    it attends over (1152 B per token, or 656 B for FP8 rows) plus the queries it reads."""
     L = workloads.lengths(w)
-    cache = int(L.sum()) * w.row * 2
+    cache = int(L.sum()) * (FP8_ROW_BYTES if name.endswith("_fp8") else w.row * 2)
     if name.startswith("tc_"):
         return cache + w.B * w.H * w.row * 2
     return cache + w.B * w.H * (w.d_c * 4 + w.d_hR * 2)
@@ -368,6 +380,19 @@ def build_step(w, inp, dev, mla):
                                     q_rope=g["q_rope"])
         h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
         return g, dims, weights, out, step, h2d, alg_step(w), w.B
+    if w.kind == "decode_fp8":
+        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
+        out = torch.empty(w.B, w.H, w.v_head, dtype=dt, device=dev)
+        ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
+        # the cache in FP8 rows, quantised once before the timed steps
+        cache8 = torch.empty(g["cache"].shape[0], mla.mla_fp8_row_bytes(dims), dtype=torch.uint8, device=dev)
+        mla.mla_quantize_cache_fp8(dims, g["cache"], cache8)
+        del g["cache"]
+
+        def step():
+            mla.mla_decode_absorbed_fp8(dims, weights, cache8, g["offsets"], out, ws, g["q_nope"], g["q_rope"])
+        h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
+        return g, dims, weights, out, step, h2d, alg_step_fp8(w), w.B
     if w.kind == "decode_multi":
         weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"])
         out = torch.empty(w.B, w.q_len, w.H, w.v_head, dtype=dt, device=dev)
@@ -529,7 +554,19 @@ def run_ours(args, w0):
         launches_per_step = sum(v[0] for v in prof.values()) / args.steps
         step_s = ms * 1e-3
         roof_s = max(a["bytes"] / (pk["hbm_gbs"] * 1e9), a["flops"] / (pk["bf16_tflops"] * 1e12))
-        if w.kind == "decode_attn":
+        if w.kind == "decode_fp8":
+            # FP8 rows halve the bytes: the attention kernel sits on the tensor side of the ridge
+            kflops = alg_kernel_flops(dom, w)
+            kbytes = alg_kernel_bytes(dom, w)
+            tf = kflops / launch_s / 1e12
+            roofline = {"kernel": dom, "bound": "tensor", "achieved": tf, "peak": pk["bf16_tflops"],
+                        "unit": "TFLOP/s", "frac": tf / pk["bf16_tflops"], "traffic": traffic_for(dom),
+                        "alg_flops_per_launch": kflops, "launch_us": launch_s * 1e6,
+                        "peak_source": f"{pk_kind} bf16_tflops (fp16 operands run at the bf16 rate)",
+                        "hbm_side": {"alg_bytes_per_launch": kbytes, "achieved_gbs": kbytes / launch_s / 1e9,
+                                     "frac": kbytes / launch_s / 1e9 / pk["hbm_gbs"]}}
+            metric, unit = "MLA decode tokens/s over an FP8 latent cache (H=128,d_c=512,ctx 4k)", "tokens/s"
+        elif w.kind == "decode_attn":
             kbytes = alg_kernel_bytes(dom, w)
             achieved = kbytes / launch_s / 1e9
             roofline = {"kernel": dom, "bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"],
@@ -583,7 +620,7 @@ def run_ours(args, w0):
             "cpu_baseline": cpu,
             "decode_path": "tcgen05" if mla.mla_decode_path(dims) == 1 else "cuda-core",
         }
-        if w.kind == "decode_attn":
+        if w.kind in ("decode_attn", "decode_fp8"):
             line["latent_cache_GBps"] = a["cache_bytes"] / step_s / 1e9
         print(json.dumps(line), flush=True)
     weights.close()

@@ -61,6 +61,13 @@ SIGNATURES = {
     "mla_decode_multi_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "mla_decode_absorbed_host": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P,
                                       ctypes.c_size_t, _P]),
+    "mla_fp8_row_bytes": (ctypes.c_int64, [_D]),
+    "mla_quantize_cache_fp8": (_S, [_D, _P, _P, ctypes.c_int32, _P, ctypes.c_int64, _P]),
+    "mla_append_fp8_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32]),
+    "mla_append_cache_fp8": (_S, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64, _P, ctypes.c_size_t,
+                                  _P]),
+    "mla_decode_absorbed_fp8": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t,
+                                     _P]),
     "mla_set_wait_limit": (_S, [ctypes.c_uint32]),
     "mla_test_starve_projection": (_S, [ctypes.c_int32]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
@@ -227,6 +234,39 @@ def mla_decode_absorbed_host(dims, weights: MLAWeights, cache, offsets, q_nope_h
     _check(_lib.mla_decode_absorbed_host(ctypes.byref(dims), weights.handle, _ptr(q_nope_host), _ptr(q_rope_host),
                                          _ptr(cache), cache.shape[0], _ptr(offsets), B, _ptr(out_host), _ptr(ws),
                                          ws.numel(), _stream(stream)), "mla_decode_absorbed_host")
+
+
+def mla_fp8_row_bytes(dims) -> int:
+    """Bytes of one FP8 cache row (-1 for shapes without FP8 rows)."""
+    return int(_lib.mla_fp8_row_bytes(ctypes.byref(dims)))
+
+
+def mla_quantize_cache_fp8(dims, rows, cache_fp8, slot=None, stream=None) -> None:
+    """FP8 rows of bf16 cache rows [n, d_c + d_hR] into cache_fp8 (uint8 [capacity, row bytes])
+    at slot (int64 [n], device) or at rows 0 .. n-1."""
+    _check(_lib.mla_quantize_cache_fp8(ctypes.byref(dims), _ptr(rows), _ptr(slot), rows.shape[0], _ptr(cache_fp8),
+                                       cache_fp8.shape[0], _stream(stream)), "mla_quantize_cache_fp8")
+
+
+def mla_append_fp8_workspace_size(dims, n: int) -> int:
+    return int(_lib.mla_append_fp8_workspace_size(ctypes.byref(dims), n))
+
+
+def mla_append_cache_fp8(dims, h, W_DKV, W_KR, pos, slot, cache_fp8, ws, stream=None) -> None:
+    """mla_append_cache into an FP8 cache (uint8 [capacity, row bytes])."""
+    n = h.shape[0]
+    _check(_lib.mla_append_cache_fp8(ctypes.byref(dims), _ptr(h), _ptr(W_DKV), _ptr(W_KR), _ptr(pos), _ptr(slot), n,
+                                     _ptr(cache_fp8), cache_fp8.shape[0], _ptr(ws), ws.numel(), _stream(stream)),
+           "mla_append_cache_fp8")
+
+
+def mla_decode_absorbed_fp8(dims, weights: MLAWeights, cache_fp8, offsets, out, ws, q_nope, q_rope,
+                            stream=None) -> None:
+    """mla_decode_absorbed over an FP8 cache (uint8 [rows, row bytes])."""
+    B = offsets.numel() - 1
+    _check(_lib.mla_decode_absorbed_fp8(ctypes.byref(dims), weights.handle, _ptr(q_nope), _ptr(q_rope),
+                                        _ptr(cache_fp8), cache_fp8.shape[0], _ptr(offsets), B, _ptr(out), _ptr(ws),
+                                        ws.numel(), _stream(stream)), "mla_decode_absorbed_fp8")
 
 
 def mla_prefill_causal(dims, weights: MLAWeights, h, W_DKV, W_KR, cache, out, ws, stream=None) -> None:

@@ -7,6 +7,7 @@
 
 #include "common.cuh"
 #include "decode_tc.cuh"
+#include "fp8.cuh"
 #include "gemm_tc.cuh"
 #include "multi.cuh"
 #include "prefill_tc.cuh"
@@ -414,7 +415,7 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     if (tc_path) {
         e = mla::tc::decode_absorbed_tc((const bf16*)qn, sQn_b, sQn_h, (const bf16*)qr, sQr_b, sQr_h,
                                         (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                        (const bf16*)cache, cache_rows, offsets, nullptr, nullptr, 0, B, 1, true,
+                                        cache, false, cache_rows, offsets, nullptr, nullptr, 0, B, 1, true,
                                         scale_of(d), (bf16*)o_dst,
                                         ws.tc, num_sms(), err.code, err.detail, s);
     } else {
@@ -521,7 +522,7 @@ extern "C" mla_status mla_decode_absorbed_paged(const mla_dims* d, mla_weights w
     const long long H = d->H;
     cudaError_t e = mla::tc::decode_absorbed_tc(
         (const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope, H * d->d_hR, d->d_hR,
-        (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, (const bf16*)cache, rows, nullptr, seq_lens,
+        (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, cache, false, rows, nullptr, seq_lens,
         block_table, max_blocks, B, 1, true, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged");
 }
@@ -594,7 +595,7 @@ extern "C" mla_status mla_decode_absorbed_paged_multi(const mla_dims* d, mla_wei
         // streams from HBM once
         e = mla::tc::decode_absorbed_tc((const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope,
                                         H * d->d_hR, d->d_hR, (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                        (const bf16*)cache, rows, nullptr, seq_lens, block_table, max_blocks, B,
+                                        cache, false, rows, nullptr, seq_lens, block_table, max_blocks, B,
                                         q_len, false, scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code,
                                         err.detail, s);
         return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged_multi");
@@ -610,9 +611,86 @@ extern "C" mla_status mla_decode_absorbed_paged_multi(const mla_dims* d, mla_wei
     if (e != cudaSuccess) return cuda_fail(e, "mla_decode_absorbed_paged_multi");
     e = mla::tc::decode_absorbed_tc((const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope,
                                     H * d->d_hR, d->d_hR, (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled,
-                                    (const bf16*)cache, rows, nullptr, ws.vlen, ws.vbt, max_blocks, B * q_len, 1,
+                                    cache, false, rows, nullptr, ws.vlen, ws.vbt, max_blocks, B * q_len, 1,
                                     false, scale_of(d), (bf16*)out, ws.dec.tc, num_sms(), err.code, err.detail, s);
     return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_paged_multi");
+}
+
+// -------------------------------------------------------------- FP8 latent cache
+
+extern "C" int64_t mla_fp8_row_bytes(const mla_dims* d) {
+    if (dims_supported(d) != MLA_OK || !tc_decode_ok(d)) return -1;
+    return mla::tc::kF8RowBytes;
+}
+
+extern "C" mla_status mla_quantize_cache_fp8(const mla_dims* d, const void* rows, const int64_t* slot, int32_t n,
+                                             void* cache_fp8, int64_t capacity, mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!tc_decode_ok(d)) return MLA_ERR_UNSUPPORTED;
+    if (n < 0 || capacity < 0) return MLA_ERR_INVALID_ARG;
+    if (n == 0) return MLA_OK;
+    if (!rows || !cache_fp8 || !aligned16(rows) || !aligned16(cache_fp8)) return MLA_ERR_INVALID_ARG;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaError_t e = mla::tc::quantize_rows_fp8((const bf16*)rows, slot, n, (uint8_t*)cache_fp8, capacity, err.code,
+                                               err.detail, (cudaStream_t)stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_quantize_cache_fp8");
+}
+
+extern "C" size_t mla_append_fp8_workspace_size(const mla_dims* d, int32_t n) {
+    if (dims_supported(d) != MLA_OK || !tc_decode_ok(d) || n < 0) return 0;
+    return ((size_t)n * (d->d_c + d->d_hR) * 2 + 255) & ~(size_t)255;
+}
+
+extern "C" mla_status mla_append_cache_fp8(const mla_dims* d, const void* h, const void* W_DKV, const void* W_KR,
+                                           const int32_t* pos, const int64_t* slot, int32_t n, void* cache_fp8,
+                                           int64_t capacity, void* workspace, size_t ws_bytes, mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!tc_decode_ok(d)) return MLA_ERR_UNSUPPORTED;
+    if (n < 0 || capacity < 0 || d->d_model <= 0) return MLA_ERR_INVALID_ARG;
+    if (n == 0) return MLA_OK;
+    if (!h || !W_DKV || !W_KR || !pos || !slot || !cache_fp8 || !aligned16(cache_fp8)) return MLA_ERR_INVALID_ARG;
+    if (!workspace || ws_bytes < mla_append_fp8_workspace_size(d, n) || ((uintptr_t)workspace & 255))
+        return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    // the bf16 rows of the n tokens into the workspace (rows 0 .. n-1, no slot scatter), then
+    // quantised into their slots
+    cudaError_t e = append_impl<bf16>(d, h, W_DKV, W_KR, pos, 1, nullptr, n, workspace, n, err, s);
+    if (e == cudaSuccess) {
+        mla::ProfScope ps(s, "fp8_quantize_rows");
+        e = mla::tc::quantize_rows_fp8((const bf16*)workspace, slot, n, (uint8_t*)cache_fp8, capacity, err.code,
+                                       err.detail, s);
+    }
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_append_cache_fp8");
+}
+
+extern "C" mla_status mla_decode_absorbed_fp8(const mla_dims* d, mla_weights w, const void* q_nope,
+                                              const void* q_rope, const void* cache_fp8, int64_t cache_rows,
+                                              const int32_t* offsets, int32_t B, void* out, void* workspace,
+                                              size_t ws_bytes, mla_stream_t stream) {
+    mla_status st = dims_supported(d);
+    if (st != MLA_OK) return st;
+    if (!w || B < 0) return MLA_ERR_INVALID_ARG;
+    if (memcmp(&w->dims, d, sizeof(mla_dims)) != 0) return MLA_ERR_INVALID_ARG;
+    if (!tc_decode_ok(d) || w->W_O) return MLA_ERR_UNSUPPORTED;
+    if (B == 0) return MLA_OK;
+    if (!q_nope || !q_rope || !cache_fp8 || !offsets || !out || cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL ||
+        !aligned16(cache_fp8))
+        return MLA_ERR_INVALID_ARG;
+    DecodeWs ws = carve_decode(d, B, workspace, true);
+    if (!workspace || ws_bytes < ws.bytes || ((uintptr_t)workspace & 255)) return MLA_ERR_WORKSPACE;
+    DevErr err;
+    if ((st = dev_err(&err)) != MLA_OK) return st;
+    const long long H = d->H;
+    cudaError_t e = mla::tc::decode_absorbed_tc(
+        (const bf16*)q_nope, H * d->qk_nope, d->qk_nope, (const bf16*)q_rope, H * d->d_hR, d->d_hR,
+        (const bf16*)w->ukt_tiled, (const bf16*)w->uv_tiled, cache_fp8, true, cache_rows, offsets, nullptr, nullptr, 0,
+        B, 1, true, scale_of(d), (bf16*)out, ws.tc, num_sms(), err.code, err.detail, (cudaStream_t)stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_decode_absorbed_fp8");
 }
 
 // ----------------------------------------------------------------------- prefill

@@ -49,7 +49,6 @@ namespace tc {
 namespace {
 
 constexpr int kT = 64;                        // tokens per tile
-constexpr int kStages = 4;
 constexpr int kChunkBytes = kT * 128;         // one 64-column latent box of a tile (128-byte swizzle)
 constexpr int kRopeBytes = kT * 64;           // this CTA's 32 rotary columns of a tile (64-byte swizzle)
 constexpr int kTileBytes = 4 * kChunkBytes + kRopeBytes;
@@ -57,14 +56,38 @@ constexpr int kQRopeBytes = 128 * 64;         // this CTA's 32 rotary query colu
 constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
 constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
 constexpr int kBarBytes = 256 + 2048 + 256;
-// tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer)
-// The dynamic shared memory of a kernel without static shared memory starts 1024-byte
-// aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
-constexpr int kSmem = kStages * kTileBytes + 4 * kXBytes + kQRopeBytes + kBarBytes;
-static_assert(kSmem <= 232448, "decode kernel shared memory over the 227 KB limit");
+// FP8 cache rows (see decode_tc.cuh): per tile and CTA, this CTA's 256 codes (two 128-byte
+// boxes, 128-byte swizzle), its 32 rotary columns (bf16, 64-byte swizzle) and the 64 rows'
+// 16-byte scale fields (the fp32 scale first)
+constexpr int kF8CodeBytes = kT * 128;
+constexpr int kF8StageBytes = 2 * kF8CodeBytes + kRopeBytes + kT * 16;
+static_assert(kF8StageBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment of the swizzled boxes");
+
+// Two variants of the kernel.  bf16 cache rows: TMA fills a ring of kStages tiles that the
+// MMAs read directly.  FP8 cache rows: TMA fills a ring of kF8Stages FP8 stages, and two
+// dequantisation warps turn each into an fp16 tile (code x scale) of the same layout in the
+// tile ring; the latent MMAs then run on fp16 operands (q_lat and P in fp16 too).
+template <bool kF8> struct DecCfg;
+template <> struct DecCfg<false> {
+    static constexpr int kStages = 4, kF8Stages = 0;
+    static constexpr int kThreads = 448;   // producer, MMA, 4 sender and 8 softmax warps
+};
+template <> struct DecCfg<true> {
+    static constexpr int kStages = 3, kF8Stages = 2;
+    static constexpr int kThreads = 512;   // + 2 dequantisation warps
+};
+// tiles, FP8 stages, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the
+// peer).  The dynamic shared memory of a kernel without static shared memory starts
+// 1024-byte aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
+template <bool kF8>
+constexpr int dec_smem() {
+    return DecCfg<kF8>::kStages * kTileBytes + DecCfg<kF8>::kF8Stages * kF8StageBytes + 4 * kXBytes + kQRopeBytes +
+           kBarBytes;
+}
+static_assert(dec_smem<false>() <= 232448, "decode kernel shared memory over the 227 KB limit");
+static_assert(dec_smem<true>() <= 232448, "FP8 decode kernel shared memory over the 227 KB limit");
 constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
-constexpr int kThreads = 448;                 // producer, MMA, 4 sender and 8 softmax warps
 
 // The work split counts cost units: one per tile plus kPieceCost for every sequence start
 // (a new piece costs its partial's epilogue and a query reload, measured at about three
@@ -194,14 +217,36 @@ __device__ __forceinline__ void fail(int* code, long long* detail, volatile int*
     *abort_flag = 1;
 }
 
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+// FP8 -> fp16 of 16 codes (one 16-byte unit), each times the row's scale (fp16)
+__device__ __forceinline__ void dequant16(const uint4 c, __half2 s, uint4& lo, uint4& hi) {
+    const uint32_t w[4] = {c.x, c.y, c.z, c.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint32_t a, b;
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(a) : "h"((unsigned short)(w[i] & 0xFFFFu)));
+        asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(b) : "h"((unsigned short)(w[i] >> 16)));
+        __half2 ha = __hmul2(*reinterpret_cast<__half2*>(&a), s);
+        __half2 hb = __hmul2(*reinterpret_cast<__half2*>(&b), s);
+        o[2 * i] = *reinterpret_cast<uint32_t*>(&ha);
+        o[2 * i + 1] = *reinterpret_cast<uint32_t*>(&hb);
+    }
+    lo = make_uint4(o[0], o[1], o[2], o[3]);
+    hi = make_uint4(o[4], o[5], o[6], o[7]);
+}
+
+template <bool kF8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DecCfg<kF8>::kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_rope,
+                 const __grid_constant__ CUtensorMap tm_scale,
                  const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const SeqSrc src, int B, int Q, int stream_once, long long cache_rows,
                  float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
+    constexpr int kStages = DecCfg<kF8>::kStages, kF8Stages = DecCfg<kF8>::kF8Stages;
+    constexpr int kThreads = DecCfg<kF8>::kThreads;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if (ptx::smem_u32(smem_raw) & 1023) {   // uniform across the CTA: leave before any sync
         if (threadIdx.x == 0) latch(DevErr{err_code, err_detail}, kErrTimeout, 7000000);
@@ -212,7 +257,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     const int len0 = threadIdx.x < B ? src.raw_len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
-    uint8_t* xbuf = smem + kStages * kTileBytes;   // [2] partial scores received from the peer
+    uint8_t* f8 = smem + kStages * kTileBytes;      // [kF8Stages] FP8 stages (FP8 cache rows)
+    uint8_t* xbuf = f8 + kF8Stages * kF8StageBytes; // [2] partial scores received from the peer
     uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
     uint8_t* qrope = xstage + 2 * kXBytes;         // rotary query columns (A operand, 64-byte swizzle)
     uint64_t* bars = (uint64_t*)(qrope + kQRopeBytes);
@@ -233,7 +279,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     uint64_t* xs_ready = s_full + 12;  // [2] all 128 rows of xstage[g & 1] written
     uint64_t* xs_free = s_full + 14;   // [2] the local softmax has read xstage[g & 1]
     uint64_t* pair_bar = s_full + 16;  // [4] the two softmax warps of a subpartition
-    float* pair_val = (float*)(s_full + 20);   // [2][2][128] values the two warps swap
+    uint64_t* f8_full = s_full + 20;   // [2] an FP8 stage landed (FP8 rows)
+    uint64_t* f8_empty = s_full + 22;  // [2] an FP8 stage was dequantised (FP8 rows)
+    float* pair_val = (float*)(s_full + 24);   // [2][2][128] values the two warps swap
     uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* plan_wsum = (int*)(tmem_slot + 2);   // [16] per-warp sums of the planning scans
@@ -245,8 +293,12 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < kStages; ++s) {
-            ptx::mbar_init(&tile_full[s], 1);
+            ptx::mbar_init(&tile_full[s], kF8 ? 64 : 1);   // the dequantisation warps, or TMA
             ptx::mbar_init(&tile_empty[s], 1);
+        }
+        for (int s = 0; s < kF8Stages; ++s) {
+            ptx::mbar_init(&f8_full[s], 1);
+            ptx::mbar_init(&f8_empty[s], 64);
         }
         ptx::mbar_init(s_full, 1);
         ptx::mbar_init(s_free, 128);
@@ -348,21 +400,29 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
+            // bf16 rows: the tile ring itself; FP8 rows: the FP8 stages the dequantisation
+            // warps read
+            constexpr int NR = kF8 ? kF8Stages : kStages;
+            constexpr int kRingBytes = kF8 ? kF8StageBytes : kTileBytes;
+            uint8_t* ring = kF8 ? f8 : tiles;
+            uint64_t* ring_full = kF8 ? f8_full : tile_full;
+            uint64_t* ring_empty = kF8 ? f8_empty : tile_empty;
             ptx::tma_prefetch(&tm_cache);
             ptx::tma_prefetch(&tm_rope);
+            if (kF8) ptx::tma_prefetch(&tm_scale);
             // a cache read once is let go from L2 first, keeping the partials and weights; with
             // sibling queries (or other calls' queries) reading the same tiles it is kept
             const uint64_t stream_policy = stream_once ? ptx::policy_evict_first() : ptx::policy_evict_normal();
             uint32_t g = 0;
             while (!*abort_flag && it.next(sg)) {
                 for (int j = sg.j0; j < sg.j1; ++j, ++g) {
-                    const int s = g % kStages;
-                    const uint32_t n = g / kStages;
-                    if (g >= (uint32_t)kStages && !ptx::mbar_wait(&tile_empty[s], (n - 1) & 1, abort_flag)) {
+                    const int s = g % NR;
+                    const uint32_t n = g / NR;
+                    if (g >= (uint32_t)NR && !ptx::mbar_wait(&ring_empty[s], (n - 1) & 1, abort_flag)) {
                         fail(err_code, err_detail, abort_flag, 1);
                         break;
                     }
-                    uint8_t* dst = tiles + s * kTileBytes;
+                    uint8_t* dst = ring + s * kRingBytes;
                     long long row_l = sg.row0 + (long long)j * kT;
                     if (src.block_table) {
                         const long long page = src.block_table[(long long)sg.b * src.bt_stride + j];
@@ -377,13 +437,26 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         }
                     }
                     const int row = (int)row_l;
-                    ptx::mbar_expect_tx(&tile_full[s], kTileBytes);
+                    ptx::mbar_expect_tx(&ring_full[s], kRingBytes);
+                    if (kF8) {
+                        // this CTA's 256 codes (bytes 256 rank ..), its 32 rotary columns (bf16
+                        // elements 256 + 32 rank ..) and the scale fields (fp32 element 160)
 #pragma unroll
-                    for (int i = 0; i < 4; ++i)
-                        ptx::tma_load_2d_hint(dst + i * kChunkBytes, &tm_cache, &tile_full[s], 256 * (int)rank + 64 * i,
+                        for (int i = 0; i < 2; ++i)
+                            ptx::tma_load_2d_hint(dst + i * kF8CodeBytes, &tm_cache, &ring_full[s],
+                                                  256 * (int)rank + 128 * i, row, stream_policy);
+                        ptx::tma_load_2d_hint(dst + 2 * kF8CodeBytes, &tm_rope, &ring_full[s], 256 + 32 * (int)rank,
                                               row, stream_policy);
-                    ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_rope, &tile_full[s], 512 + 32 * (int)rank, row,
-                                          stream_policy);
+                        ptx::tma_load_2d_hint(dst + 2 * kF8CodeBytes + kRopeBytes, &tm_scale, &ring_full[s], 160, row,
+                                              stream_policy);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            ptx::tma_load_2d_hint(dst + i * kChunkBytes, &tm_cache, &ring_full[s],
+                                                  256 * (int)rank + 64 * i, row, stream_policy);
+                        ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_rope, &ring_full[s], 512 + 32 * (int)rank,
+                                              row, stream_policy);
+                    }
                 }
             }
             // All tiles requested: pull this CTA's share of the next kernel's weights (W_UV)
@@ -397,16 +470,66 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     ptx::bulk_prefetch_l2(next_weights + o, (uint32_t)min(16384LL, e - o), keep);
             }
             // loads still in flight after an abort complete before the CTA leaves
-            for (uint32_t k = 0; k < (uint32_t)kStages && k < g; ++k) {
+            for (uint32_t k = 0; k < (uint32_t)NR && k < g; ++k) {
                 const uint32_t gg = g - 1 - k;
-                ptx::mbar_wait(&tile_full[gg % kStages], (gg / kStages) & 1, nullptr);
+                ptx::mbar_wait(&ring_full[gg % NR], (gg / NR) & 1, nullptr);
             }
         }
+    } else if (kF8 && warp >= 14) {
+        // ------------------------------------------------- FP8 dequantisation (FP8 rows)
+        // 64 threads turn FP8 stage g % kF8Stages into the fp16 tile g % kStages: every 16
+        // codes of a row (one 16-byte unit of a 128-byte-swizzled code box) times the row's
+        // scale become two 16-byte units of a 128-byte-swizzled fp16 latent box, and the
+        // rotary box (bf16, 64-byte swizzle) is copied as it is (same alignment, same
+        // swizzle pattern).
+        const int dt = threadIdx.x - 14 * 32;
+        uint32_t g = 0;
+        bool ok = true;
+        Seg cur;
+        while (ok && !*abort_flag && it.next(cur)) {
+            for (int j = cur.j0; j < cur.j1; ++j, ++g) {
+                const int s = g % kF8Stages, d = g % kStages;
+                if (!ptx::mbar_wait(&f8_full[s], (g / kF8Stages) & 1, abort_flag) ||
+                    (g >= (uint32_t)kStages && !ptx::mbar_wait(&tile_empty[d], ((g / kStages) - 1) & 1, abort_flag))) {
+                    ok = false;
+                    break;
+                }
+                const uint8_t* st = f8 + s * kF8StageBytes;
+                uint8_t* tl = tiles + d * kTileBytes;
+#pragma unroll 4
+                for (int k = 0; k < 16; ++k) {
+                    const int e = dt + 64 * k;          // 0 .. 1023: (row, code unit)
+                    const int r = e >> 4, u = e & 15;   // code box u >> 3, unit u & 7
+                    const int sw = r & 7;
+                    const uint4 c = *(const uint4*)(st + (u >> 3) * kF8CodeBytes + r * 128 + (((u & 7) ^ sw) << 4));
+                    const float sc = *(const float*)(st + 2 * kF8CodeBytes + kRopeBytes + r * 16);
+                    uint4 lo, hi;
+                    dequant16(c, __float2half2_rn(sc), lo, hi);
+                    // latent columns 16 u .. 16 u + 15 of this CTA: fp16 box u >> 2, units
+                    // 2 (u & 3) and 2 (u & 3) + 1
+                    uint8_t* rowp = tl + (u >> 2) * kChunkBytes + r * 128;
+                    const int a = 2 * (u & 3);
+                    *(uint4*)(rowp + ((a ^ sw) << 4)) = lo;
+                    *(uint4*)(rowp + (((a + 1) ^ sw) << 4)) = hi;
+                }
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int i = dt + 64 * k;   // 16-byte units of the 4 KB rotary box
+                    ((uint4*)(tl + 4 * kChunkBytes))[i] = ((const uint4*)(st + 2 * kF8CodeBytes))[i];
+                }
+                ptx::fence_proxy_async_smem();   // read by the tensor cores
+                ptx::mbar_arrive(&f8_empty[s]);
+                ptx::mbar_arrive(&tile_full[d]);
+            }
+        }
+        if (!ok) fail(err_code, err_detail, abort_flag, 6);
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, kT, 0, 0);
-            constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 256, 0, 1);
+            // the latent scores and P c: bf16 operands, or fp16 for FP8 rows; the rotary scores bf16
+            constexpr uint32_t idesc_s = kF8 ? ptx::idesc_f16_f32(128, kT, 0, 0) : ptx::idesc_bf16_f32(128, kT, 0, 0);
+            constexpr uint32_t idesc_sr = ptx::idesc_bf16_f32(128, kT, 0, 0);
+            constexpr uint32_t idesc_o = kF8 ? ptx::idesc_f16_f32(128, 256, 0, 1) : ptx::idesc_bf16_f32(128, 256, 0, 1);
             uint32_t g = 0, sidx = 0;
             bool ok = true;
             // Event-driven issue: O of the oldest tile as soon as its P is in TMEM (it frees the
@@ -465,7 +588,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 #pragma unroll
                         for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
                             ptx::mma_ss(tmem + kColS, ptx::desc_kmajor_sw64(ptx::smem_u32(qrope) + 32 * ks),
-                                        ptx::desc_kmajor_sw64(t + 4 * kChunkBytes + 32 * ks), idesc_s, 1);
+                                        ptx::desc_kmajor_sw64(t + 4 * kChunkBytes + 32 * ks), idesc_sr, 1);
                         ptx::mma_commit(s_full);
                         ++s_g;
                         q_ok = false;
@@ -654,7 +777,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     const float p0 = ex2_ftz(fmaf(s[i], scale_log2, -m_run));
                     const float p1 = ex2_ftz(fmaf(s[i + 1], scale_log2, -m_run));
                     sum += p0 + p1;
-                    pw[i / 2] = ptx::pack_bf16(p0, p1);
+                    pw[i / 2] = kF8 ? ptx::pack_f16(p0, p1) : ptx::pack_bf16(p0, p1);
                 }
                 l_run = l_run * alpha + sum;
                 const uint32_t pb = g & 1;
@@ -1032,7 +1155,9 @@ constexpr int kAbsorbTiles = 2;   // 128-row tiles of W_UK^T[h] per CTA (two CTA
 template <int BN>
 constexpr int absorb_smem() { return 2 * kAbsorbTiles * 16384 + 2 * BN * 128 + 1024 + 64; }
 
-template <int BN>
+// q_lat is stored as bf16, or (kF16) as fp16 saturated to +-65504 for the FP8-row decode,
+// whose latent MMAs run on fp16 operands.
+template <int BN, bool kF16>
 __global__ void __launch_bounds__(kAbsorbThreads, 1)
 absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ CUtensorMap tm_q, int B,
                 __nv_bfloat16* __restrict__ q_lat, int* err_code, long long* err_detail) {
@@ -1107,7 +1232,12 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
                 ptx::tmem_ld32(tmem + ((uint32_t)(warp * 32) << 16) + mt * BN + c0, r);
                 ptx::tmem_wait_ld();
 #pragma unroll
-                for (int j = 0; j < 32; ++j) stage[(c0 + j) * W + 128 * mt + m] = __float2bfloat16_rn(__uint_as_float(r[j]));
+                for (int j = 0; j < 32; ++j) {
+                    const float x = __uint_as_float(r[j]);
+                    stage[(c0 + j) * W + 128 * mt + m] =
+                        kF16 ? __ushort_as_bfloat16(__half_as_ushort(__float2half_rn(fminf(fmaxf(x, -65504.f), 65504.f))))
+                             : __float2bfloat16_rn(x);
+                }
             }
     }
     __syncthreads();
@@ -1120,32 +1250,47 @@ absorb_q_kernel(const __nv_bfloat16* __restrict__ ukt, const __grid_constant__ C
     if (warp == 1) ptx::tmem_dealloc(tmem, kCols);
 }
 
-template <int BN>
+template <int BN, bool kF16>
 cudaError_t launch_absorb(const __nv_bfloat16* ukt, const CUtensorMap& mq, int B, __nv_bfloat16* q_lat, int* err_code,
                           long long* err_detail, cudaStream_t s) {
-    static const cudaError_t attr = set_smem_attrs(absorb_q_kernel<BN>, absorb_smem<BN>());
+    static const cudaError_t attr = set_smem_attrs(absorb_q_kernel<BN, kF16>, absorb_smem<BN>());
     if (attr != cudaSuccess) return attr;
-    return launch_pdl(absorb_q_kernel<BN>, dim3(128 * (4 / kAbsorbTiles), (B + BN - 1) / BN), dim3(kAbsorbThreads),
-                      absorb_smem<BN>(), s,
-                      ukt, mq, B, q_lat, err_code, err_detail);
+    return launch_pdl(absorb_q_kernel<BN, kF16>, dim3(128 * (4 / kAbsorbTiles), (B + BN - 1) / BN),
+                      dim3(kAbsorbThreads), absorb_smem<BN>(), s, ukt, mq, B, q_lat, err_code, err_detail);
+}
+
+template <bool kF16>
+cudaError_t launch_absorb_any(int NV, const __nv_bfloat16* ukt, const CUtensorMap& mq, __nv_bfloat16* q_lat,
+                              int* err_code, long long* err_detail, cudaStream_t s) {
+    return NV <= 32   ? launch_absorb<32, kF16>(ukt, mq, NV, q_lat, err_code, err_detail, s)
+           : NV <= 64 ? launch_absorb<64, kF16>(ukt, mq, NV, q_lat, err_code, err_detail, s)
+                      : launch_absorb<128, kF16>(ukt, mq, NV, q_lat, err_code, err_detail, s);
 }
 
 int g_clusters_cached = 0;
 
-int max_clusters(int num_sms) {
-    if (g_clusters_cached > 0) return g_clusters_cached;
-    set_smem_attrs(decode_tc_kernel, kSmem);
+template <bool kF8>
+int resident_clusters(int num_sms) {
+    set_smem_attrs(decode_tc_kernel<kF8>, dec_smem<kF8>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
-    cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmem;
+    cfg.blockDim = dim3(DecCfg<kF8>::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = dec_smem<kF8>();
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<kF8>, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = num_sms / 2;
     }
-    g_clusters_cached = n;
     return n;
+}
+
+// Clusters of one decode launch: all resident at once, for both cache formats (the merge
+// kernel and the workspace size depend on this count only).
+int max_clusters(int num_sms) {
+    if (g_clusters_cached > 0) return g_clusters_cached;
+    const int a = resident_clusters<false>(num_sms), b = resident_clusters<true>(num_sms);
+    g_clusters_cached = a < b ? a : b;
+    return g_clusters_cached;
 }
 
 }  // namespace
@@ -1187,7 +1332,7 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
 
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h, const __nv_bfloat16* qr,
                                long long sQr_b, long long sQr_h, const __nv_bfloat16* ukt,
-                               const __nv_bfloat16* uv, const __nv_bfloat16* cache, long long cache_rows,
+                               const __nv_bfloat16* uv, const void* cache, bool fp8, long long cache_rows,
                                const int32_t* offsets, const int32_t* seq_lens, const int32_t* block_table,
                                int bt_stride, int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms,
@@ -1209,29 +1354,51 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         const uint64_t sq[2] = {(uint64_t)sQn_b * 2, (uint64_t)sQn_h * 2};
         const uint32_t bq[3] = {64, (uint32_t)BN, 1};
         if (!make_tmap_bf16(&mq, qn, 3, dq, sq, bq)) return cudaErrorInvalidValue;
-        e = BN == 32   ? launch_absorb<32>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s)
-            : BN == 64 ? launch_absorb<64>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s)
-                       : launch_absorb<128>(ukt, mq, NV, ws.q_lat, err_code, err_detail, s);
+        e = fp8 ? launch_absorb_any<true>(NV, ukt, mq, ws.q_lat, err_code, err_detail, s)
+                : launch_absorb_any<false>(NV, ukt, mq, ws.q_lat, err_code, err_detail, s);
         if (e != cudaSuccess) return e;
     }
     {
-        ProfScope ps(s, "tc_flash_decode");
-        CUtensorMap m, mr;
-        const uint64_t dims[2] = {576, (uint64_t)cache_rows};
-        const uint64_t strides[1] = {576 * 2};
-        const uint32_t box[2] = {64, (uint32_t)kT};
-        const uint32_t box_rope[2] = {32, (uint32_t)kT};
-        if (!make_tmap_bf16(&m, cache, 2, dims, strides, box) ||
-            !make_tmap_bf16(&mr, cache, 2, dims, strides, box_rope, 64))
-            return cudaErrorInvalidValue;
-        static const cudaError_t attr = set_smem_attrs(decode_tc_kernel, kSmem);
-        if (attr != cudaSuccess) return attr;
-        if ((e = launch_pdl(decode_tc_kernel, dim3(2 * P), dim3(kThreads), kSmem, s, m, mr, ws.q_lat, qr, sQr_b, sQr_h,
-                            seqs, B, Q, (int)(stream_once ? 1 : 0), (long long)cache_rows,
-                            scale * 1.4426950408889634f,
-                            ws.part_o, ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code,
-                            err_detail)) != cudaSuccess)
-            return e;
+        ProfScope ps(s, fp8 ? "tc_flash_decode_fp8" : "tc_flash_decode");
+        CUtensorMap m, mr, msc;
+        const float scale_log2 = scale * 1.4426950408889634f;
+        if (!fp8) {
+            const uint64_t dims[2] = {576, (uint64_t)cache_rows};
+            const uint64_t strides[1] = {576 * 2};
+            const uint32_t box[2] = {64, (uint32_t)kT};
+            const uint32_t box_rope[2] = {32, (uint32_t)kT};
+            if (!make_tmap_bf16(&m, cache, 2, dims, strides, box) ||
+                !make_tmap_bf16(&mr, cache, 2, dims, strides, box_rope, 64))
+                return cudaErrorInvalidValue;
+            msc = mr;   // unused
+            static const cudaError_t attr = set_smem_attrs(decode_tc_kernel<false>, dec_smem<false>());
+            if (attr != cudaSuccess) return attr;
+            e = launch_pdl(decode_tc_kernel<false>, dim3(2 * P), dim3(DecCfg<false>::kThreads), dec_smem<false>(), s,
+                           m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h, seqs, B, Q, (int)(stream_once ? 1 : 0),
+                           (long long)cache_rows, scale_log2, ws.part_o, ws.part_ml, (const uint8_t*)uv,
+                           (long long)kTiledWeightBytes, err_code, err_detail);
+        } else {
+            // FP8 rows of kF8RowBytes: codes as bytes, the rotary key as bf16 elements, the
+            // scale field as fp32 elements
+            const uint64_t sr[1] = {(uint64_t)kF8RowBytes};
+            const uint64_t dc[2] = {(uint64_t)kF8RowBytes, (uint64_t)cache_rows};
+            const uint32_t bc[2] = {128, (uint32_t)kT};
+            const uint64_t dr[2] = {(uint64_t)kF8RowBytes / 2, (uint64_t)cache_rows};
+            const uint32_t br[2] = {32, (uint32_t)kT};
+            const uint64_t ds[2] = {(uint64_t)kF8RowBytes / 4, (uint64_t)cache_rows};
+            const uint32_t bs[2] = {4, (uint32_t)kT};
+            if (!make_tmap(&m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, cache, 2, dc, sr, bc, 128) ||
+                !make_tmap(&mr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, 2, dr, sr, br, 64) ||
+                !make_tmap(&msc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cache, 2, ds, sr, bs, 0))
+                return cudaErrorInvalidValue;
+            static const cudaError_t attr = set_smem_attrs(decode_tc_kernel<true>, dec_smem<true>());
+            if (attr != cudaSuccess) return attr;
+            e = launch_pdl(decode_tc_kernel<true>, dim3(2 * P), dim3(DecCfg<true>::kThreads), dec_smem<true>(), s,
+                           m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h, seqs, B, Q, (int)(stream_once ? 1 : 0),
+                           (long long)cache_rows, scale_log2, ws.part_o, ws.part_ml, (const uint8_t*)uv,
+                           (long long)kTiledWeightBytes, err_code, err_detail);
+        }
+        if (e != cudaSuccess) return e;
     }
     {
         // merge of the pieces fused with o[v,h,:] = W_UV[h] o_lat[v,h,:]

@@ -17,6 +17,12 @@ constexpr int kRow = kDc + kDr;  // 576 cache elements per token
 constexpr int kPageTokens = 64;  // tokens per page of a paged cache (one decode tile)
 constexpr bool kEnabled = true;
 
+// An FP8 cache row: the latent c as d_c = 512 FP8 E4M3 codes (bytes 0 .. 511), the rotary key
+// as 64 bf16 (bytes 512 .. 639), the token's scale as fp32 (bytes 640 .. 643) and 12 bytes
+// of zero padding, so that rows stay 16-byte aligned: c = code x scale.
+constexpr int kF8RowBytes = 656;
+constexpr int kF8ScaleOffset = 640;
+
 // Workspace pieces of the tensor-core decode (all device memory, carved by the caller).
 struct DecodeWs {
     __nv_bfloat16* q_lat;   // [B, H, d_c] absorbed query, bf16
@@ -51,10 +57,11 @@ cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_U
 // stream_once: the call reads each cache tile once (loads carry an L2 evict-first hint);
 // pass false when other queries of the call read the same tiles.  1 <= Q <= the cluster
 // count; the workspace is that of B * Q queries.
+// fp8: the cache holds FP8 rows (kF8RowBytes each) instead of bf16 rows.
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
                                const __nv_bfloat16* ukt, const __nv_bfloat16* uv,
-                               const __nv_bfloat16* cache, long long cache_rows, const int32_t* offsets,
+                               const void* cache, bool fp8, long long cache_rows, const int32_t* offsets,
                                const int32_t* seq_lens, const int32_t* block_table, int bt_stride,
                                int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms, int* err_code, long long* err_detail, cudaStream_t s);

@@ -331,5 +331,8 @@ __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
 // swizzle_bytes: 128 (default) or 64; the box's inner extent must not exceed it.
 bool make_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                     const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes = 128);
+// Any element type of elem_bytes bytes; swizzle_bytes 128, 64 or 0 (none).
+bool make_tmap(CUtensorMap* map, CUtensorMapDataType dtype, int elem_bytes, const void* base, int rank,
+               const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box, int swizzle_bytes);
 
 }  // namespace mla

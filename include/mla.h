@@ -253,6 +253,53 @@ mla_status mla_decode_absorbed_noalloc(const mla_dims* dims, mla_weights w, cons
                                        const int32_t* offsets, int32_t B, void* out,
                                        mla_stream_t stream);
 
+/* -------------------------------------------------------------- FP8 latent cache */
+
+/* A quantised latent cache, which the pages name as a further compression ["02 - Multi-
+ * Latent Attention (MLA)", "Lo que esta fase NO cubre"] and as an engine's own cache format
+ * ["Multi-head Latent Attention (MLA) si arhitectura DeepSeekMoE", "Exemplul 1"], without
+ * giving a format.  An FP8 cache row holds one token: the latent c as d_c FP8 E4M3 codes
+ * (bytes [0, d_c)), the rotary key as d_hR bf16 values (bytes [d_c, d_c + 2 d_hR)), the
+ * token's scale s as fp32 (next 4 bytes), then zeros up to mla_fp8_row_bytes() (a multiple
+ * of 16); c_i = code_i * s.  Quantisation: s = max_i |c_i| / 448 (1 for an all-zero c) and
+ * code_i = e4m3(c_i / s), nearest even, every decision in fp32 from the bf16 row.  Half the
+ * bytes of a bf16 row per token (656 against 1152 for the V2/V3 shape).
+ * Tensor-core shape only (bf16, H = 128, d_c = 512, d_hR = 64, qk_nope = v_head = 128);
+ * other dims get -1 / 0 / MLA_ERR_UNSUPPORTED. */
+
+/* Bytes of one FP8 cache row (656 for the supported shape), or -1. */
+int64_t mla_fp8_row_bytes(const mla_dims* dims);
+
+/* FP8 rows of n bf16 cache rows (rows [n, d_c + d_hR], device, 16-byte aligned):
+ * cache_fp8[slot[i]] for i < n (slot int64 [n], device; NULL writes rows 0 .. n-1).
+ * cache_fp8: device, [capacity, mla_fp8_row_bytes()] bytes, 16-byte aligned.  A slot outside
+ * [0, capacity) is skipped and latches MLA_ERR_OUT_OF_RANGE.  n = 0 is a no-op. */
+mla_status mla_quantize_cache_fp8(const mla_dims* dims, const void* rows, const int64_t* slot, int32_t n,
+                                  void* cache_fp8, int64_t capacity, mla_stream_t stream);
+
+/* Workspace bytes of mla_append_cache_fp8 for n tokens (their bf16 rows), 0 if unsupported. */
+size_t mla_append_fp8_workspace_size(const mla_dims* dims, int32_t n);
+
+/* mla_append_cache into an FP8 cache: the same down-projection and RoPE give each token's
+ * bf16 row (in the workspace), which is quantised into cache_fp8[slot[i]] as by
+ * mla_quantize_cache_fp8.  workspace: device, >= mla_append_fp8_workspace_size(dims, n)
+ * bytes, 256-byte aligned. */
+mla_status mla_append_cache_fp8(const mla_dims* dims, const void* h, const void* W_DKV, const void* W_KR,
+                                const int32_t* pos, const int64_t* slot, int32_t n, void* cache_fp8,
+                                int64_t capacity, void* workspace, size_t ws_bytes, mla_stream_t stream);
+
+/* mla_decode_absorbed over an FP8 cache: the result of the decode on the dequantised rows
+ * [code * s | k_r].  Queries from q_nope/q_rope only, handles without W_O; cache_fp8
+ * [cache_rows, mla_fp8_row_bytes()] bytes, 16-byte aligned; offsets, invalid sequences and
+ * the workspace (mla_decode_workspace_size) as for mla_decode_absorbed.  The kernel
+ * dequantises each tile in shared memory to fp16 (code x s) and runs the latent products on
+ * fp16 operands (the absorbed query and the probabilities in fp16 too), the rotary ones in
+ * bf16, all accumulating in fp32. */
+mla_status mla_decode_absorbed_fp8(const mla_dims* dims, mla_weights w, const void* q_nope,
+                                   const void* q_rope, const void* cache_fp8, int64_t cache_rows,
+                                   const int32_t* offsets, int32_t B, void* out, void* workspace,
+                                   size_t ws_bytes, mla_stream_t stream);
+
 /* ---------------------------------------------------------------- causal prefill */
 
 /* Bytes of workspace mla_prefill_causal needs for B sequences of S tokens. */

@@ -47,6 +47,9 @@ def _declare(lib):
     lib.oracle_round_e4m3.restype = _D
     lib.oracle_round_e4m3.argtypes = [_D]
     lib.oracle_quantize_latent_fp8.argtypes = [_I32, _I32, _I32, _P, _P, _P]
+    lib.oracle_e4m3_bits.restype = ctypes.c_uint8
+    lib.oracle_e4m3_bits.argtypes = [_D]
+    lib.oracle_fp8_row_f32.argtypes = [_I32, _I32, _P, _I32, _P, _P]
     lib.oracle_rope.argtypes = [_I32, _P, _D, _D, _P]
     lib.oracle_latent_rows.argtypes = [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _D, _P]
     lib.oracle_query.argtypes = [_I32, _I32, _I32, _I32, _I32, _P, _P, _P, _D, _P, _P]
@@ -128,6 +131,26 @@ def quantize_latent_fp8(rows, d_c: int, lib=None) -> Tuple[np.ndarray, np.ndarra
     scales = np.empty(n)
     (lib or load()).oracle_quantize_latent_fp8(n, d_c, rw - d_c, _p(rows), _p(deq), _p(scales))
     return deq, scales
+
+
+def e4m3_bits(x, lib=None) -> np.ndarray:
+    """The E4M3 byte of each value (values as round_e4m3 returns them)."""
+    x = f64(x)
+    fn = (lib or load()).oracle_e4m3_bits
+    return np.array([fn(float(v)) for v in x.reshape(-1)], dtype=np.uint8).reshape(x.shape)
+
+
+def fp8_rows_f32(rows, d_c: int, row_bytes: int, lib=None) -> Tuple[np.ndarray, np.ndarray]:
+    """FP8 cache rows of bf16-valued rows [n, d_c + d_hR], every decision in float:
+    (bytes uint8 [n, row_bytes], dequantised rows float64 [n, d_c + d_hR])."""
+    rows = f64(rows)
+    n, rw = rows.shape
+    out = np.zeros((n, row_bytes), dtype=np.uint8)
+    deq = np.empty_like(rows)
+    fn = (lib or load()).oracle_fp8_row_f32
+    for i in range(n):
+        fn(d_c, rw - d_c, _p(rows[i]), row_bytes, _p(out[i]), _p(deq[i]))
+    return out, deq
 
 
 def rope(x, pos: float, theta: float = 10000.0, lib=None) -> np.ndarray:

@@ -110,6 +110,58 @@ void oracle_quantize_latent_fp8(int n, int d_c, int d_hR, const double* rows, do
     }
 }
 
+/* The E4M3 bit pattern of a value that round_e4m3 returns: sign in bit 7, the exponent field
+ * (bias 7; 0 for subnormals) in bits 6-3, the 3 mantissa bits in 2-0.  448 = 1.75 * 2^8 is
+ * 0x7E; the pattern 0x7F (NaN) never comes out. */
+uint8_t oracle_e4m3_bits(double v) {
+    uint8_t sign = signbit(v) ? 0x80 : 0x00;
+    double a = fabs(v);
+    if (a == 0.0) return sign;
+    int e;
+    double m = frexp(a, &e);               /* a = m * 2^e, m in [0.5, 1) */
+    int ex = e - 1;                        /* a = (2m) * 2^ex, 2m in [1, 2) */
+    if (ex < -6) {                         /* subnormal: a = k * 2^-9, k in 1 .. 7 */
+        int k = (int)rint(ldexp(a, 9));
+        return (uint8_t)(sign | k);
+    }
+    int mant = (int)rint((2.0 * m - 1.0) * 8.0);
+    return (uint8_t)(sign | ((ex + 7) << 3) | mant);
+}
+
+/* The FP8 cache row a kernel writes for one bf16 row [c | k_r] (d_c latent values, d_hR
+ * rotary values, both exactly representable in float), with every rounding decision taken
+ * in float (IEEE single, nearest even), as a kernel working in fp32 takes it:
+ *     amax = max |c_i|,  s = amax / 448 (s = 1 for amax = 0),  code_i = e4m3(c_i / s).
+ * Writes row_bytes bytes: the d_c codes, the d_hR rotary values as bf16 (the top 16 bits
+ * of their float patterns, exact for bf16 inputs), s as a float, zeros up to row_bytes.
+ * deq (nullable, d_c + d_hR doubles) receives [code_i * s | k_r]. */
+void oracle_fp8_row_f32(int d_c, int d_hR, const double* row, int row_bytes, uint8_t* out, double* deq) {
+    float amax = 0.0f;
+    for (int i = 0; i < d_c; ++i) {
+        float a = fabsf((float)row[i]);
+        if (a > amax) amax = a;
+    }
+    volatile float num = amax, den = 448.0f;   /* one float division, not folded */
+    float s = amax > 0.0f ? num / den : 1.0f;
+    memset(out, 0, (size_t)row_bytes);
+    for (int i = 0; i < d_c; ++i) {
+        volatile float ci = (float)row[i];
+        float q = ci / s;
+        double code = oracle_round_e4m3((double)q);
+        out[i] = oracle_e4m3_bits(code);
+        if (deq) deq[i] = code * (double)s;
+    }
+    for (int i = 0; i < d_hR; ++i) {
+        float v = (float)row[d_c + i];
+        uint32_t bits;
+        memcpy(&bits, &v, 4);
+        uint16_t b = (uint16_t)(bits >> 16);
+        memcpy(out + d_c + 2 * i, &b, 2);
+        if (deq) deq[d_c + i] = row[d_c + i];
+    }
+    memcpy(out + d_c + 2 * d_hR, &s, 4);
+}
+
 /* ------------------------------------------------------------------- RoPE [L1][L2] */
 
 /* out = x rotated: for i < d/2, angle = pos * theta^(-2i/d),

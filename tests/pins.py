@@ -315,6 +315,52 @@ def pin_fp8_latent(lib):
     assert np.array_equal(deq2[:, :d_c], deq[:, :d_c] * 8.0) and np.array_equal(sc2[[0, 1, 2, 3, 5]], sc[[0, 1, 2, 3, 5]] * 8)
 
 
+def pin_e4m3_bits(lib):
+    """The E4M3 byte encoding: every finite E4M3 value (all 254 non-NaN patterns) encodes to
+    the byte torch's float8_e4m3fn gives it, and a few patterns worked out by hand."""
+    codes = torch.arange(256, dtype=torch.int32).to(torch.uint8)
+    vals = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    finite = ~np.isnan(vals)
+    got = oracle.e4m3_bits(vals[finite], lib)
+    assert np.array_equal(got, codes.numpy()[finite]), "E4M3 bytes differ from torch's encoding"
+    for v, byte in [(448.0, 0x7E), (-448.0, 0xFE), (1.0, 0x38), (-0.0, 0x80), (2.0 ** -9, 0x01), (2.0 ** -6, 0x08),
+                    (1.125, 0x39), (-0.1015625, 0x9D)]:
+        assert int(oracle.e4m3_bits(np.array([v]), lib)[0]) == byte, (v, byte)
+
+
+def pin_fp8_row_f32(lib):
+    """The FP8 cache row with its decisions in float: codes equal torch's float8_e4m3fn cast
+    of the float quotients c / s (s = float(amax) / 448 in float), the rotary key is the
+    row's bf16 bytes, the scale field holds s, the rest is zero; it differs from the
+    float64-decision quantiser only where a quotient's float rounding crosses an E4M3
+    rounding boundary."""
+    r = _rs(23)
+    d_c, d_hR, nb = 64, 8, 96
+    rows = r.standard_normal((40, d_c + d_hR)) * np.exp2(r.uniform(-10, 10, (40, 1)))
+    rows[3, :d_c] = 0.0
+    rows[5, 7] = -0.0
+    rows = torch.from_numpy(rows).to(torch.bfloat16).to(torch.float64).numpy()   # bf16-valued rows
+    out, deq = oracle.fp8_rows_f32(rows, d_c, nb, lib)
+    t = torch.from_numpy(rows).to(torch.float32)
+    amax = t[:, :d_c].abs().amax(1)
+    s = torch.where(amax > 0, amax / torch.tensor(448.0, dtype=torch.float32), torch.ones_like(amax))
+    codes = (t[:, :d_c] / s[:, None]).to(torch.float8_e4m3fn)
+    assert np.array_equal(out[:, :d_c], codes.view(torch.uint8).numpy()), "codes differ from torch's float cast"
+    kr = t[:, d_c:].to(torch.bfloat16).contiguous().view(torch.uint8).numpy()
+    assert np.array_equal(out[:, d_c:d_c + 2 * d_hR], kr), "the rotary key is the row's bf16 bytes"
+    assert np.array_equal(out[:, d_c + 2 * d_hR:d_c + 2 * d_hR + 4].copy().view(np.float32)[:, 0], s.numpy())
+    assert not out[:, d_c + 2 * d_hR + 4:].any(), "padding is zero"
+    assert np.all(out[3, :d_c] == 0) and s[3] == 1.0, "a zero latent: codes 0, scale 1"
+    _close(deq[:, :d_c], codes.to(torch.float64).numpy() * s.double().numpy()[:, None], 0.0, "dequantised = code x s")
+    assert np.array_equal(deq[:, d_c:], rows[:, d_c:])
+    ref, sc64 = oracle.quantize_latent_fp8(rows, d_c, lib)
+    assert np.allclose(s.double().numpy(), sc64, rtol=2.0 ** -23, atol=0), "scales agree to float rounding"
+    code32 = codes.to(torch.float64).numpy()
+    code64 = oracle.round_e4m3(ref[:, :d_c] / sc64[:, None], lib)   # snaps the division's last-bit noise
+    same = code32 == code64
+    assert same.mean() > 0.99, "codes agree with the float64 decisions except near rounding boundaries"
+
+
 def pin_decode_multi(lib):
     """Multi-token decode: token t of the q_len new ones attends to the keys up to itself.
     Checked against torch attention with an explicit boolean mask, against the causal
@@ -362,4 +408,5 @@ def pin_decode_multi(lib):
 ALL_PINS = [pin_page_figures, pin_round_bf16, pin_rope, pin_latent_rows, pin_query,
             pin_decode_vs_library_attention, pin_decode_textbook_reduction, pin_decode_score_split,
             pin_decode_special_cases, pin_naive_equals_absorbed, pin_decode_batch_driver,
-            pin_out_proj, pin_prefill, pin_decode_multi, pin_e4m3, pin_fp8_latent]
+            pin_out_proj, pin_prefill, pin_decode_multi, pin_e4m3, pin_fp8_latent, pin_e4m3_bits,
+            pin_fp8_row_f32]

@@ -92,3 +92,13 @@ def test_cpu_baseline_runs_the_oracle_on_several_threads():
     s = bench.time_oracle_units(w, inp, 0.0, min_units=3, max_units=3, tokens=16)
     assert s["cores"] == 1 and "first 16 rows" in s["sample"]
     assert bench.host_cores() >= 1
+
+
+def test_fp8_step_counts_656_bytes_per_token():
+    w = workloads.WORKLOADS["v3_decode_fp8_b32_ctx4096"]
+    a = bench.alg_step_fp8(w)
+    tokens = 32 * 4096
+    assert a["cache_bytes"] == tokens * 656
+    assert a["bytes"] == tokens * 656 + 2 * 128 * 128 * 512 * 2 + 32 * 128 * 192 * 2 + 32 * 128 * 128 * 2
+    assert a["flops"] == bench.alg_step(workloads.WORKLOADS["v3_decode_b32_ctx4096"])["flops"]
+    assert bench.alg_kernel_bytes("tc_flash_decode_fp8", w) == tokens * 656 + 32 * 128 * 576 * 2

@@ -34,6 +34,11 @@ MUTANTS = {
     "e4m3_subnormal_quantum": ("int ue = e - 1 < -6 ? -6 : e - 1;", "int ue = e - 1 < -7 ? -7 : e - 1;"),
     "fp8_scale_to_240": ("double sc = amax > 0.0 ? amax / 448.0 : 1.0;", "double sc = amax > 0.0 ? amax / 240.0 : 1.0;"),
     "mla_row_without_rope": ("return (d_c + d_hR) * layers;", "return d_c * layers;"),
+    "e4m3_bits_bias": ("return (uint8_t)(sign | ((ex + 7) << 3) | mant);", "return (uint8_t)(sign | ((ex + 8) << 3) | mant);"),
+    "e4m3_bits_no_sign": ("uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
+    "fp8_row_scale_not_stored": ("memcpy(out + d_c + 2 * d_hR, &s, 4);", ""),
+    "fp8_row_rope_low_half": ("uint16_t b = (uint16_t)(bits >> 16);", "uint16_t b = (uint16_t)(bits & 0xFFFF);"),
+    "fp8_row_scale_to_240": ("float s = amax > 0.0f ? num / den : 1.0f;", "float s = amax > 0.0f ? num / 240.0f : 1.0f;"),
     "out_proj_transposed": ("acc += W_O[(size_t)j * Hv + k] * o[(size_t)i * Hv + k];",
                             "acc += W_O[(size_t)(k % d_model) * Hv + j % Hv] * o[(size_t)i * Hv + k];"),
 }

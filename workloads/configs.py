@@ -27,7 +27,7 @@ TENSOR_IDS = {
 @dataclass(frozen=True)
 class Workload:
     name: str
-    kind: str                 # "decode_layer" | "decode_attn" | "decode_multi" | "prefill"
+    kind: str                 # "decode_layer" | "decode_attn" | "decode_fp8" | "decode_multi" | "prefill"
     B: int
     H: int
     d_model: int              # 0 when the workload starts from given queries
@@ -79,6 +79,11 @@ WORKLOADS: Dict[str, Workload] = {
     "v2_prefill_b4_s4096": Workload("v2_prefill_b4_s4096", "prefill", B=4, H=128, d_model=5120,
                                     d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
                                     seed=_seed(5), ctx=4096),
+    # the V3 decode workload over an FP8 latent cache (its bf16 rows quantised once, before
+    # the step: E4M3 codes with one fp32 scale per token, bf16 rotary key)
+    "v3_decode_fp8_b32_ctx4096": Workload("v3_decode_fp8_b32_ctx4096", "decode_fp8", B=32, H=128, d_model=0,
+                                          d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
+                                          seed=_seed(2), ctx=4096),
     # multi-token decode (speculative verification): 2 new tokens per sequence over 4096
     # cached tokens, paged cache
     "v3_mtp_b32_ctx4096_q2": Workload("v3_mtp_b32_ctx4096_q2", "decode_multi", B=32, H=128, d_model=0,
@@ -87,7 +92,8 @@ WORKLOADS: Dict[str, Workload] = {
 }
 
 # the order the workloads are listed in (smallest first)
-ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_mtp_b32_ctx4096_q2", "v3_ragged_b64",
+ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_decode_fp8_b32_ctx4096", "v3_mtp_b32_ctx4096_q2",
+         "v3_ragged_b64",
          "v3_layer_b128_ctx8192", "v2_prefill_b4_s4096"]
 
 
@@ -140,6 +146,7 @@ def make_inputs(w: Workload) -> Dict[str, torch.Tensor]:
 
     decode_attn : cache [sum L, row], offsets int32 [B+1], q_nope [B,H,qk_nope],
                   q_rope [B,H,d_hR] (already rotated), W_UK, W_UV.
+    decode_fp8  : as decode_attn (the bf16 rows are quantised to FP8 rows before the step).
     decode_multi: cache [sum (L + q_len), row] (the new tokens' rows last in each sequence),
                   offsets int32 [B+1], q_nope [B,q_len,H,qk_nope], q_rope [B,q_len,H,d_hR],
                   W_UK, W_UV.
@@ -151,7 +158,7 @@ def make_inputs(w: Workload) -> Dict[str, torch.Tensor]:
     """
     d = make_weights(w)
     L = lengths(w)
-    if w.kind == "decode_attn":
+    if w.kind in ("decode_attn", "decode_fp8"):
         offs = np.concatenate([[0], np.cumsum(L)]).astype(np.int32)
         d["offsets"] = torch.from_numpy(offs)
         d["cache"] = _tensor(w, "cache", (int(offs[-1]), w.row), w.cache_std)
