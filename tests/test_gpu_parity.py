@@ -547,12 +547,13 @@ def test_multi_token_decode_over_pages_matches_the_oracle(q_len):
     assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", "multi-token decode")
 
 
-def test_chunked_prefill_over_an_existing_cache():
-    """Absorbed chunked prefill: a chunk of 100 new tokens per sequence attends to a cached
-    prefix (300 and 77 tokens) and causally to itself, K and V never materialised: the
-    multi-token call with q_len = the chunk (200 per-token sequences).  Sampled tokens of
+@pytest.mark.parametrize("chunk,prefix", [(100, [300, 77]), (1000, [4096])])
+def test_chunked_prefill_over_an_existing_cache(chunk, prefix):
+    """Absorbed chunked prefill: a chunk of new tokens per sequence attends to a cached
+    prefix and causally to itself, K and V never materialised: the multi-token call with
+    q_len = the chunk (one query sequence per new token).  100-token chunks over 300- and
+    77-token prefixes, and a 1000-token chunk over a 4096-token prefix.  Sampled tokens of
     the chunk against the oracle, whose multi-token decode is pinned to its causal prefill."""
-    chunk, prefix = 100, [300, 77]
     lengths = [p + chunk for p in prefix]
     w, inp = reduced_attn_inputs(lengths, seed=59)
     r = np.random.default_rng(59)
@@ -581,10 +582,11 @@ def test_chunked_prefill_over_an_existing_cache():
                                         q_nope=qn.to(DEV), q_rope=qr.to(DEV))
     assert mla.mla_get_device_error() == (0, 0)
     out = out.cpu()
-    units = [(b, t, h) for b in range(w.B) for t in (0, 1, 63, 64, 99) for h in (0, 64, 127)]
+    ts = sorted({0, 1, 63, 64, chunk // 2, chunk - 2, chunk - 1})
+    units = [(b, t, h) for b in range(w.B) for t in ts for h in (0, 64, 127)]
     want = oracle.decode_multi(qn, qr, inp["cache"], inp["offsets"], inp["W_UK"], inp["W_UV"], w.scale,
                                units=units, absorbed=True)
-    assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", "chunked prefill")
+    assert_close(torch.stack([out[b, t, h] for b, t, h in units]), want, "bf16", f"chunked prefill {chunk}")
 
 
 def test_decode_large_batch_spans_several_sequence_blocks():

@@ -89,11 +89,16 @@ WORKLOADS: Dict[str, Workload] = {
     "v3_mtp_b32_ctx4096_q2": Workload("v3_mtp_b32_ctx4096_q2", "decode_multi", B=32, H=128, d_model=0,
                                       d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
                                       seed=_seed(6), ctx=4096, q_len=2),
+    # absorbed chunked prefill over a cached prefix: 1024 new tokens per sequence over 4096
+    # cached tokens, causal inside the chunk, paged cache (every new token a query sequence)
+    "v3_chunk_b4_ctx4096_c1024": Workload("v3_chunk_b4_ctx4096_c1024", "decode_multi", B=4, H=128, d_model=0,
+                                          d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
+                                          seed=_seed(7), ctx=4096, q_len=1024),
 }
 
 # the order the workloads are listed in (smallest first)
 ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_decode_fp8_b32_ctx4096", "v3_mtp_b32_ctx4096_q2",
-         "v3_ragged_b64",
+         "v3_ragged_b64", "v3_chunk_b4_ctx4096_c1024",
          "v3_layer_b128_ctx8192", "v2_prefill_b4_s4096"]
 
 
