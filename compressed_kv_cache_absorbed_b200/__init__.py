@@ -68,6 +68,7 @@ SIGNATURES = {
                                   _P]),
     "mla_decode_absorbed_fp8": (_S, [_D, _P, _P, _P, _P, ctypes.c_int64, _P, ctypes.c_int32, _P, _P, ctypes.c_size_t,
                                      _P]),
+    "mla_rope_apply": (_S, [_P, _P, ctypes.c_int64, _P, _P]),
     "mla_set_wait_limit": (_S, [ctypes.c_uint32]),
     "mla_test_starve_projection": (_S, [ctypes.c_int32]),
     "mla_profile_enable": (None, [ctypes.c_int32]),
@@ -281,6 +282,11 @@ def mla_get_device_error(stream=None):
     d = ctypes.c_int64(0)
     st = _lib.mla_get_device_error(_stream(stream), ctypes.byref(d))
     return int(st), int(d.value)
+
+
+def mla_rope_apply(x, cos_sin, y, stream=None) -> None:
+    """y = the RoPE pairs of x (float32 [..., 2k]) rotated by cos_sin (float64 [..., k, 2])."""
+    _check(_lib.mla_rope_apply(_ptr(x), _ptr(cos_sin), x.numel() // 2, _ptr(y), _stream(stream)), "mla_rope_apply")
 
 
 def mla_set_wait_limit(polls: int) -> None:

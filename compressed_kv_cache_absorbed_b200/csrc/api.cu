@@ -821,6 +821,15 @@ extern "C" mla_status mla_prefill_causal(const mla_dims* d, mla_weights w, const
 
 // ------------------------------------------------------------------- diagnostics
 
+extern "C" mla_status mla_rope_apply(const float* x, const double* cos_sin, int64_t pairs, float* y,
+                                     mla_stream_t stream) {
+    if (pairs < 0) return MLA_ERR_INVALID_ARG;
+    if (pairs == 0) return MLA_OK;
+    if (!x || !cos_sin || !y || ((uintptr_t)cos_sin & 15)) return MLA_ERR_INVALID_ARG;
+    cudaError_t e = mla::tc::rope_apply(x, (const double2*)cos_sin, pairs, y, (cudaStream_t)stream);
+    return e == cudaSuccess ? MLA_OK : cuda_fail(e, "mla_rope_apply");
+}
+
 extern "C" mla_status mla_set_wait_limit(uint32_t polls) {
     const uint32_t p = polls ? polls : 1u << 22;
     MLA_CUDA(mla::tc::set_wait_limit_decode(p));

@@ -18,6 +18,21 @@ template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float
     return __float2bfloat16_rn(x);
 }
 
+// ------------------------------------------------------------------------ RoPE
+
+// The rotation of one RoPE pair (x0, x1) by the angle whose cosine and sine are (c, s):
+//     (x0 c - x1 s, x0 s + x1 c)
+// in double, every product and sum rounded on its own (no fused multiply-add), then rounded
+// to float.  Every kernel that rotates uses this, so an IEEE double restatement on the CPU
+// with the same inputs gives the same bits.
+__device__ __forceinline__ void rope_rotate(float& x0, float& x1, double c, double s) {
+    const double a = (double)x0, b = (double)x1;
+    const double r0 = __dsub_rn(__dmul_rn(a, c), __dmul_rn(b, s));
+    const double r1 = __dadd_rn(__dmul_rn(a, s), __dmul_rn(b, c));
+    x0 = __double2float_rn(r0);
+    x1 = __double2float_rn(r1);
+}
+
 // ------------------------------------------------------------ device error word
 
 // Kernels that meet bad device-side data (a slot outside the cache, decreasing offsets)

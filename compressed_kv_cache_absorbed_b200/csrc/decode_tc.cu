@@ -483,13 +483,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         // rotary box (bf16, 64-byte swizzle) is copied as it is (same alignment, same
         // swizzle pattern).
         const int dt = threadIdx.x - 14 * 32;
+        constexpr int NF = kF8Stages > 0 ? kF8Stages : 1;   // (the bf16 variant never gets here)
         uint32_t g = 0;
         bool ok = true;
         Seg cur;
         while (ok && !*abort_flag && it.next(cur)) {
             for (int j = cur.j0; j < cur.j1; ++j, ++g) {
-                const int s = g % kF8Stages, d = g % kStages;
-                if (!ptx::mbar_wait(&f8_full[s], (g / kF8Stages) & 1, abort_flag) ||
+                const int s = g % NF, d = g % kStages;
+                if (!ptx::mbar_wait(&f8_full[s], (g / NF) & 1, abort_flag) ||
                     (g >= (uint32_t)kStages && !ptx::mbar_wait(&tile_empty[d], ((g / kStages) - 1) & 1, abort_flag))) {
                     ok = false;
                     break;

@@ -274,9 +274,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                             const int within = (f0 + j) % out.period;
                             if (within < out.rope_start) continue;
                             const double2 t = rope_cs(out.rope_tab, out.d_rope, out.pos, out.pos_mod, out.theta, xr, (within - out.rope_start) >> 1);
-                            const double ve = v[j], vo = v[j + 1];
-                            v[j] = (float)(ve * t.x - vo * t.y);
-                            v[j + 1] = (float)(ve * t.y + vo * t.x);
+                            rope_rotate(v[j], v[j + 1], t.x, t.y);
                         }
                     }
                     uint4* dst = (uint4*)((__nv_bfloat16*)base + (long long)tl.z * out.sz + f0 + orow * out.sn);
@@ -312,8 +310,9 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                         const float partner = __shfl_xor_sync(0xffffffffu, v, 1);
                         if (rope_row) {
                             const double2 t = rope_cs(out.rope_tab, out.d_rope, out.pos, out.pos_mod, out.theta, n, (within - out.rope_start) >> 1);
-                            v = (row & 1) ? (float)((double)partner * t.y + (double)v * t.x)
-                                          : (float)((double)v * t.x - (double)partner * t.y);
+                            float x0 = (row & 1) ? partner : v, x1 = (row & 1) ? v : partner;
+                            rope_rotate(x0, x1, t.x, t.y);
+                            v = (row & 1) ? x1 : x0;
                         }
                     }
                     if (row >= Mx) continue;
@@ -375,6 +374,25 @@ rope_table_kernel(const int32_t* __restrict__ pos, int pos_mod, int N, int half,
 }
 
 }  // namespace
+
+namespace {
+__global__ void __launch_bounds__(256)
+rope_apply_kernel(const float* __restrict__ x, const double2* __restrict__ cs, long long pairs, float* __restrict__ y) {
+    for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < pairs; i += (long long)gridDim.x * blockDim.x) {
+        float x0 = x[2 * i], x1 = x[2 * i + 1];
+        rope_rotate(x0, x1, cs[i].x, cs[i].y);
+        y[2 * i] = x0;
+        y[2 * i + 1] = x1;
+    }
+}
+}  // namespace
+
+cudaError_t rope_apply(const float* x, const double2* cs, long long pairs, float* y, cudaStream_t s) {
+    if (pairs <= 0) return cudaSuccess;
+    const long long want = (pairs + 255) / 256;
+    rope_apply_kernel<<<(int)(want < 4096 ? want : 4096), 256, 0, s>>>(x, cs, pairs, y);
+    return cudaGetLastError();
+}
 
 cudaError_t set_wait_limit_gemm(uint32_t polls) { return ptx::set_wait_limit_of_this_file(polls); }
 

@@ -50,6 +50,10 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
                          const __nv_bfloat16* B, long long sBz, long long sBn, const GemmOut& out,
                          int* err_code, long long* err_detail, cudaStream_t s, bool chain_head = false);
 
+// y = each pair (x[2i], x[2i+1]) rotated by (cos, sin) = cs[i] with the arithmetic every
+// rotating epilogue uses (rope_rotate).
+cudaError_t rope_apply(const float* x, const double2* cs, long long pairs, float* y, cudaStream_t s);
+
 // Sets the polls a bounded wait of the GEMM kernel makes before giving up (current device).
 cudaError_t set_wait_limit_gemm(uint32_t polls);
 

@@ -90,10 +90,7 @@ proj_rope_kernel(const T* __restrict__ A, int M, int K, const T* __restrict__ W1
                 const double inv = pow((double)theta, -2.0 * (double)pi / (double)d_rope);
                 double sn, cs;
                 sincos((double)p * inv, &sn, &cs);
-                const double r0 = (double)v0 * cs - (double)v1 * sn;
-                const double r1 = (double)v0 * sn + (double)v1 * cs;
-                v0 = (float)r0;
-                v1 = (float)r1;
+                rope_rotate(v0, v1, cs, sn);
             }
             T* o = out + dst * ld_out + gn;
             o[0] = from_f<T>(v0);

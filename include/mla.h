@@ -326,6 +326,15 @@ mla_status mla_prefill_causal(const mla_dims* dims, mla_weights w, const void* h
  * receives a kernel-specific detail value. */
 mla_status mla_get_device_error(mla_stream_t stream, int64_t* detail);
 
+/* The rotary step alone, for checking its arithmetic: y[2i], y[2i+1] = the pair (x[2i],
+ * x[2i+1]) rotated by the angle whose (cos, sin) are cos_sin[2i], cos_sin[2i+1] ["02 -
+ * Multi-Latent Attention (MLA)", "Truco de codificacion posicional": the decoupled key
+ * carries the rotary position].  The rotation is the one every rotating kernel of the
+ * library applies (the cache append's k_r and the query projection's rotary part): in
+ * double, each product and sum rounded on its own, then rounded to float.  x, y: float
+ * [2 pairs], cos_sin: double [2 pairs] (16-byte aligned); device pointers. */
+mla_status mla_rope_apply(const float* x, const double* cos_sin, int64_t pairs, float* y, mla_stream_t stream);
+
 /* Failure-detection test hooks.  Leave both at their defaults outside tests.
  *
  * mla_set_wait_limit: on the current device, the number of polls each bounded wait in the

@@ -51,6 +51,7 @@ def _declare(lib):
     lib.oracle_e4m3_bits.argtypes = [_D]
     lib.oracle_fp8_row_f32.argtypes = [_I32, _I32, _P, _I32, _P, _P]
     lib.oracle_rope.argtypes = [_I32, _P, _D, _D, _P]
+    lib.oracle_rope_pairs_f32.argtypes = [_I64, _P, _P, _P]
     lib.oracle_latent_rows.argtypes = [_I32, _I32, _I32, _I32, _P, _P, _P, _P, _D, _P]
     lib.oracle_query.argtypes = [_I32, _I32, _I32, _I32, _I32, _P, _P, _P, _D, _P, _P]
     att = [_I32, _I32, _I32, _I32, _I32, _D, _P, _P, _P, _P, _P, _P, _P, _P]
@@ -151,6 +152,17 @@ def fp8_rows_f32(rows, d_c: int, row_bytes: int, lib=None) -> Tuple[np.ndarray, 
     for i in range(n):
         fn(d_c, rw - d_c, _p(rows[i]), row_bytes, _p(out[i]), _p(deq[i]))
     return out, deq
+
+
+def rope_pairs_f32(x, cos_sin, lib=None) -> np.ndarray:
+    """float32 pairs rotated by given (cos, sin) in double, each operation rounded, then
+    rounded to float32 (the kernels' rotation arithmetic)."""
+    x = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    cs = np.ascontiguousarray(np.asarray(cos_sin, dtype=np.float64))
+    assert cs.size == x.size
+    y = np.empty_like(x)
+    (lib or load()).oracle_rope_pairs_f32(x.size // 2, _p(x), _p(cs), _p(y))
+    return y
 
 
 def rope(x, pos: float, theta: float = 10000.0, lib=None) -> np.ndarray:

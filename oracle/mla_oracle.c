@@ -176,6 +176,20 @@ void oracle_rope(int d, const double* x, double pos, double theta, double* out) 
     }
 }
 
+/* The rotation of RoPE pairs restated in the precision kernels rotate in: for pair i, with
+ * (c, s) = cs[2i], cs[2i+1],
+ *     y[2i] = float(x0 c - x1 s),   y[2i+1] = float(x0 s + x1 c)
+ * in IEEE double, each product and sum rounded on its own (this file is compiled without
+ * contraction into fused multiply-adds), then rounded to float once. */
+void oracle_rope_pairs_f32(int64_t pairs, const float* x, const double* cs, float* y) {
+    for (int64_t i = 0; i < pairs; ++i) {
+        double x0 = x[2 * i], x1 = x[2 * i + 1], c = cs[2 * i], s = cs[2 * i + 1];
+        double p0 = x0 * c, p1 = x1 * s, p2 = x0 * s, p3 = x1 * c;
+        y[2 * i] = (float)(p0 - p1);
+        y[2 * i + 1] = (float)(p2 + p3);
+    }
+}
+
 /* ------------------------------------------------- latent cache rows [L1][L4][L5] */
 
 /* For each token i: c = W_DKV h_i (d_c values), k_r = RoPE(W_KR h_i, pos_i) (d_hR values);

@@ -315,6 +315,20 @@ def pin_fp8_latent(lib):
     assert np.array_equal(deq2[:, :d_c], deq[:, :d_c] * 8.0) and np.array_equal(sc2[[0, 1, 2, 3, 5]], sc[[0, 1, 2, 3, 5]] * 8)
 
 
+def pin_rope_pairs_f32(lib):
+    """The float-output rotation: with (cos, sin) of the oracle's own angle it is the oracle's
+    float64 RoPE rounded once to float, bit for bit (pairing, signs and order included)."""
+    r = _rs(24)
+    d, theta = 64, 10000.0
+    for pos in (0, 1, 17, 4095, 40000):
+        x = r.standard_normal(d).astype(np.float32)
+        ang = pos * theta ** (-2.0 * np.arange(d // 2) / d)
+        cs = np.stack([np.cos(ang), np.sin(ang)], 1)
+        y = oracle.rope_pairs_f32(x, cs, lib)
+        ref = oracle.rope(x.astype(np.float64), pos, theta, lib).astype(np.float32)
+        assert np.array_equal(y.view(np.uint32), ref.view(np.uint32)), f"pos {pos}"
+
+
 def pin_e4m3_bits(lib):
     """The E4M3 byte encoding: every finite E4M3 value (all 254 non-NaN patterns) encodes to
     the byte torch's float8_e4m3fn gives it, and a few patterns worked out by hand."""
@@ -409,4 +423,4 @@ ALL_PINS = [pin_page_figures, pin_round_bf16, pin_rope, pin_latent_rows, pin_que
             pin_decode_vs_library_attention, pin_decode_textbook_reduction, pin_decode_score_split,
             pin_decode_special_cases, pin_naive_equals_absorbed, pin_decode_batch_driver,
             pin_out_proj, pin_prefill, pin_decode_multi, pin_e4m3, pin_fp8_latent, pin_e4m3_bits,
-            pin_fp8_row_f32]
+            pin_fp8_row_f32, pin_rope_pairs_f32]

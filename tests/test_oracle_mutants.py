@@ -34,6 +34,9 @@ MUTANTS = {
     "e4m3_subnormal_quantum": ("int ue = e - 1 < -6 ? -6 : e - 1;", "int ue = e - 1 < -7 ? -7 : e - 1;"),
     "fp8_scale_to_240": ("double sc = amax > 0.0 ? amax / 448.0 : 1.0;", "double sc = amax > 0.0 ? amax / 240.0 : 1.0;"),
     "mla_row_without_rope": ("return (d_c + d_hR) * layers;", "return d_c * layers;"),
+    "rope_pairs_sign": ("y[2 * i] = (float)(p0 - p1);", "y[2 * i] = (float)(p0 + p1);"),
+    "rope_pairs_swapped": ("double x0 = x[2 * i], x1 = x[2 * i + 1], c = cs[2 * i], s = cs[2 * i + 1];",
+                           "double x1 = x[2 * i], x0 = x[2 * i + 1], c = cs[2 * i], s = cs[2 * i + 1];"),
     "e4m3_bits_bias": ("return (uint8_t)(sign | ((ex + 7) << 3) | mant);", "return (uint8_t)(sign | ((ex + 8) << 3) | mant);"),
     "e4m3_bits_no_sign": ("uint8_t sign = signbit(v) ? 0x80 : 0x00;", "uint8_t sign = 0x00;"),
     "fp8_row_scale_not_stored": ("memcpy(out + d_c + 2 * d_hR, &s, 4);", ""),
