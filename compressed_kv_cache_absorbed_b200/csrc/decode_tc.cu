@@ -179,11 +179,15 @@ struct SeqSrc {
 // Partial slots: a piece that starts at its query's first tile takes slot v; the one piece
 // of a cluster that continues a query begun in an earlier range takes slot B Q + cluster.
 // So B Q + clusters slots suffice.
+template <bool kSib>
 struct SegIter {
     SeqSrc src;
     int B, lo, hi, cluster, b, cs;
-    int Q, t;
+    int Qr, tr;   // siblings and this cluster's query (used with kSib only)
+    __device__ __forceinline__ int Q() const { return kSib ? Qr : 1; }
+    __device__ __forceinline__ int t() const { return kSib ? tr : 0; }
     __device__ bool next(Seg& s) {
+        const int Q = this->Q(), t = this->t();
         while (b < B && cs < hi) {
             const int L = src.len(b);
             const long long r0 = src.row0(b);
@@ -235,17 +239,18 @@ __device__ __forceinline__ void dequant16(const uint4 c, __half2 s, uint4& lo, u
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-template <bool kF8>
+template <bool kF8, bool kSib>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(DecCfg<kF8>::kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_constant__ CUtensorMap tm_rope,
                  const __grid_constant__ CUtensorMap tm_scale,
                  const __nv_bfloat16* __restrict__ q_lat,
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
-                 const SeqSrc src, int B, int Q, int stream_once, long long cache_rows,
+                 const SeqSrc src, int B, int Q_arg, int stream_once, long long cache_rows,
                  float scale_log2,
                  float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
     constexpr int kStages = DecCfg<kF8>::kStages, kF8Stages = DecCfg<kF8>::kF8Stages;
+    const int Q = kSib ? Q_arg : 1;   // queries per sequence (sibling clusters)
     constexpr int kThreads = DecCfg<kF8>::kThreads;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     if (ptx::smem_u32(smem_raw) & 1023) {   // uniform across the CTA: leave before any sync
@@ -394,7 +399,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             __syncthreads();
         }
     }
-    SegIter it{src, B, lo, hi, cluster, plan_first[0], plan_first[1], Q, tok};
+    SegIter<kSib> it{src, B, lo, hi, cluster, plan_first[0], plan_first[1], Q, tok};
     Seg sg;
 
     if (warp == 0) {
@@ -538,7 +543,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             // the next tile as soon as that tile has landed and the S columns are free.  S may
             // run ahead of O by as many tiles as the ring holds.  Tiles are taken in one flat
             // pass over all pieces (two iterators: one for S, one for O).
-            SegIter its = it;
+            SegIter<kSib> its = it;
             Seg ss;
             bool s_have = !*abort_flag && its.next(ss);
             int s_j = s_have ? ss.j0 : 0;
@@ -547,8 +552,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             bool o_have = !*abort_flag && it.next(sg);
             int o_j = o_have ? sg.j0 : 0;
             // the issuer polls its barriers without blocking: allow 16 polls per wait poll
-            const uint64_t idle_limit = (uint64_t)ptx::g_wait_limit << 4;
-            uint64_t idle = 0;
+            uint32_t idle = 0;
             while (o_have) {
                 // ---- O of tile g
                 if (g < s_g && ptx::mbar_test(&p_ready[g & 1], (g >> 1) & 1)) {
@@ -601,7 +605,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         continue;
                     }
                 }
-                if (++idle > idle_limit || *abort_flag) {
+                if (++idle > (ptx::g_wait_limit << 4) || *abort_flag) {
                     ok = false;
                     break;
                 }
@@ -880,13 +884,14 @@ constexpr int kMergeABytes = 8 * 128 * 128;   // W_UV[h]: 8 chunks of 128 rows x
 template <int BN>
 constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
-template <int BN>
+template <int BN, bool kSib>
 __global__ void __launch_bounds__(kMergeThreads, 1)
-merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B, int Q,
+merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B, int Q_arg,
                  const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)merge_smem_raw + 1023) & ~(uintptr_t)1023);
+    const int Q = kSib ? Q_arg : 1;   // queries per sequence
     uint8_t* sA = smem;
     uint8_t* sB = smem + kMergeABytes;
     uint64_t* a_full = (uint64_t*)(sB + 8 * BN * 128);
@@ -954,18 +959,20 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
                 chunk += v;
             }
             const int cs = before + incl - cb;
-            if (b < B && nt > 0) {
+            if (!kSib) {
+                if (b < B && b >= n0 && b < n0 + BN) {
+                    s_pos[0][b - n0] = cs + kPieceCost;
+                    s_pos[1][b - n0] = cs + kPieceCost + nt;
+                }
+            } else if (b < B) {
+                const int Lb = nt > 0 ? src.len(b) : 0;
                 for (int t = 0; t < Q; ++t) {
                     const int v = b * Q + t;
                     if (v >= n0 && v < n0 + BN) {
-                        s_pos[0][v - n0] = cs + kPieceCost;
-                        s_pos[1][v - n0] = cs + kPieceCost + tiles_of_len(src.len(b) - (Q - 1 - t));
+                        const int ntt = tiles_of_len(Lb - (Q - 1 - t));
+                        s_pos[0][v - n0] = ntt > 0 ? cs + kPieceCost : 0;
+                        s_pos[1][v - n0] = ntt > 0 ? cs + kPieceCost + ntt : 0;
                     }
-                }
-            } else if (b < B) {
-                for (int t = 0; t < Q; ++t) {
-                    const int v = b * Q + t;
-                    if (v >= n0 && v < n0 + BN) s_pos[0][v - n0] = s_pos[1][v - n0] = 0;
                 }
             }
             carry += chunk;
@@ -984,7 +991,7 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
     }
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int r = warp + kW * i, v = n0 + r, tq = v % Q;
+        const int r = warp + kW * i, v = n0 + r, tq = kSib ? v % Q : 0;
         const int t0 = t0r[i], t1 = t1r[i];
         float acc[16];
 #pragma unroll
@@ -995,7 +1002,9 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
             // NV + that cluster
             const int cfirst = t0 / per;
             const int np = (t1 - 1) / per - cfirst + 1;
-            auto slot_of = [&](int p) -> long long { return p == 0 ? v : NV + (long long)(cfirst + p) * Q + tq; };
+            auto slot_of = [&](int p) -> long long {
+                return p == 0 ? v : kSib ? NV + (long long)(cfirst + p) * Q + tq : B + cfirst + p;
+            };
             // (m, l) of up to 32 pieces (lane p) and the first 4 pieces' partial rows are
             // requested together; the weights need the maximum, the loads do not
             float2 ml = lane < np ? *(const float2*)(part_ml + (slot_of(lane) * 128 + h) * 2)
@@ -1268,17 +1277,34 @@ cudaError_t launch_absorb_any(int NV, const __nv_bfloat16* ukt, const CUtensorMa
                       : launch_absorb<128, kF16>(ukt, mq, NV, q_lat, err_code, err_detail, s);
 }
 
+template <bool kSib>
+cudaError_t launch_merge(int NV, const __nv_bfloat16* uv, const SeqSrc& seqs, int P, int B, int Q, const DecodeWs& ws,
+                         __nv_bfloat16* o, int* err_code, long long* err_detail, cudaStream_t s) {
+    if (NV <= 32) {
+        static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32, kSib>, merge_smem<32>());
+        if (attr != cudaSuccess) return attr;
+        return launch_pdl(merge_wuv_kernel<32, kSib>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
+                          seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
+                          err_code, err_detail);
+    }
+    static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64, kSib>, merge_smem<64>());
+    if (attr != cudaSuccess) return attr;
+    return launch_pdl(merge_wuv_kernel<64, kSib>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
+                      uv, seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
+                      err_code, err_detail);
+}
+
 int g_clusters_cached = 0;
 
 template <bool kF8>
 int resident_clusters(int num_sms) {
-    set_smem_attrs(decode_tc_kernel<kF8>, dec_smem<kF8>());
+    set_smem_attrs(decode_tc_kernel<kF8, false>, dec_smem<kF8>());
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(2 * (num_sms / 2), 1, 1);
     cfg.blockDim = dim3(DecCfg<kF8>::kThreads, 1, 1);
     cfg.dynamicSmemBytes = dec_smem<kF8>();
     int n = 0;
-    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<kF8>, &cfg) != cudaSuccess || n <= 0) {
+    if (cudaOccupancyMaxActiveClusters(&n, decode_tc_kernel<kF8, false>, &cfg) != cudaSuccess || n <= 0) {
         cudaGetLastError();
         n = num_sms / 2;
     }
@@ -1372,12 +1398,14 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
                 !make_tmap_bf16(&mr, cache, 2, dims, strides, box_rope, 64))
                 return cudaErrorInvalidValue;
             msc = mr;   // unused
-            static const cudaError_t attr = set_smem_attrs(decode_tc_kernel<false>, dec_smem<false>());
-            if (attr != cudaSuccess) return attr;
-            e = launch_pdl(decode_tc_kernel<false>, dim3(2 * P), dim3(DecCfg<false>::kThreads), dec_smem<false>(), s,
-                           m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h, seqs, B, Q, (int)(stream_once ? 1 : 0),
-                           (long long)cache_rows, scale_log2, ws.part_o, ws.part_ml, (const uint8_t*)uv,
-                           (long long)kTiledWeightBytes, err_code, err_detail);
+            static const cudaError_t attr1 = set_smem_attrs(decode_tc_kernel<false, false>, dec_smem<false>());
+            static const cudaError_t attr2 = set_smem_attrs(decode_tc_kernel<false, true>, dec_smem<false>());
+            if (attr1 != cudaSuccess) return attr1;
+            if (attr2 != cudaSuccess) return attr2;
+            e = launch_pdl(Q > 1 ? decode_tc_kernel<false, true> : decode_tc_kernel<false, false>, dim3(2 * P),
+                           dim3(DecCfg<false>::kThreads), dec_smem<false>(), s, m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h,
+                           seqs, B, Q, (int)(stream_once ? 1 : 0), (long long)cache_rows, scale_log2, ws.part_o,
+                           ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code, err_detail);
         } else {
             // FP8 rows of kF8RowBytes: codes as bytes, the rotary key as bf16 elements, the
             // scale field as fp32 elements
@@ -1392,9 +1420,10 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
                 !make_tmap(&mr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, cache, 2, dr, sr, br, 64) ||
                 !make_tmap(&msc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, cache, 2, ds, sr, bs, 0))
                 return cudaErrorInvalidValue;
-            static const cudaError_t attr = set_smem_attrs(decode_tc_kernel<true>, dec_smem<true>());
+            if (Q != 1) return cudaErrorInvalidValue;   // FP8 rows: one query per sequence
+            static const cudaError_t attr = set_smem_attrs(decode_tc_kernel<true, false>, dec_smem<true>());
             if (attr != cudaSuccess) return attr;
-            e = launch_pdl(decode_tc_kernel<true>, dim3(2 * P), dim3(DecCfg<true>::kThreads), dec_smem<true>(), s,
+            e = launch_pdl(decode_tc_kernel<true, false>, dim3(2 * P), dim3(DecCfg<true>::kThreads), dec_smem<true>(), s,
                            m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h, seqs, B, Q, (int)(stream_once ? 1 : 0),
                            (long long)cache_rows, scale_log2, ws.part_o, ws.part_ml, (const uint8_t*)uv,
                            (long long)kTiledWeightBytes, err_code, err_detail);
@@ -1404,19 +1433,8 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     {
         // merge of the pieces fused with o[v,h,:] = W_UV[h] o_lat[v,h,:]
         ProfScope ps(s, "tc_merge_w_uv");
-        if (NV <= 32) {
-            static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32>, merge_smem<32>());
-            if (attr != cudaSuccess) return attr;
-            e = launch_pdl(merge_wuv_kernel<32>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                           seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o,
-                           128LL * 128, 128LL, err_code, err_detail);
-        } else {
-            static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64>, merge_smem<64>());
-            if (attr != cudaSuccess) return attr;
-            e = launch_pdl(merge_wuv_kernel<64>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                           uv, seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o,
-                           128LL * 128, 128LL, err_code, err_detail);
-        }
+        e = Q > 1 ? launch_merge<true>(NV, uv, seqs, P, B, Q, ws, o, err_code, err_detail, s)
+                  : launch_merge<false>(NV, uv, seqs, P, B, Q, ws, o, err_code, err_detail, s);
     }
     return e;
 }

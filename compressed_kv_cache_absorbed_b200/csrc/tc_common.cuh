@@ -97,7 +97,7 @@ __device__ __forceinline__ bool mbar_try_cluster(uint64_t* bar, uint32_t parity)
 // shorten it (mla_set_wait_limit); every file that includes this header has its own copy,
 // which set_wait_limit_of_this_file() sets on the current device.
 constexpr uint32_t kDefaultWaitLimit = 1u << 22;
-static __device__ uint32_t g_wait_limit = kDefaultWaitLimit;
+static __constant__ uint32_t g_wait_limit = kDefaultWaitLimit;   // constant bank: read as an operand
 
 static inline cudaError_t set_wait_limit_of_this_file(uint32_t polls) {
     return cudaMemcpyToSymbol(g_wait_limit, &polls, sizeof polls);
