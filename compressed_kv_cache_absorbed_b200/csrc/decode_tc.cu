@@ -35,7 +35,8 @@
 //
 // Work split: the tiles of all sequences, in order, are cut into equal ranges, one per
 // cluster; a range may hold pieces of several sequences.  Each piece writes an
-// un-normalised partial (O, running max, row sum) that the merge kernel combines.
+// partial (its normalised output O / l in fp16, its running max and row sum) that the merge
+// kernel combines.
 // Every wait is bounded; a timeout latches an error and the kernel drains and exits.
 #include <math.h>
 
@@ -247,7 +248,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                  const __nv_bfloat16* __restrict__ q_rope, long long sQr_b, long long sQr_h,
                  const SeqSrc src, int B, int Q_arg, int stream_once, long long cache_rows,
                  float scale_log2,
-                 float* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
+                 __half* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
     constexpr int kStages = DecCfg<kF8>::kStages, kF8Stages = DecCfg<kF8>::kF8Stages;
     const int Q = kSib ? Q_arg : 1;   // queries per sequence (sibling clusters)
@@ -824,30 +825,30 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                 ptx::tc_fence_before();
                 ptx::mbar_arrive(&p_ready[pb]);
                 if (j + 1 == cur.j1) {
-                    // piece epilogue: un-normalised O_r -> part_o[slot][h][c] (each half
-                    // writes 128 columns); (m, l) from CTA 0
+                    // piece epilogue: this piece's normalised output O_r / l -> part_o[slot][h][c]
+                    // as fp16 (each half writes 128 columns, a thread 64 contiguous bytes of
+                    // its head's row at a time); (m, l) from CTA 0
                     const float l_all = l_run + pair_exchange(l_run);
                     if (!ok) break;
                     if (!uwait(&o_done[g & 1], (g >> 1) & 1)) { ok = false; break; }
                     ptx::tc_fence_after();
-                    // fragment order: four threads hold 32 contiguous bytes of one head's row,
-                    // so every store instruction writes whole sectors
-                    const int hq = sub * 32 + (lane >> 2), cq = 2 * (lane & 3);
+                    const float inv_l = 1.f / l_all;   // l_all >= 1: the maximum's own p is 1
+                    __half* po = part_o + ((long long)cur.slot * 128 + h) * 512 + 256 * rank;
 #pragma unroll 1
-                    for (int k = 0; k < 2; ++k) {
-                        float* poA = part_o + ((long long)cur.slot * 128 + hq + 16 * k) * 512 + 256 * rank + cq;
-                        float* poB = poA + 8 * 512;
-#pragma unroll 1
-                        for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
-                            uint32_t r[16];
-                            ptx::tmem_ld16x256b_x4(lane_addr + ((uint32_t)(16 * k) << 16) + kColO + c0, r);
-                            ptx::tmem_wait_ld();
+                    for (int c0 = 128 * half; c0 < 128 * half + 128; c0 += 32) {
+                        uint32_t r[32];
+                        ptx::tmem_ld32(lane_addr + kColO + c0, r);
+                        ptx::tmem_wait_ld();
+                        uint32_t hw[16];
 #pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                *(uint2*)(poA + c0 + 8 * j) = make_uint2(r[4 * j], r[4 * j + 1]);
-                                *(uint2*)(poB + c0 + 8 * j) = make_uint2(r[4 * j + 2], r[4 * j + 3]);
-                            }
+                        for (int j = 0; j < 16; ++j) {
+                            const float a = fminf(fmaxf(__uint_as_float(r[2 * j]) * inv_l, -65504.f), 65504.f);
+                            const float b = fminf(fmaxf(__uint_as_float(r[2 * j + 1]) * inv_l, -65504.f), 65504.f);
+                            hw[j] = ptx::pack_f16(a, b);
                         }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q)
+                            *(uint4*)(po + c0 + 8 * q) = make_uint4(hw[4 * q], hw[4 * q + 1], hw[4 * q + 2], hw[4 * q + 3]);
                     }
                     if (rank == 0 && half == 0) {
                         part_ml[((long long)cur.slot * 128 + h) * 2] = m_run;
@@ -871,8 +872,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 }
 
 // ------------------------------------------------------------- merge + W_UV
-// o[v,h,:] = W_UV[h] o_lat[v,h,:],  o_lat[v,h,c] = sum_p 2^(m_p - M) O_p[h,c] / sum_p 2^(m_p - M) l_p
-// over the pieces p of query v (M = max_p m_p; a query with no row gives o = 0); query v is
+// o[v,h,:] = W_UV[h] o_lat[v,h,:],  o_lat[v,h,c] = sum_p 2^(m_p - M) l_p Ob_p[h,c] / sum_p 2^(m_p - M) l_p
+// over the pieces p of query v, Ob_p = O_p / l_p being piece p's normalised output (fp16)
+// (M = max_p m_p; a query with no row gives o = 0); query v is
 // query v % Q of sequence v / Q.  One CTA per (head h, block of BN queries).  Thread 0 starts the bulk loads of the tiled
 // W_UV[h] (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
 // then merge the partials of their rows (warp per row, lane per 16 columns) straight into
@@ -887,7 +889,7 @@ constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 template <int BN, bool kSib>
 __global__ void __launch_bounds__(kMergeThreads, 1)
 merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B, int Q_arg,
-                 const float* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
+                 const __half* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
                  long long sO_b, long long sO_h, int* err_code, long long* err_detail) {
     extern __shared__ uint8_t merge_smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)merge_smem_raw + 1023) & ~(uintptr_t)1023);
@@ -982,6 +984,8 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
     pdl_wait();   // the partials come from the decode kernel
 
     constexpr int kRowsPerWarp = BN / kW;
+    // rows merged per load round: the requests of kRound rows are in flight together
+    constexpr int kRound = kRowsPerWarp < 2 ? kRowsPerWarp : 2;
     int t0r[kRowsPerWarp], t1r[kRowsPerWarp];
 #pragma unroll
     for (int i = 0; i < kRowsPerWarp; ++i) {
@@ -989,82 +993,102 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         t0r[i] = v < NV ? s_pos[0][warp + kW * i] : 0;
         t1r[i] = v < NV ? s_pos[1][warp + kW * i] : 0;
     }
+    // Piece p of a row holds its normalised partial O_p / l_p (fp16, 16 columns per lane)
+    // and (m_p, l_p); piece 0 (from range t0 / per) is in slot v, piece p > 0 continues the
+    // query in range t0 / per + p, i.e. in sibling cluster (t0 / per + p) Q + tq, and is in
+    // slot NV + that cluster.  The weight of piece p is 2^(m_p - M) l_p.
+#pragma unroll 1
+    for (int i0 = 0; i0 < kRowsPerWarp; i0 += kRound) {
+        float2 ml[kRound];
+        uint4 x[kRound][4][2];
+        int np[kRound], cfirst[kRound];
+        long long slot_base[kRound];   // slot of piece p > 0: slot_base + p * Q
+        auto slot_of = [&](int k, int p) -> long long {
+            return p == 0 ? (long long)(n0 + warp + kW * (i0 + k)) : slot_base[k] + (long long)p * Q;
+        };
+        // requests of every row of the round: (m, l) of up to 32 pieces (lane p) and the
+        // first four pieces' partial rows
 #pragma unroll
-    for (int i = 0; i < kRowsPerWarp; ++i) {
-        const int r = warp + kW * i, v = n0 + r, tq = kSib ? v % Q : 0;
-        const int t0 = t0r[i], t1 = t1r[i];
-        float acc[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) acc[k] = 0.f;
-        if (t1 > t0) {
-            // piece 0 (from range t0 / per) is in slot v; piece p > 0 continues the query in
-            // range t0 / per + p, i.e. in sibling cluster (t0 / per + p) Q + tq, and is in slot
-            // NV + that cluster
-            const int cfirst = t0 / per;
-            const int np = (t1 - 1) / per - cfirst + 1;
-            auto slot_of = [&](int p) -> long long {
-                return p == 0 ? v : kSib ? NV + (long long)(cfirst + p) * Q + tq : B + cfirst + p;
-            };
-            // (m, l) of up to 32 pieces (lane p) and the first 4 pieces' partial rows are
-            // requested together; the weights need the maximum, the loads do not
-            float2 ml = lane < np ? *(const float2*)(part_ml + (slot_of(lane) * 128 + h) * 2)
-                                  : make_float2(-INFINITY, 0.f);
-            float4 x[4][4];
+        for (int k = 0; k < kRound; ++k) {
+            const int i = i0 + k, v = n0 + warp + kW * i, tq = kSib ? v % Q : 0;
+            const int t0 = t0r[i], t1 = t1r[i];
+            cfirst[k] = t1 > t0 ? t0 / per : 0;
+            np[k] = t1 > t0 ? (t1 - 1) / per - cfirst[k] + 1 : 0;
+            slot_base[k] = kSib ? NV + (long long)cfirst[k] * Q + tq : (long long)B + cfirst[k];
+            ml[k] = lane < np[k] ? *(const float2*)(part_ml + (slot_of(k, lane) * 128 + h) * 2)
+                                 : make_float2(-INFINITY, 0.f);
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-                const float4* src = (const float4*)(part_o + (slot_of(q < np ? q : 0) * 128 + h) * 512 + 16 * lane);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) x[q][v] = q < np ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
+                const uint4* src =
+                    (const uint4*)(part_o + (slot_of(k, q < np[k] ? q : 0) * 128 + h) * 512 + 16 * lane);
+                x[k][q][0] = q < np[k] ? src[0] : make_uint4(0, 0, 0, 0);
+                x[k][q][1] = q < np[k] ? src[1] : make_uint4(0, 0, 0, 0);
             }
-            float M = ml.x;
-            for (int p = 32 + lane; p < np; p += 32) M = fmaxf(M, part_ml[(slot_of(p) * 128 + h) * 2]);
+        }
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-            const float w_lane = lane < np ? exp2f(ml.x - M) : 0.f;
-            float L = w_lane * ml.y;
-            for (int p = 32 + lane; p < np; p += 32) {
-                const float2 v = *(const float2*)(part_ml + (slot_of(p) * 128 + h) * 2);
-                L += exp2f(v.x - M) * v.y;
-            }
+        for (int k = 0; k < kRound; ++k) {
+            const int r = warp + kW * (i0 + k);
+            float acc[16];
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
-            for (int p0 = 0;; p0 += 4) {
+            for (int c = 0; c < 16; ++c) acc[c] = 0.f;
+            if (np[k] > 0) {
+                float M = ml[k].x;
+                for (int p = 32 + lane; p < np[k]; p += 32) M = fmaxf(M, part_ml[(slot_of(k, p) * 128 + h) * 2]);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int p = p0 + q;
-                    float w = __shfl_sync(0xffffffffu, w_lane, p & 31);
-                    if (p >= 32) w = p < np ? exp2f(part_ml[(slot_of(p) * 128 + h) * 2] - M) : 0.f;
-                    if (p >= np) w = 0.f;
+                for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+                const float w_lane = lane < np[k] ? exp2f(ml[k].x - M) * ml[k].y : 0.f;
+                float L = w_lane;
+                for (int p = 32 + lane; p < np[k]; p += 32) {
+                    const float2 v2 = *(const float2*)(part_ml + (slot_of(k, p) * 128 + h) * 2);
+                    L += exp2f(v2.x - M) * v2.y;
+                }
 #pragma unroll
-                    for (int v = 0; v < 4; ++v) {
-                        acc[4 * v] = fmaf(w, x[q][v].x, acc[4 * v]);
-                        acc[4 * v + 1] = fmaf(w, x[q][v].y, acc[4 * v + 1]);
-                        acc[4 * v + 2] = fmaf(w, x[q][v].z, acc[4 * v + 2]);
-                        acc[4 * v + 3] = fmaf(w, x[q][v].w, acc[4 * v + 3]);
+                for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+                for (int p0 = 0;; p0 += 4) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int p = p0 + q;
+                        float w = __shfl_sync(0xffffffffu, w_lane, p & 31);
+                        if (p >= 32 && p < np[k]) {
+                            const float2 v2 = *(const float2*)(part_ml + (slot_of(k, p) * 128 + h) * 2);
+                            w = exp2f(v2.x - M) * v2.y;
+                        }
+                        if (p >= np[k]) w = 0.f;
+#pragma unroll
+                        for (int hv = 0; hv < 2; ++hv) {
+                            const uint32_t wd[4] = {x[k][q][hv].x, x[k][q][hv].y, x[k][q][hv].z, x[k][q][hv].w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&wd[e]));
+                                acc[8 * hv + 2 * e] = fmaf(w, f.x, acc[8 * hv + 2 * e]);
+                                acc[8 * hv + 2 * e + 1] = fmaf(w, f.y, acc[8 * hv + 2 * e + 1]);
+                            }
+                        }
+                    }
+                    if (p0 + 4 >= np[k]) break;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {   // the next four pieces
+                        const int p = p0 + 4 + q;
+                        const uint4* src =
+                            (const uint4*)(part_o + (slot_of(k, p < np[k] ? p : 0) * 128 + h) * 512 + 16 * lane);
+                        x[k][q][0] = p < np[k] ? src[0] : make_uint4(0, 0, 0, 0);
+                        x[k][q][1] = p < np[k] ? src[1] : make_uint4(0, 0, 0, 0);
                     }
                 }
-                if (p0 + 4 >= np) break;
+                const float inv = 1.f / L;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {   // the next four pieces
-                    const int p = p0 + 4 + q;
-                    const float4* src = (const float4*)(part_o + (slot_of(p < np ? p : 0) * 128 + h) * 512 + 16 * lane);
-#pragma unroll
-                    for (int v = 0; v < 4; ++v) x[q][v] = p < np ? src[v] : make_float4(0.f, 0.f, 0.f, 0.f);
-                }
+                for (int c = 0; c < 16; ++c) acc[c] *= inv;
             }
-            const float inv = 1.f / L;
+            // columns 16 lane .. +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
+            uint8_t* rowp = sB + (lane >> 2) * (BN * 128) + r * 128;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) acc[k] *= inv;
-        }
-        // columns 16 lane .. +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
-        uint8_t* rowp = sB + (lane >> 2) * (BN * 128) + r * 128;
-#pragma unroll
-        for (int hv = 0; hv < 2; ++hv) {
-            const int u = 2 * (lane & 3) + hv;
-            *(uint4*)(rowp + ((u ^ (r & 7)) << 4)) =
-                make_uint4(ptx::pack_bf16(acc[8 * hv], acc[8 * hv + 1]), ptx::pack_bf16(acc[8 * hv + 2], acc[8 * hv + 3]),
-                           ptx::pack_bf16(acc[8 * hv + 4], acc[8 * hv + 5]),
-                           ptx::pack_bf16(acc[8 * hv + 6], acc[8 * hv + 7]));
+            for (int hv = 0; hv < 2; ++hv) {
+                const int u = 2 * (lane & 3) + hv;
+                *(uint4*)(rowp + ((u ^ (r & 7)) << 4)) =
+                    make_uint4(ptx::pack_bf16(acc[8 * hv], acc[8 * hv + 1]), ptx::pack_bf16(acc[8 * hv + 2], acc[8 * hv + 3]),
+                               ptx::pack_bf16(acc[8 * hv + 4], acc[8 * hv + 5]),
+                               ptx::pack_bf16(acc[8 * hv + 6], acc[8 * hv + 7]));
+            }
         }
     }
     ptx::fence_proxy_async_smem();   // the tensor cores read what the threads wrote
@@ -1284,13 +1308,13 @@ cudaError_t launch_merge(int NV, const __nv_bfloat16* uv, const SeqSrc& seqs, in
         static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32, kSib>, merge_smem<32>());
         if (attr != cudaSuccess) return attr;
         return launch_pdl(merge_wuv_kernel<32, kSib>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                          seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
+                          seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
                           err_code, err_detail);
     }
     static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64, kSib>, merge_smem<64>());
     if (attr != cudaSuccess) return attr;
     return launch_pdl(merge_wuv_kernel<64, kSib>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                      uv, seqs, P, B, Q, (const float*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
+                      uv, seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
                       err_code, err_detail);
 }
 
@@ -1336,7 +1360,7 @@ size_t decode_ws_bytes(int B, int num_sms) {
     const size_t P = (size_t)(num_sms / 2);
     const size_t slots = (size_t)B + P + 1;
     auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
-    return up((size_t)B * 128 * 512 * 2) + up(slots * 512 * 128 * 4) + up(slots * 128 * 2 * 4);
+    return up((size_t)B * 128 * 512 * 2) + up(slots * 512 * 128 * 2) + up(slots * 128 * 2 * 4);
 }
 
 DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
@@ -1351,7 +1375,7 @@ DecodeWs carve_decode_ws(char* base, int B, int num_sms) {
         return p;
     };
     w.q_lat = (__nv_bfloat16*)take((size_t)B * 128 * 512 * 2);
-    w.part_o = (float*)take(slots * 512 * 128 * 4);
+    w.part_o = (__half*)take(slots * 512 * 128 * 2);
     w.part_ml = (float*)take(slots * 128 * 2 * 4);
     w.max_parts = (int)slots;
     return w;

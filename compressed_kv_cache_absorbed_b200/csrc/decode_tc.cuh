@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -26,7 +27,7 @@ constexpr int kF8ScaleOffset = 640;
 // Workspace pieces of the tensor-core decode (all device memory, carved by the caller).
 struct DecodeWs {
     __nv_bfloat16* q_lat;   // [B, H, d_c] absorbed query, bf16
-    float* part_o;          // [max_parts, H, d_c] un-normalised partial o_lat
+    __half* part_o;         // [max_parts, H, d_c] a piece's normalised partial o_lat (fp16)
     float* part_ml;         // [max_parts, H, 2] running max (log2 domain) and sum
     int max_parts;
 };
