@@ -1002,7 +1002,7 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         float2 ml[kRound];
         uint4 x[kRound][4][2];
         int np[kRound], cfirst[kRound];
-        long long slot_base[kRound];   // slot of piece p > 0: slot_base + p * Q
+        long long slot_base[kRound] = {};   // slot of piece p > 0: slot_base + p * Q
         auto slot_of = [&](int k, int p) -> long long {
             return p == 0 ? (long long)(n0 + warp + kW * (i0 + k)) : slot_base[k] + (long long)p * Q;
         };
