@@ -59,31 +59,36 @@ constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads 
 constexpr int kBarBytes = 256 + 2048 + 256;
 // FP8 cache rows (see decode_tc.cuh): per tile and CTA, this CTA's 256 codes (two 128-byte
 // boxes, 128-byte swizzle), its 32 rotary columns (bf16, 64-byte swizzle) and the 64 rows'
-// 16-byte scale fields (the fp32 scale first)
+// 16-byte scale fields (the fp32 scale first).  They land in place in a stage one KB larger
+// than a bf16 tile: the codes in the upper half of the latent area (fp16 boxes 2 and 3), the
+// rotary box where the tile keeps it, the scales after it; the dequantisation warps then
+// expand the codes into the four fp16 latent boxes.
 constexpr int kF8CodeBytes = kT * 128;
-constexpr int kF8StageBytes = 2 * kF8CodeBytes + kRopeBytes + kT * 16;
-static_assert(kF8StageBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment of the swizzled boxes");
+constexpr int kF8CodeOffset = 2 * kChunkBytes;        // code boxes at fp16 boxes 2, 3
+constexpr int kF8StageScaleOffset = kTileBytes;        // after the rotary box
+constexpr int kF8TileBytes = kTileBytes + kT * 16;     // 37 KB
+constexpr int kF8LoadBytes = 2 * kF8CodeBytes + kRopeBytes + kT * 16;
+static_assert(kF8TileBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment of the swizzled boxes");
 
 // Two variants of the kernel.  bf16 cache rows: TMA fills a ring of kStages tiles that the
-// MMAs read directly.  FP8 cache rows: TMA fills a ring of kF8Stages FP8 stages, and two
-// dequantisation warps turn each into an fp16 tile (code x scale) of the same layout in the
-// tile ring; the latent MMAs then run on fp16 operands (q_lat and P in fp16 too).
+// MMAs read directly.  FP8 cache rows: TMA fills each stage with FP8 data and two
+// dequantisation warps turn it in place into an fp16 tile (code x scale) of the same layout;
+// the latent MMAs then run on fp16 operands (q_lat and P in fp16 too).
 template <bool kF8> struct DecCfg;
 template <> struct DecCfg<false> {
-    static constexpr int kStages = 4, kF8Stages = 0;
+    static constexpr int kStages = 4, kStageBytes = kTileBytes;
     static constexpr int kThreads = 448;   // producer, MMA, 4 sender and 8 softmax warps
 };
 template <> struct DecCfg<true> {
-    static constexpr int kStages = 3, kF8Stages = 2;
+    static constexpr int kStages = 4, kStageBytes = kF8TileBytes;
     static constexpr int kThreads = 512;   // + 2 dequantisation warps
 };
-// tiles, FP8 stages, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the
-// peer).  The dynamic shared memory of a kernel without static shared memory starts
-// 1024-byte aligned (the 128-byte swizzle needs it); the kernel checks this instead of padding.
+// tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer).  The
+// dynamic shared memory of a kernel without static shared memory starts 1024-byte aligned
+// (the 128-byte swizzle needs it); the kernel checks this instead of padding.
 template <bool kF8>
 constexpr int dec_smem() {
-    return DecCfg<kF8>::kStages * kTileBytes + DecCfg<kF8>::kF8Stages * kF8StageBytes + 4 * kXBytes + kQRopeBytes +
-           kBarBytes;
+    return DecCfg<kF8>::kStages * DecCfg<kF8>::kStageBytes + 4 * kXBytes + kQRopeBytes + kBarBytes;
 }
 static_assert(dec_smem<false>() <= 232448, "decode kernel shared memory over the 227 KB limit");
 static_assert(dec_smem<true>() <= 232448, "FP8 decode kernel shared memory over the 227 KB limit");
@@ -250,7 +255,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                  float scale_log2,
                  __half* __restrict__ part_o, float* __restrict__ part_ml, const uint8_t* __restrict__ next_weights,
                  long long next_weight_bytes, int* err_code, long long* err_detail) {
-    constexpr int kStages = DecCfg<kF8>::kStages, kF8Stages = DecCfg<kF8>::kF8Stages;
+    constexpr int kStages = DecCfg<kF8>::kStages, kStride = DecCfg<kF8>::kStageBytes;
     const int Q = kSib ? Q_arg : 1;   // queries per sequence (sibling clusters)
     constexpr int kThreads = DecCfg<kF8>::kThreads;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -263,8 +268,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     const int len0 = threadIdx.x < B ? src.raw_len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
-    uint8_t* f8 = smem + kStages * kTileBytes;      // [kF8Stages] FP8 stages (FP8 cache rows)
-    uint8_t* xbuf = f8 + kF8Stages * kF8StageBytes; // [2] partial scores received from the peer
+    uint8_t* xbuf = smem + kStages * kStride;      // [2] partial scores received from the peer
     uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
     uint8_t* qrope = xstage + 2 * kXBytes;         // rotary query columns (A operand, 64-byte swizzle)
     uint64_t* bars = (uint64_t*)(qrope + kQRopeBytes);
@@ -285,8 +289,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     uint64_t* xs_ready = s_full + 12;  // [2] all 128 rows of xstage[g & 1] written
     uint64_t* xs_free = s_full + 14;   // [2] the local softmax has read xstage[g & 1]
     uint64_t* pair_bar = s_full + 16;  // [4] the two softmax warps of a subpartition
-    uint64_t* f8_full = s_full + 20;   // [2] an FP8 stage landed (FP8 rows)
-    uint64_t* f8_empty = s_full + 22;  // [2] an FP8 stage was dequantised (FP8 rows)
+    uint64_t* f8_full = s_full + 20;   // [4] a stage's FP8 data landed (FP8 rows)
     float* pair_val = (float*)(s_full + 24);   // [2][2][128] values the two warps swap
     uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
@@ -302,10 +305,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             ptx::mbar_init(&tile_full[s], kF8 ? 64 : 1);   // the dequantisation warps, or TMA
             ptx::mbar_init(&tile_empty[s], 1);
         }
-        for (int s = 0; s < kF8Stages; ++s) {
-            ptx::mbar_init(&f8_full[s], 1);
-            ptx::mbar_init(&f8_empty[s], 64);
-        }
+        if (kF8)
+            for (int s = 0; s < kStages; ++s) ptx::mbar_init(&f8_full[s], 1);
         ptx::mbar_init(s_full, 1);
         ptx::mbar_init(s_free, 128);
         ptx::mbar_init(&p_ready[0], 256);
@@ -406,13 +407,13 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     if (warp == 0) {
         // ------------------------------------------------------------ TMA producer
         if (lane == 0) {
-            // bf16 rows: the tile ring itself; FP8 rows: the FP8 stages the dequantisation
-            // warps read
-            constexpr int NR = kF8 ? kF8Stages : kStages;
-            constexpr int kRingBytes = kF8 ? kF8StageBytes : kTileBytes;
-            uint8_t* ring = kF8 ? f8 : tiles;
+            // bf16 rows complete the tile itself; FP8 rows complete f8_full, on which the
+            // dequantisation warps wait
+            constexpr int NR = kStages;
+            constexpr int kRingBytes = kF8 ? kF8LoadBytes : kTileBytes;
+            uint8_t* ring = tiles;
             uint64_t* ring_full = kF8 ? f8_full : tile_full;
-            uint64_t* ring_empty = kF8 ? f8_empty : tile_empty;
+            uint64_t* ring_empty = tile_empty;
             ptx::tma_prefetch(&tm_cache);
             ptx::tma_prefetch(&tm_rope);
             if (kF8) ptx::tma_prefetch(&tm_scale);
@@ -428,7 +429,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         fail(err_code, err_detail, abort_flag, 1);
                         break;
                     }
-                    uint8_t* dst = ring + s * kRingBytes;
+                    uint8_t* dst = ring + s * kStride;
                     long long row_l = sg.row0 + (long long)j * kT;
                     if (src.block_table) {
                         const long long page = src.block_table[(long long)sg.b * src.bt_stride + j];
@@ -449,12 +450,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                         // elements 256 + 32 rank ..) and the scale fields (fp32 element 160)
 #pragma unroll
                         for (int i = 0; i < 2; ++i)
-                            ptx::tma_load_2d_hint(dst + i * kF8CodeBytes, &tm_cache, &ring_full[s],
+                            ptx::tma_load_2d_hint(dst + kF8CodeOffset + i * kF8CodeBytes, &tm_cache, &ring_full[s],
                                                   256 * (int)rank + 128 * i, row, stream_policy);
-                        ptx::tma_load_2d_hint(dst + 2 * kF8CodeBytes, &tm_rope, &ring_full[s], 256 + 32 * (int)rank,
+                        ptx::tma_load_2d_hint(dst + 4 * kChunkBytes, &tm_rope, &ring_full[s], 256 + 32 * (int)rank,
                                               row, stream_policy);
-                        ptx::tma_load_2d_hint(dst + 2 * kF8CodeBytes + kRopeBytes, &tm_scale, &ring_full[s], 160, row,
-                                              stream_policy);
+                        ptx::tma_load_2d_hint(dst + kF8StageScaleOffset, &tm_scale, &ring_full[s], 160, row, stream_policy);
                     } else {
 #pragma unroll
                         for (int i = 0; i < 4; ++i)
@@ -483,50 +483,52 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         }
     } else if (kF8 && warp >= 14) {
         // ------------------------------------------------- FP8 dequantisation (FP8 rows)
-        // 64 threads turn FP8 stage g % kF8Stages into the fp16 tile g % kStages: every 16
-        // codes of a row (one 16-byte unit of a 128-byte-swizzled code box) times the row's
-        // scale become two 16-byte units of a 128-byte-swizzled fp16 latent box, and the
-        // rotary box (bf16, 64-byte swizzle) is copied as it is (same alignment, same
-        // swizzle pattern).
+        // 64 threads expand the FP8 data of stage g % kStages in place into its fp16 tile:
+        // every 16 codes of a row (one 16-byte unit of a 128-byte-swizzled code box) times the
+        // row's scale become two 16-byte units of a 128-byte-swizzled fp16 latent box.  Code
+        // box 0 (in fp16 box 2's place) becomes fp16 boxes 0 and 1, which it does not overlap;
+        // code box 1 (in fp16 box 3's place) is read into registers by all 64 threads before
+        // any of them writes fp16 boxes 2 and 3 over both code boxes.  The rotary box landed
+        // where the tile keeps it.
         const int dt = threadIdx.x - 14 * 32;
-        constexpr int NF = kF8Stages > 0 ? kF8Stages : 1;   // (the bf16 variant never gets here)
         uint32_t g = 0;
         bool ok = true;
         Seg cur;
+        auto expand = [&](uint8_t* tl, int k, uint4 c, int box) {   // unit e = dt + 64 k of code box `box`
+            const int e = dt + 64 * k;
+            const int r = e >> 3, u = e & 7, sw = r & 7;       // row, unit within the code box
+            const float sc = *(const float*)(tl + kF8StageScaleOffset + r * 16);
+            uint4 lo, hi;
+            dequant16(c, __float2half2_rn(sc), lo, hi);
+            // latent columns 128 box + 16 u .. + 15: fp16 box 2 box + (u >> 2), units 2 (u & 3), + 1
+            uint8_t* rowp = tl + (2 * box + (u >> 2)) * kChunkBytes + r * 128;
+            const int a = 2 * (u & 3);
+            *(uint4*)(rowp + ((a ^ sw) << 4)) = lo;
+            *(uint4*)(rowp + (((a + 1) ^ sw) << 4)) = hi;
+        };
+        auto code_unit = [&](const uint8_t* tl, int k, int box) {
+            const int e = dt + 64 * k;
+            const int r = e >> 3, u = e & 7;
+            return *(const uint4*)(tl + kF8CodeOffset + box * kF8CodeBytes + r * 128 + ((u ^ (r & 7)) << 4));
+        };
         while (ok && !*abort_flag && it.next(cur)) {
             for (int j = cur.j0; j < cur.j1; ++j, ++g) {
-                const int s = g % NF, d = g % kStages;
-                if (!ptx::mbar_wait(&f8_full[s], (g / NF) & 1, abort_flag) ||
-                    (g >= (uint32_t)kStages && !ptx::mbar_wait(&tile_empty[d], ((g / kStages) - 1) & 1, abort_flag))) {
+                const int s = g % kStages;
+                if (!ptx::mbar_wait(&f8_full[s], (g / kStages) & 1, abort_flag)) {
                     ok = false;
                     break;
                 }
-                const uint8_t* st = f8 + s * kF8StageBytes;
-                uint8_t* tl = tiles + d * kTileBytes;
+                uint8_t* tl = tiles + s * kStride;
 #pragma unroll 4
-                for (int k = 0; k < 16; ++k) {
-                    const int e = dt + 64 * k;          // 0 .. 1023: (row, code unit)
-                    const int r = e >> 4, u = e & 15;   // code box u >> 3, unit u & 7
-                    const int sw = r & 7;
-                    const uint4 c = *(const uint4*)(st + (u >> 3) * kF8CodeBytes + r * 128 + (((u & 7) ^ sw) << 4));
-                    const float sc = *(const float*)(st + 2 * kF8CodeBytes + kRopeBytes + r * 16);
-                    uint4 lo, hi;
-                    dequant16(c, __float2half2_rn(sc), lo, hi);
-                    // latent columns 16 u .. 16 u + 15 of this CTA: fp16 box u >> 2, units
-                    // 2 (u & 3) and 2 (u & 3) + 1
-                    uint8_t* rowp = tl + (u >> 2) * kChunkBytes + r * 128;
-                    const int a = 2 * (u & 3);
-                    *(uint4*)(rowp + ((a ^ sw) << 4)) = lo;
-                    *(uint4*)(rowp + (((a + 1) ^ sw) << 4)) = hi;
-                }
+                for (int k = 0; k < 8; ++k) expand(tl, k, code_unit(tl, k, 0), 0);
+                uint4 c1[8];
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int i = dt + 64 * k;   // 16-byte units of the 4 KB rotary box
-                    ((uint4*)(tl + 4 * kChunkBytes))[i] = ((const uint4*)(st + 2 * kF8CodeBytes))[i];
-                }
+                for (int k = 0; k < 8; ++k) c1[k] = code_unit(tl, k, 1);
+                ptx::named_barrier_sync(8, 64);   // every code of the stage is read
+#pragma unroll
+                for (int k = 0; k < 8; ++k) expand(tl, k, c1[k], 1);
                 ptx::fence_proxy_async_smem();   // read by the tensor cores
-                ptx::mbar_arrive(&f8_empty[s]);
-                ptx::mbar_arrive(&tile_full[d]);
+                ptx::mbar_arrive(&tile_full[s]);
             }
         }
         if (!ok) fail(err_code, err_detail, abort_flag, 6);
@@ -558,7 +560,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                 // ---- O of tile g
                 if (g < s_g && ptx::mbar_test(&p_ready[g & 1], (g >> 1) & 1)) {
                     ptx::tc_fence_after();
-                    const uint32_t v = ptx::smem_u32(tiles + (g % kStages) * kTileBytes);
+                    const uint32_t v = ptx::smem_u32(tiles + (g % kStages) * kStride);
                     const bool first = (o_j == sg.j0);
 #pragma unroll
                     for (int k = 0; k < kT / 16; ++k)
@@ -585,7 +587,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     if ((!first || q_ok) && ptx::mbar_test(&tile_full[st], (s_g / kStages) & 1) &&
                         (s_g == 0 || ptx::mbar_test(s_free, (s_g - 1) & 1))) {
                         ptx::tc_fence_after();
-                        const uint32_t t = ptx::smem_u32(tiles + st * kTileBytes);
+                        const uint32_t t = ptx::smem_u32(tiles + st * kStride);
 #pragma unroll
                         for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
                             ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
@@ -813,7 +815,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     // (another sequence, unused capacity, the rest of a page), possibly NaN or
                     // Inf bit patterns, which the O MMA would turn into NaN even with P = 0:
                     // zero them (the score MMA that also read them has completed).
-                    uint4* t4 = (uint4*)(tiles + (g % kStages) * kTileBytes);
+                    uint4* t4 = (uint4*)(tiles + (g % kStages) * kStride);
                     const int tid = (warp - 6) * 32 + lane;   // 0 .. 255 over the softmax warps
                     for (int e = tid; e < (kT - n_valid) * 4 * 8; e += 256) {
                         const int r = n_valid + (e >> 5), c = (e >> 3) & 3, u = e & 7;
@@ -874,12 +876,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 // ------------------------------------------------------------- merge + W_UV
 // o[v,h,:] = W_UV[h] o_lat[v,h,:],  o_lat[v,h,c] = sum_p 2^(m_p - M) l_p Ob_p[h,c] / sum_p 2^(m_p - M) l_p
 // over the pieces p of query v, Ob_p = O_p / l_p being piece p's normalised output (fp16)
-// (M = max_p m_p; a query with no row gives o = 0); query v is
-// query v % Q of sequence v / Q.  One CTA per (head h, block of BN queries).  Thread 0 starts the bulk loads of the tiled
-// W_UV[h] (128 x 512 bf16, the A operand) before waiting for the decode kernel; the sixteen warps
-// then merge the partials of their rows (warp per row, lane per 16 columns) straight into
-// the B operand in shared memory (K-major, 128-byte swizzle, as TMA would lay it out);
-// one thread issues the 32 MMAs (M = 128, N = BN) and four warps store D = o[:, h, :]^T.
+// (M = max_p m_p; a query with no row gives o = 0); query v is query v % Q of sequence
+// v / Q.  One CTA per (head h, block of BN queries).  Thread 0 starts the bulk loads of the
+// tiled W_UV[h] (128 x 512 fp16, the A operand) before waiting for the decode kernel; the
+// sixteen warps then merge the partials of their rows (lane per 16 columns, two rows per
+// load round) straight into the B operand in shared memory as fp16 (K-major, 128-byte
+// swizzle, as TMA would lay it out); one thread issues the 32 MMAs (M = 128, N = BN, fp16
+// operands, fp32 accumulation) and four warps store D = o[:, h, :]^T as bf16.  fp16 keeps
+// o_lat's rounding at 2^-12 (bf16 would add 2^-9 after the partials' own fp16 rounding).
 constexpr int kMergeThreads = 512;
 constexpr int kMergeABytes = 8 * 128 * 128;   // W_UV[h]: 8 chunks of 128 rows x 64 columns
 
@@ -1079,15 +1083,18 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
 #pragma unroll
                 for (int c = 0; c < 16; ++c) acc[c] *= inv;
             }
-            // columns 16 lane .. +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
+            // o_lat as fp16 (saturated), the B operand of the W_UV product: columns 16 lane ..
+            // +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
             uint8_t* rowp = sB + (lane >> 2) * (BN * 128) + r * 128;
+#pragma unroll
+            for (int c = 0; c < 16; ++c) acc[c] = fminf(fmaxf(acc[c], -65504.f), 65504.f);
 #pragma unroll
             for (int hv = 0; hv < 2; ++hv) {
                 const int u = 2 * (lane & 3) + hv;
                 *(uint4*)(rowp + ((u ^ (r & 7)) << 4)) =
-                    make_uint4(ptx::pack_bf16(acc[8 * hv], acc[8 * hv + 1]), ptx::pack_bf16(acc[8 * hv + 2], acc[8 * hv + 3]),
-                               ptx::pack_bf16(acc[8 * hv + 4], acc[8 * hv + 5]),
-                               ptx::pack_bf16(acc[8 * hv + 6], acc[8 * hv + 7]));
+                    make_uint4(ptx::pack_f16(acc[8 * hv], acc[8 * hv + 1]), ptx::pack_f16(acc[8 * hv + 2], acc[8 * hv + 3]),
+                               ptx::pack_f16(acc[8 * hv + 4], acc[8 * hv + 5]),
+                               ptx::pack_f16(acc[8 * hv + 6], acc[8 * hv + 7]));
             }
         }
     }
@@ -1103,7 +1110,8 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
             ok = false;
         } else {
             ptx::tc_fence_after();
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, BN, 0, 0);
+            // A = W_UV[h] and B = o_lat, both fp16
+            constexpr uint32_t idesc = ptx::idesc_f16_f32(128, BN, 0, 0);
 #pragma unroll
             for (int kc = 0; kc < 8; ++kc)
 #pragma unroll
@@ -1161,7 +1169,17 @@ tile_weights_kernel(const __nv_bfloat16* __restrict__ W_UKT, const __nv_bfloat16
         else          // chunk c: W_UV[h][r][64c + 8u ..]
             src = (const uint4*)(W_UV + ((long long)h * 128 + r) * kDc + 64 * c + 8 * u);
         uint4* dst = (uint4*)((is_uv ? uv : ukt) + (((long long)h * 8 + c) * 128 + r) * 64) + (u ^ (r & 7));
-        *dst = *src;
+        uint4 x = *src;
+        if (is_uv) {   // W_UV in fp16 (the merge's product runs on fp16 operands)
+            uint32_t w[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const float lo = __uint_as_float(w[q] << 16), hi = __uint_as_float(w[q] & 0xFFFF0000u);
+                w[q] = ptx::pack_f16(fminf(fmaxf(lo, -65504.f), 65504.f), fminf(fmaxf(hi, -65504.f), 65504.f));
+            }
+            x = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        *dst = x;
     }
 }
 

@@ -43,7 +43,8 @@ constexpr size_t kTiledWeightBytes = (size_t)kH * kDc * 128 * 2;
 // chunks of 128 rows x 64 columns (16 KB), each row 128 bytes with its 16-byte units in the
 // 128-byte-swizzle order (unit u of row r at u ^ (r % 8)).
 //   ukt: chunk (t, k) = rows 128t .. +127 of W_UK^T[h] (latent index), columns 64k .. +63 (qk_nope)
-//   uv:  chunk k      = rows 0 .. 127 of W_UV[h] (v_head), columns 64k .. +63 (latent)
+//   uv:  chunk k      = rows 0 .. 127 of W_UV[h] (v_head), columns 64k .. +63 (latent), in
+//        fp16 (saturated at +-65504): the merge's W_UV product takes o_lat in fp16
 // W_UKT [H, d_c, qk_nope] and W_UV [H, v_head, d_c] are the plain layouts.
 cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_UV, __nv_bfloat16* ukt,
                             __nv_bfloat16* uv, cudaStream_t s);
