@@ -4,8 +4,10 @@
 One step = one mla_decode_absorbed call (query absorption, split-KV attention over the
 latent cache, log-sum-exp merge, W_UV) for the DeepSeek-V3-shaped workload: 32 sequences
 of 4096 cached tokens, 128 heads, d_c = 512, d_hR = 64, bf16 storage, fp32 accumulation.
-Inputs are resident in HBM when the timed region starts; L2 is flushed (256 MiB write)
-between steps, outside the per-step events.
+Inputs are resident in HBM when the timed region starts; L2 is flushed between steps,
+outside the per-step events: a 256 MiB buffer is written, then another 256 MiB buffer is
+read, so L2 holds none of the step's inputs and no dirty line of the flush is written back
+inside the next step (the write-only flush is timed too and reported beside it).
 
 Prints ONE JSON line (rank 0).  `--impl reference` times the float64 CPU oracle instead.
 Multi-GPU (torchrun): every rank decodes its own batch (weak scaling, no collective on the
@@ -36,6 +38,22 @@ METRIC = "MLA decode tokens/s + latent-cache GB/s, % roofline (H=128,d_c=512,ctx
 WORKLOAD = "v3_decode_b32_ctx4096"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 FLUSH_BYTES = 256 << 20
+
+
+class L2Flush:
+    """Evicts the step's data from L2 between steps.  The write (256 MiB, twice the L2) leaves
+    L2 full of dirty lines, which the next step would write back to HBM while it reads its
+    own data; the read of a second 256 MiB buffer that follows displaces them, so the lines
+    left in L2 are clean.  `clean=False` is the write alone."""
+
+    def __init__(self, dev, clean: bool = True):
+        self.w = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.r = torch.ones(FLUSH_BYTES // 4, dtype=torch.float32, device=dev) if clean else None
+
+    def __call__(self):
+        self.w.zero_()
+        if self.r is not None:
+            torch.sum(self.r)
 
 
 # ------------------------------------------------------------------ arithmetic
@@ -361,7 +379,10 @@ def run_reference(args, w):
 def config_of(w, world):
     return {"workload": w.name, "B_per_gpu": w.B, "ctx": w.ctx, "H": w.H, "d_c": w.d_c, "d_hR": w.d_hR,
             "qk_nope": w.qk_nope, "v_head": w.v_head, "global_batch": w.B * world,
-            "parallelism": f"replicas{world}", "l2": "flushed between steps (256 MiB write, outside the step events)",
+            "parallelism": f"replicas{world}",
+            "l2": "flushed between steps, outside the step events: 256 MiB written, then another 256 MiB read "
+                  "(no dirty flush line is written back inside a step); ms_per_step_write_only_flush is the "
+                  "same step after the write alone",
             **({"q_len": w.q_len} if w.kind == "decode_multi" else {})}
 
 
@@ -445,12 +466,13 @@ def run_ours(args, w0):
     inp = workloads.make_inputs(w)
     dev = torch.device("cuda", local)
     g, dims, weights, out, step, h2d, a, units = build_step(w, inp, dev, mla)
-    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    flush_w = L2Flush(dev, clean=False)
     stream = torch.cuda.current_stream()
 
     # warm-up
     for _ in range(args.warmup):
-        flush.zero_()
+        flush()
         step()
     torch.cuda.synchronize()
     st, det = mla.mla_get_device_error()
@@ -460,7 +482,7 @@ def run_ours(args, w0):
     clocks = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     time.sleep(0.3 if clocks else 0)
 
-    def timed_pass(profile: bool):
+    def timed_pass(profile: bool, fl=flush):
         ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
         if profile:
@@ -470,7 +492,7 @@ def run_ours(args, w0):
         torch.cuda.synchronize()
         t0 = time.time()
         for i in range(args.steps):
-            flush.zero_()
+            fl()
             ev[i][0].record(stream)
             step()
             ev[i][1].record(stream)
@@ -495,6 +517,9 @@ def run_ours(args, w0):
     # kernel's live launch duration (events between launches stop the kernels from
     # overlapping, so this pass is slower than the first)
     prof_ms, prof, _, _ = timed_pass(True)
+    # the same steps after the write-only flush (its dirty lines are written back in the step)
+    wo_ms, _, _, _ = timed_pass(False, flush_w)
+    ms_wo = max_over_ranks(float(np.median(wo_ms)))
     ms_prof = max_over_ranks(float(np.median(prof_ms)))
     clk = clocks.summary(t0, t1) if clocks else None
     if clocks:
@@ -520,7 +545,7 @@ def run_ours(args, w0):
             out_h.copy_(out, non_blocking=True)
     ev3 = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     for i in range(args.steps + args.warmup):
-        flush.zero_()
+        flush()
         j = i - args.warmup
         if j >= 0:
             ev3[j][0].record(stream)
@@ -609,6 +634,7 @@ def run_ours(args, w0):
             "roofline": roofline,
             "kernels": {k: {"launches": v[0], "avg_us": v[1] / v[0] * 1e3} for k, v in prof.items()},
             "ms_per_step_with_kernel_events": ms_prof,
+            "ms_per_step_write_only_flush": ms_wo,
             "e2e": {"value": world * units / (e2e_ms * 1e-3), "unit": unit,
                     "h2d_bytes_per_step": int(sum(v.numel() * v.element_size() for _, v in h2d)),
                     "d2h_bytes_per_step": int(out.numel() * out.element_size()), "ms_per_step": e2e_ms,

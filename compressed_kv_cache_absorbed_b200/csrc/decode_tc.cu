@@ -76,19 +76,21 @@ static_assert(kF8TileBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment
 // the latent MMAs then run on fp16 operands (q_lat and P in fp16 too).
 template <bool kF8> struct DecCfg;
 template <> struct DecCfg<false> {
-    static constexpr int kStages = 4, kStageBytes = kTileBytes;
+    static constexpr int kStages = 4, kStageBytes = kTileBytes, kXBufs = 2;
     static constexpr int kThreads = 448;   // producer, MMA, 4 sender and 8 softmax warps
 };
 template <> struct DecCfg<true> {
-    static constexpr int kStages = 4, kStageBytes = kF8TileBytes;
+    static constexpr int kStages = 4, kStageBytes = kF8TileBytes, kXBufs = 2;
     static constexpr int kThreads = 512;   // + 2 dequantisation warps
 };
-// tiles, 2 receive buffers (filled by the peer), 2 staging buffers (sent to the peer).  The
+// Shared memory: the ring of kStages tiles, kXBufs receive buffers for the peer's partial
+// scores and kXBufs staging buffers for this CTA's own (each kXBytes).  The
 // dynamic shared memory of a kernel without static shared memory starts 1024-byte aligned
 // (the 128-byte swizzle needs it); the kernel checks this instead of padding.
 template <bool kF8>
 constexpr int dec_smem() {
-    return DecCfg<kF8>::kStages * DecCfg<kF8>::kStageBytes + 4 * kXBytes + kQRopeBytes + kBarBytes;
+    return DecCfg<kF8>::kStages * DecCfg<kF8>::kStageBytes + 2 * DecCfg<kF8>::kXBufs * kXBytes + kQRopeBytes +
+           kBarBytes;
 }
 static_assert(dec_smem<false>() <= 232448, "decode kernel shared memory over the 227 KB limit");
 static_assert(dec_smem<true>() <= 232448, "FP8 decode kernel shared memory over the 227 KB limit");
@@ -268,9 +270,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     const int len0 = threadIdx.x < B ? src.raw_len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
-    uint8_t* xbuf = smem + kStages * kStride;      // [2] partial scores received from the peer
-    uint8_t* xstage = xbuf + 2 * kXBytes;          // [2] this CTA's partial scores, being sent
-    uint8_t* qrope = xstage + 2 * kXBytes;         // rotary query columns (A operand, 64-byte swizzle)
+    constexpr uint32_t kXB = DecCfg<kF8>::kXBufs;
+    uint8_t* xbuf = smem + kStages * kStride;      // [kXB] partial scores received from the peer
+    uint8_t* xstage = xbuf + kXB * kXBytes;        // [kXB] this CTA's partial scores, being sent
+    uint8_t* qrope = xstage + kXB * kXBytes;       // rotary query columns (A operand, 64-byte swizzle)
     uint64_t* bars = (uint64_t*)(qrope + kQRopeBytes);
     uint64_t* tile_full = bars;
     uint64_t* tile_empty = bars + kStages;
@@ -279,15 +282,15 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     uint64_t* p_ready = s_full + 2;    // [2] P of tile g is in P buffer g & 1
     uint64_t* o_done = s_full + 4;     // [2] the O MMAs of tile g (and all before) completed
     uint64_t* q_ready = s_full + 6;
-    // [2] the peer's partial scores for tile g landed in xbuf[g & 1]: armed locally with the
-    // byte count, completed by the peer's bulk copy
+    // [kXB] the peer's partial scores for tile g landed in xbuf[g % kXB]: armed locally with
+    // the byte count, completed by the peer's bulk copy
     uint64_t* x_full = s_full + 7;
-    // [2] the peer has read what this CTA sent into its xbuf[g & 1]; that copy therefore also
-    // finished reading this CTA's xstage[g & 1] (one arrive per peer warp)
+    // [kXB] the peer has read what this CTA sent into its xbuf[g % kXB]; that copy therefore
+    // also finished reading this CTA's xstage[g % kXB] (one arrive per peer warp)
     uint64_t* x_empty = s_full + 9;
     uint64_t* drain = s_full + 11;     // all MMAs issued by this CTA have completed
-    uint64_t* xs_ready = s_full + 12;  // [2] all 128 rows of xstage[g & 1] written
-    uint64_t* xs_free = s_full + 14;   // [2] the local softmax has read xstage[g & 1]
+    uint64_t* xs_ready = s_full + 12;  // [kXB] all 128 rows of xstage[g % kXB] written
+    uint64_t* xs_free = s_full + 14;   // [kXB] the local softmax has read xstage[g % kXB]
     uint64_t* pair_bar = s_full + 16;  // [4] the two softmax warps of a subpartition
     uint64_t* f8_full = s_full + 20;   // [4] a stage's FP8 data landed (FP8 rows)
     float* pair_val = (float*)(s_full + 24);   // [2][2][128] values the two warps swap
@@ -666,7 +669,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             pdl_wait();   // q_lat is written by the previous kernel of this call
             if (have) load_q(cur.v);
             while (have) {
-                const uint32_t b = g & 1, u = g >> 1;
+                const uint32_t b = g % kXB, u = g / kXB;
                 // partial scores: TMEM -> registers -> bf16 pairs
                 if (!uwait(s_full, g & 1)) { ok = false; break; }
                 ptx::tc_fence_after();
@@ -683,9 +686,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
 #pragma unroll
                     for (int i = 0; i < kT; i += 2) own[i / 2] = ptx::pack_bf16(sc[i], sc[i + 1]);
                 }
-                // staging buffer b is free once the local softmax read it (tile g-2) and the
-                // peer read the copy made from it
-                if (g >= 2 && !(uwait(&xs_free[b], (u - 1) & 1) && uwait_cluster(&x_empty[b], (u - 1) & 1))) {
+                // staging buffer b is free once the local softmax read it (tile g - kXB) and
+                // the peer read the copy made from it
+                if (g >= kXB && !(uwait(&xs_free[b], (u - 1) & 1) && uwait_cluster(&x_empty[b], (u - 1) & 1))) {
                     ok = false;
                     break;
                 }
@@ -729,7 +732,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                 return o;
             };
             while (have) {
-                const uint32_t b = g & 1, u = g >> 1;
+                const uint32_t b = g % kXB, u = g / kXB;
                 if (h == 0 && half == 0) ptx::mbar_expect_tx(&x_full[b], kXBytes);
                 if (!uwait(&xs_ready[b], u & 1)) { ok = false; break; }
                 if (!uwait_cluster(&x_full[b], u & 1)) { ok = false; break; }
