@@ -56,8 +56,6 @@ constexpr int kTileBytes = 4 * kChunkBytes + kRopeBytes;
 constexpr int kQRopeBytes = 128 * 64;         // this CTA's 32 rotary query columns, 128 heads
 constexpr int kXRowBytes = kT * 2;            // one head's 64 bf16 partial scores (128 B)
 constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads x 64 tokens
-// barriers (2 per stage + 24), the softmax pair exchange (2 KB), then the TMEM address, the
-// abort flag, the planning scratch and the sequence cache (128 B)
 constexpr int kBarBytes = 256 + 2048 + 256;
 // FP8 cache rows (see decode_tc.cuh): per tile and CTA, this CTA's 256 codes (two 128-byte
 // boxes, 128-byte swizzle), its 32 rotary columns (bf16, 64-byte swizzle) and the 64 rows'
@@ -94,8 +92,6 @@ constexpr int dec_smem() {
     return DecCfg<kF8>::kStages * DecCfg<kF8>::kStageBytes + 2 * DecCfg<kF8>::kXBufs * kXBytes + kQRopeBytes +
            kBarBytes;
 }
-static_assert((2 * DecCfg<false>::kStages + 24) * 8 <= 256 && (2 * DecCfg<true>::kStages + 24) * 8 <= 256,
-              "the barriers fit the first 256 bytes of the barrier area");
 static_assert(dec_smem<false>() <= 232448, "decode kernel shared memory over the 227 KB limit");
 static_assert(dec_smem<true>() <= 232448, "FP8 decode kernel shared memory over the 227 KB limit");
 constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols = 512;
@@ -174,29 +170,7 @@ struct SeqSrc {
         return L > 0 ? L : 0;
     }
     __device__ long long row0(int b) const { return block_table ? 0 : offsets[b]; }
-    // raw_len(b), with the sequence's first row in r0 from the same reads
-    __device__ int raw_len_row0(int b, long long& r0) const {
-        if (block_table) {
-            r0 = 0;
-            return raw_len(b);
-        }
-        const long long a = offsets[b], e = offsets[b + 1];
-        r0 = a;
-        return (a < 0 || e < a || e > cache_rows) ? -1 : (int)(e - a);
-    }
 };
-
-// The first kSeqCache sequences of a cluster's range: their lengths and first rows are kept
-// in shared memory by the planning, so the iterators of all roles start (and make their
-// first switches) without a global read.
-constexpr int kSeqCache = 4;
-struct SeqEnt {
-    long long row0;
-    int len, pad;
-};
-// TMEM address, abort flag, 16 warp sums, plan_first and the cache, in the barrier area's last 256 bytes
-static_assert(8 + 16 * 4 + 2 * 4 + 8 + kSeqCache * (int)sizeof(SeqEnt) <= 256, "the planning words fit the last 256 bytes");
-
 
 // Walks the pieces of sequences in this cluster's cost range [lo, hi), in sequence order,
 // starting from the sequence whose cost region holds lo (cost start cs).  The same walk runs
@@ -218,18 +192,13 @@ struct SegIter {
     SeqSrc src;
     int B, lo, hi, cluster, b, cs;
     int Qr, tr;   // siblings and this cluster's query (used with kSib only)
-    // (first row, len) of sequences c_b0 .. c_b0 + c_n - 1, in shared memory
-    const SeqEnt* c_seq;
-    int c_b0, c_n;
     __device__ __forceinline__ int Q() const { return kSib ? Qr : 1; }
     __device__ __forceinline__ int t() const { return kSib ? tr : 0; }
     __device__ bool next(Seg& s) {
         const int Q = this->Q(), t = this->t();
         while (b < B && cs < hi) {
-            const int ci = b - c_b0;
-            const bool cached = ci >= 0 && ci < c_n;
-            const int L = cached ? c_seq[ci].len : src.len(b);
-            const long long r0 = cached ? c_seq[ci].row0 : src.row0(b);
+            const int L = src.len(b);
+            const long long r0 = src.row0(b);
             const int n = tiles_of_len(L);
             const int f = cs + kPieceCost;   // cost position of tile 0
             const int bb = b;
@@ -298,8 +267,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     }
     // this thread's sequence length for the planning below, requested before the set-up
     // so that the load overlaps it
-    long long row0_0 = 0;
-    const int len0 = threadIdx.x < B ? src.raw_len_row0(threadIdx.x, row0_0) : 0;
+    const int len0 = threadIdx.x < B ? src.raw_len(threadIdx.x) : 0;
     uint8_t* smem = smem_raw;
     uint8_t* tiles = smem;
     constexpr uint32_t kXB = DecCfg<kF8>::kXBufs;
@@ -330,8 +298,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* plan_wsum = (int*)(tmem_slot + 2);   // [16] per-warp sums of the planning scans
     int* plan_first = plan_wsum + 16;         // [2] sequence holding this cluster's first tile, its first tile
-    // [kSeqCache] first rows and lengths of the range's first sequences (8-byte aligned)
-    SeqEnt* seq_c = (SeqEnt*)(plan_first + 4);
 
     const uint32_t rank = cluster_rank(), peer = rank ^ 1;
     const int cluster = (int)cluster_id_x();
@@ -438,19 +404,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             __syncthreads();
         }
     }
-    // the range's first sequences, from the lengths and first rows this CTA's threads read at
-    // entry (thread b holds sequence b)
-    const int b_first = plan_first[0];
-    const int c_n = max(0, min(kSeqCache, min(B, kThreads) - b_first));
-    {
-        const int ci = (int)threadIdx.x - b_first;
-        if (ci >= 0 && ci < c_n) {
-            seq_c[ci].row0 = row0_0;
-            seq_c[ci].len = len0 > 0 ? len0 : 0;
-        }
-        __syncthreads();
-    }
-    SegIter<kSib> it{src, B, lo, hi, cluster, b_first, plan_first[1], Q, tok, seq_c, b_first, c_n};
+    SegIter<kSib> it{src, B, lo, hi, cluster, plan_first[0], plan_first[1], Q, tok};
     Seg sg;
 
     if (warp == 0) {
