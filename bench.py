@@ -127,7 +127,8 @@ def paged_layout(w, inp, seed):
 
 def alg_layer(w: workloads.Workload) -> dict:
     """Bytes and flops of one full decode-layer step: append the new token, project the
-    query, absorbed attention over L + 1 rows, W_UV, W_O."""
+    query, absorbed attention over L + 1 rows, W_UV, W_O.  The same figures serve the folded
+    weights: they are the method's, and the folded products only add to what is moved."""
     L = workloads.lengths(w) + 1
     tokens = int(L.sum())
     e = 2 if w.dtype == "bf16" else 4
@@ -428,7 +429,7 @@ def build_step(w, inp, dev, mla):
         h2d = [("q_nope", inp["q_nope"]), ("q_rope", inp["q_rope"])]
         return g, dims, weights, out, step, h2d, alg_multi(w), w.B * w.q_len
     if w.kind == "decode_layer":
-        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"])
+        weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"], fold=w.fold)
         out = torch.empty(w.B, w.d_model, dtype=dt, device=dev)
         ws = mla.workspace(mla.mla_decode_workspace_size(dims, w.B), dev)
         L = workloads.lengths(w)

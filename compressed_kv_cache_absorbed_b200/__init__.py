@@ -42,7 +42,7 @@ SIGNATURES = {
     "mla_cache_row_elems": (ctypes.c_int64, [_D]),
     "mla_cache_bytes_per_token": (ctypes.c_int64, [_D, ctypes.c_int32]),
     "mla_decode_path": (ctypes.c_int32, [_D]),
-    "mla_absorb_weights": (_S, [_D, _P, _P, _P, _P, ctypes.POINTER(_P), _P]),
+    "mla_absorb_weights": (_S, [_D, _P, _P, _P, _P, ctypes.c_int32, ctypes.POINTER(_P), _P]),
     "mla_weights_destroy": (_S, [_P]),
     "mla_append_cache": (_S, [_D, _P, _P, _P, _P, _P, ctypes.c_int32, _P, ctypes.c_int64, _P]),
     "mla_decode_workspace_size": (ctypes.c_size_t, [_D, ctypes.c_int32]),
@@ -143,14 +143,15 @@ def workspace(nbytes: int, device="cuda") -> torch.Tensor:
 # -------------------------------------------------------------------- weights
 
 class MLAWeights:
-    """Owner of an mla_weights handle (packed W_UK/W_UV; borrows W_Q/W_O)."""
+    """Owner of an mla_weights handle (packed W_UK/W_UV; borrows W_Q/W_O; with fold, also the
+    folded products)."""
 
-    def __init__(self, dims: mla_dims, W_UK, W_UV, W_Q=None, W_O=None, stream=None):
+    def __init__(self, dims: mla_dims, W_UK, W_UV, W_Q=None, W_O=None, stream=None, fold=False):
         self.dims = dims
         self._keep = (W_Q, W_O)  # borrowed by the handle: keep alive
         h = ctypes.c_void_p()
         _check(_lib.mla_absorb_weights(ctypes.byref(dims), _ptr(W_UK), _ptr(W_UV), _ptr(W_Q), _ptr(W_O),
-                                       ctypes.byref(h), _stream(stream)), "mla_absorb_weights")
+                                       1 if fold else 0, ctypes.byref(h), _stream(stream)), "mla_absorb_weights")
         self.handle = h
 
     def close(self):
@@ -165,8 +166,8 @@ class MLAWeights:
             pass
 
 
-def mla_absorb_weights(dims, W_UK, W_UV, W_Q=None, W_O=None, stream=None) -> MLAWeights:
-    return MLAWeights(dims, W_UK, W_UV, W_Q, W_O, stream)
+def mla_absorb_weights(dims, W_UK, W_UV, W_Q=None, W_O=None, stream=None, fold=False) -> MLAWeights:
+    return MLAWeights(dims, W_UK, W_UV, W_Q, W_O, stream, fold)
 
 
 # ------------------------------------------------------------------------ calls

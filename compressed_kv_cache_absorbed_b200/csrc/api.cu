@@ -66,6 +66,10 @@ struct mla_weights_s {
     void* uv_tiled;    //   (bf16 V2/V3 head shape only; else null)
     const void* W_Q;
     const void* W_O;
+    // fold = 1 (bf16): W_UK folded into W_Q, W_UV into W_O, and W_Q's rotary rows
+    void* W_QUK = nullptr;   // [H*d_c, d_model]
+    void* W_OUV = nullptr;   // [d_model, H*d_c], fp16
+    void* W_QR = nullptr;    // [H*d_hR, d_model]
 };
 
 // ------------------------------------------------------------------- validation
@@ -168,8 +172,61 @@ extern "C" int32_t mla_decode_path(const mla_dims* d) {
 
 // ---------------------------------------------------------------------- weights
 
+// The folded products [L1 "Coste de computo"], per head h (fp32 sums on the tensor cores, one
+// rounding):  W_QUK[h*d_c + c, :] = sum_j W_UKT[h, c, j] W_Q[h*qh + j, :] in bf16 (it meets
+// the bf16 hidden states) and W_OUV[:, h*d_c + c] = sum_v W_O[:, h*v_head + v] W_UV[h, v, c]
+// in fp16 (it meets o_lat, which the merge keeps in fp16); and W_Q's rotary rows.
+static cudaError_t fold_weights(const mla_dims* d, mla_weights w, DevErr err, cudaStream_t s) {
+    const int H = d->H, dc = d->d_c, qk = d->qk_nope, dR = d->d_hR, vh = d->v_head, dm = d->d_model;
+    const int qh = qk + dR;
+    const size_t nQUK = (size_t)H * dc * dm, nQR = (size_t)H * dR * dm;
+    cudaError_t e = cudaSuccess;
+    if (cudaMalloc(&w->W_QUK, nQUK * 2) != cudaSuccess || cudaMalloc(&w->W_OUV, nQUK * 2) != cudaSuccess ||
+        cudaMalloc(&w->W_QR, nQR * 2) != cudaSuccess)
+        return cudaErrorMemoryAllocation;
+    void* qnT = nullptr;   // [H, d_model, qk_nope]: W_Q's content rows, transposed per head
+    void* uvT = nullptr;   // [H, d_c, v_head]
+    if ((e = cudaMallocAsync(&qnT, (size_t)H * dm * qk * 2, s)) != cudaSuccess) return e;
+    if ((e = cudaMallocAsync(&uvT, (size_t)H * dc * vh * 2, s)) != cudaSuccess) {
+        cudaFreeAsync(qnT, s);
+        return e;
+    }
+    e = mla::launch_transpose_heads((const bf16*)w->W_Q, (bf16*)qnT, H, qk, dm, s, (long long)qh * dm);
+    if (e == cudaSuccess) e = mla::launch_transpose_heads((const bf16*)w->W_UV, (bf16*)uvT, H, vh, dc, s);
+    if (e == cudaSuccess) {
+        // C[h][c][j] = sum_k W_UKT[h][c][k] qnT[h][j][k]  ->  W_QUK[h*dc + c][j]
+        mla::tc::GemmOut o{w->W_QUK, (long long)dc * dm, dm, 1, 0};
+        e = mla::tc::gemm_bf16_tc(H, dc, dm, qk, (const bf16*)w->W_UKT, (long long)dc * qk, qk, (const bf16*)qnT,
+                                  (long long)dm * qk, qk, o, err.code, err.detail, s);
+    }
+    if (e == cudaSuccess) {
+        // C[h][i][c] = sum_v W_O[i][h*vh + v] uvT[h][c][v]  ->  W_OUV[i][h*dc + c]
+        mla::tc::GemmOut o{w->W_OUV, dc, (long long)H * dc, 1, 0};
+        o.f16 = 1;
+        e = mla::tc::gemm_bf16_tc(H, dm, dc, vh, (const bf16*)w->W_O, vh, (long long)H * vh, (const bf16*)uvT,
+                                  (long long)dc * vh, vh, o, err.code, err.detail, s);
+    }
+    if (e == cudaSuccess)
+        e = cudaMemcpy2DAsync(w->W_QR, (size_t)dR * dm * 2, (const bf16*)w->W_Q + (size_t)qk * dm, (size_t)qh * dm * 2,
+                              (size_t)dR * dm * 2, H, cudaMemcpyDeviceToDevice, s);
+    const cudaError_t f1 = cudaFreeAsync(qnT, s), f2 = cudaFreeAsync(uvT, s);
+    return e != cudaSuccess ? e : f1 != cudaSuccess ? f1 : f2;
+}
+
+static void free_weights(mla_weights w) {
+    cudaFree(w->W_UK);
+    cudaFree(w->W_UKT);
+    cudaFree(w->W_UV);
+    cudaFree(w->ukt_tiled);
+    cudaFree(w->uv_tiled);
+    cudaFree(w->W_QUK);
+    cudaFree(w->W_OUV);
+    cudaFree(w->W_QR);
+    delete w;
+}
+
 extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, const void* W_UV,
-                                         const void* W_Q, const void* W_O, mla_weights* out,
+                                         const void* W_Q, const void* W_O, int32_t fold, mla_weights* out,
                                          mla_stream_t stream) {
     if (!out) return MLA_ERR_INVALID_ARG;
     *out = nullptr;
@@ -177,6 +234,12 @@ extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, co
     if (st != MLA_OK) return st;
     if (!W_UK || !W_UV) return MLA_ERR_INVALID_ARG;
     if ((W_Q || W_O) && d->d_model <= 0) return MLA_ERR_INVALID_ARG;
+    if (fold != 0 && fold != 1) return MLA_ERR_INVALID_ARG;
+    if (fold && (!W_Q || !W_O)) return MLA_ERR_INVALID_ARG;
+    if (fold && (!tc_decode_ok(d) || !tc_proj_ok(d) || !aligned16(W_Q) || !aligned16(W_O)))
+        return MLA_ERR_UNSUPPORTED;
+    DevErr fold_err;
+    if (fold && (st = dev_err(&fold_err)) != MLA_OK) return st;
     cudaStream_t s = (cudaStream_t)stream;
     const size_t es = esize(d);
     const size_t nk = (size_t)d->H * d->qk_nope * d->d_c, nv = (size_t)d->H * d->v_head * d->d_c;
@@ -216,13 +279,18 @@ extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, co
         e = mla::tc::tile_weights_tc((const bf16*)w->W_UKT, (const bf16*)w->W_UV, (bf16*)w->ukt_tiled,
                                      (bf16*)w->uv_tiled, s);
     }
+    if (e == cudaSuccess && fold) {
+        e = fold_weights(d, w, fold_err, s);
+        if (e == cudaErrorMemoryAllocation) {
+            cudaGetLastError();
+            cudaStreamSynchronize(s);
+            free_weights(w);
+            return MLA_ERR_NO_MEMORY;
+        }
+    }
     if (e != cudaSuccess) {
-        cudaFree(w->W_UK);
-        cudaFree(w->W_UKT);
-        cudaFree(w->W_UV);
-        cudaFree(w->ukt_tiled);
-        cudaFree(w->uv_tiled);
-        delete w;
+        cudaStreamSynchronize(s);
+        free_weights(w);
         return cuda_fail(e, "mla_absorb_weights");
     }
     *out = w;
@@ -232,12 +300,7 @@ extern "C" mla_status mla_absorb_weights(const mla_dims* d, const void* W_UK, co
 extern "C" mla_status mla_weights_destroy(mla_weights w) {
     if (!w) return MLA_OK;
     cudaDeviceSynchronize();
-    cudaFree(w->W_UK);
-    cudaFree(w->W_UKT);
-    cudaFree(w->W_UV);
-    cudaFree(w->ukt_tiled);
-    cudaFree(w->uv_tiled);
-    delete w;
+    free_weights(w);
     return MLA_OK;
 }
 
@@ -380,6 +443,43 @@ static cudaError_t decode_impl(const mla_dims* d, mla_weights w, const void* q_n
     cudaError_t e;
     const bool tc_proj = tc_proj_ok(d) && (q_nope || aligned16(h)) && (q_nope || aligned16(w->W_Q)) &&
                          (!w->W_O || (aligned16(w->W_O) && aligned16(out)));
+    if (!q_nope && tc_proj && tc_path && w->W_QUK) {
+        // folded weights [L1 "Coste de computo": precomputed products]:
+        //   q_lat[b] = W_QUK h[b],  q_rope[b] = RoPE(W_QR h[b]),  attention on the latent cache,
+        //   o_lat = the merged latent output,  out[b] = W_OUV o_lat[b]
+        const int dc = d->d_c, dm = d->d_model;
+        {
+            mla::ProfScope ps(s, "tc_q_lat_folded");
+            mla::tc::GemmOut oq{ws.tc.q_lat, 0, 1, (long long)H * dc, 0};
+            e = mla::tc::gemm_bf16_tc(1, H * dc, B, dm, (const bf16*)w->W_QUK, 0, dm, (const bf16*)h, 0, dm, oq,
+                                      err.code, err.detail, s, true);
+            if (e != cudaSuccess) return e;
+        }
+        {
+            mla::ProfScope ps(s, "tc_q_rope_folded");
+            e = mla::tc::rope_table(q_pos, 1, B, dR, theta_of(d), ws.rope_tab, s);
+            if (e != cudaSuccess) return e;
+            mla::tc::GemmOut oq{ws.q_buf, 0, 1, (long long)H * dR, 0};
+            oq.period = dR;
+            oq.rope_start = 0;
+            oq.d_rope = dR;
+            oq.rope_tab = ws.rope_tab;
+            e = mla::tc::gemm_bf16_tc(1, H * dR, B, dm, (const bf16*)w->W_QR, 0, dm, (const bf16*)h, 0, dm, oq,
+                                      err.code, err.detail, s);
+            if (e != cudaSuccess) return e;
+        }
+        // o_lat overwrites q_lat: the merge writes it only after the decode kernel has finished
+        e = mla::tc::decode_absorbed_tc(nullptr, 0, 0, (const bf16*)ws.q_buf, (long long)H * dR, dR, nullptr, nullptr,
+                                        cache, false, cache_rows, offsets, nullptr, nullptr, 0, B, 1, true,
+                                        scale_of(d), ws.tc.q_lat, ws.tc, num_sms(), err.code, err.detail, s,
+                                        true);
+        if (e != cudaSuccess) return e;
+        mla::ProfScope ps(s, "tc_w_o_folded");
+        mla::tc::GemmOut oo{out, 0, 1, dm, 0};
+        oo.in_f16 = 1;   // W_OUV and o_lat in fp16
+        return mla::tc::gemm_bf16_tc(1, dm, B, H * dc, (const bf16*)w->W_OUV, 0, (long long)H * dc,
+                                     (const bf16*)ws.tc.q_lat, 0, (long long)H * dc, oo, err.code, err.detail, s);
+    }
     if (!q_nope && tc_proj) {
         // q = W_Q h with RoPE on each head's rotary part at q_pos [L1 "Multi-head attention estandar"]
         const int qh = qk + dR;

@@ -126,8 +126,10 @@ cudaError_t launch_prefill_attn_simt(const T* q, const T* k_nope, const T* cache
                                      int B, int S, int H, int qk_nope, int d_hR, int d_c,
                                      int v_head, float scale, T* out, cudaStream_t s);
 
-// per-head transpose: dst[h][c][r] = src[h][r][c] (src [Hn, R, C])
+// per-head transpose: dst[h][c][r] = src[h][r][c]; head h of src starts at h * src_head_stride
+// elements (R * C when negative), dst is [Hn, C, R]
 template <typename T>
-cudaError_t launch_transpose_heads(const T* src, T* dst, int Hn, int R, int C, cudaStream_t s);
+cudaError_t launch_transpose_heads(const T* src, T* dst, int Hn, int R, int C, cudaStream_t s,
+                                   long long src_head_stride = -1);
 
 }  // namespace mla

@@ -893,7 +893,10 @@ constexpr int kMergeABytes = 8 * 128 * 128;   // W_UV[h]: 8 chunks of 128 rows x
 template <int BN>
 constexpr int merge_smem() { return kMergeABytes + 8 * BN * 128 + 1024 + 64; }
 
-template <int BN, bool kSib>
+// kLat: the merged, normalised o_lat rows themselves are the output (fp16, saturated, at
+// o[v, h, :] with strides sO_b, sO_h): no W_UV product (the folded weights apply W_UV inside
+// W_O, whose product takes o_lat in fp16).
+template <int BN, bool kSib, bool kLat = false>
 __global__ void __launch_bounds__(kMergeThreads, 1)
 merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, int B, int Q_arg,
                  const __half* __restrict__ part_o, const float* __restrict__ part_ml, __nv_bfloat16* __restrict__ o,
@@ -913,14 +916,16 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
         ptx::mbar_init(a_full, 1);
         ptx::mbar_init(d_full, 1);
         ptx::fence_mbar_init();
-        // the weights are not written by earlier kernels: load them before waiting; the tiled
-        // copy is already the shared-memory image, 8 contiguous 16 KB chunks per head
-        ptx::mbar_expect_tx(a_full, kMergeABytes);
-        const uint8_t* src = (const uint8_t*)uv + (size_t)h * kMergeABytes;
+        if (!kLat) {
+            // the weights are not written by earlier kernels: load them before waiting; the
+            // tiled copy is already the shared-memory image, 8 contiguous 16 KB chunks per head
+            ptx::mbar_expect_tx(a_full, kMergeABytes);
+            const uint8_t* src = (const uint8_t*)uv + (size_t)h * kMergeABytes;
 #pragma unroll
-        for (int kc = 0; kc < 8; ++kc) ptx::bulk_load(sA + kc * 16384, src + kc * 16384, 16384, a_full);
+            for (int kc = 0; kc < 8; ++kc) ptx::bulk_load(sA + kc * 16384, src + kc * 16384, 16384, a_full);
+        }
     }
-    if (warp == 1) {
+    if (!kLat && warp == 1) {
         ptx::tmem_alloc(tmem_slot, BN);
         ptx::tmem_relinquish();
     }
@@ -1086,6 +1091,21 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
 #pragma unroll
                 for (int c = 0; c < 16; ++c) acc[c] *= inv;
             }
+            if (kLat) {   // o_lat[v, h, 16 lane ..] as fp16 (saturated), one rounding
+                const int v = n0 + r;
+                if (v < NV) {
+#pragma unroll
+                    for (int c = 0; c < 16; ++c) acc[c] = fminf(fmaxf(acc[c], -65504.f), 65504.f);
+                    uint4* dst = (uint4*)(o + v * sO_b + h * sO_h + 16 * lane);
+#pragma unroll
+                    for (int hv = 0; hv < 2; ++hv)
+                        dst[hv] = make_uint4(ptx::pack_f16(acc[8 * hv], acc[8 * hv + 1]),
+                                             ptx::pack_f16(acc[8 * hv + 2], acc[8 * hv + 3]),
+                                             ptx::pack_f16(acc[8 * hv + 4], acc[8 * hv + 5]),
+                                             ptx::pack_f16(acc[8 * hv + 6], acc[8 * hv + 7]));
+                }
+                continue;
+            }
             // o_lat as fp16 (saturated), the B operand of the W_UV product: columns 16 lane ..
             // +15 = chunk lane / 4, 16-byte units 2 (lane % 4) and +1 of row r
             uint8_t* rowp = sB + (lane >> 2) * (BN * 128) + r * 128;
@@ -1101,6 +1121,7 @@ merge_wuv_kernel(const __nv_bfloat16* __restrict__ uv, const SeqSrc src, int P, 
             }
         }
     }
+    if (kLat) return;   // no W_UV product, no TMEM
     ptx::fence_proxy_async_smem();   // the tensor cores read what the threads wrote
     ptx::tc_fence_before();
     __syncthreads();
@@ -1322,21 +1343,23 @@ cudaError_t launch_absorb_any(int NV, const __nv_bfloat16* ukt, const CUtensorMa
                       : launch_absorb<128, kF16>(ukt, mq, NV, q_lat, err_code, err_detail, s);
 }
 
-template <bool kSib>
+template <bool kSib, bool kLat = false>
 cudaError_t launch_merge(int NV, const __nv_bfloat16* uv, const SeqSrc& seqs, int P, int B, int Q, const DecodeWs& ws,
                          __nv_bfloat16* o, int* err_code, long long* err_detail, cudaStream_t s) {
+    // o [NV, 128 heads, 128] (W_UV applied), or o_lat [NV, 128 heads, 512] (kLat)
+    const long long sO_b = kLat ? 128LL * 512 : 128LL * 128, sO_h = kLat ? 512 : 128;
     if (NV <= 32) {
-        static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32, kSib>, merge_smem<32>());
+        static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<32, kSib, kLat>, merge_smem<32>());
         if (attr != cudaSuccess) return attr;
-        return launch_pdl(merge_wuv_kernel<32, kSib>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s, uv,
-                          seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
+        return launch_pdl(merge_wuv_kernel<32, kSib, kLat>, dim3(128, 1), dim3(kMergeThreads), merge_smem<32>(), s,
+                          uv, seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o, sO_b, sO_h,
                           err_code, err_detail);
     }
-    static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64, kSib>, merge_smem<64>());
+    static const cudaError_t attr = set_smem_attrs(merge_wuv_kernel<64, kSib, kLat>, merge_smem<64>());
     if (attr != cudaSuccess) return attr;
-    return launch_pdl(merge_wuv_kernel<64, kSib>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads), merge_smem<64>(), s,
-                      uv, seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o, 128LL * 128, 128LL,
-                      err_code, err_detail);
+    return launch_pdl(merge_wuv_kernel<64, kSib, kLat>, dim3(128, (NV + 63) / 64), dim3(kMergeThreads),
+                      merge_smem<64>(), s, uv, seqs, P, B, Q, (const __half*)ws.part_o, (const float*)ws.part_ml, o,
+                      sO_b, sO_h, err_code, err_detail);
 }
 
 int g_clusters_cached = 0;
@@ -1408,7 +1431,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
                                const int32_t* offsets, const int32_t* seq_lens, const int32_t* block_table,
                                int bt_stride, int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
                                int num_sms,
-                               int* err_code, long long* err_detail, cudaStream_t s) {
+                               int* err_code, long long* err_detail, cudaStream_t s, bool folded) {
     if (B <= 0) return cudaSuccess;
     cudaError_t e;
     if (cache_rows <= 0 || cache_rows > 0x7FFFFFFFLL) return cudaErrorInvalidValue;
@@ -1417,7 +1440,7 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
     const int P = max_clusters(num_sms);
     if (Q < 1 || Q > P) return cudaErrorInvalidValue;
     const int NV = B * Q;   // queries
-    {
+    if (!folded) {
         // q_lat[v,h,:] = W_UK[h]^T q_nope[v,h,:]
         ProfScope ps(s, "tc_q_absorb");
         CUtensorMap mq;
@@ -1450,7 +1473,8 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
             e = launch_pdl(Q > 1 ? decode_tc_kernel<false, true> : decode_tc_kernel<false, false>, dim3(2 * P),
                            dim3(DecCfg<false>::kThreads), dec_smem<false>(), s, m, mr, msc, ws.q_lat, qr, sQr_b, sQr_h,
                            seqs, B, Q, (int)(stream_once ? 1 : 0), (long long)cache_rows, scale_log2, ws.part_o,
-                           ws.part_ml, (const uint8_t*)uv, (long long)kTiledWeightBytes, err_code, err_detail);
+                           ws.part_ml, folded ? nullptr : (const uint8_t*)uv, folded ? 0LL : (long long)kTiledWeightBytes,
+                           err_code, err_detail);
         } else {
             // FP8 rows of kF8RowBytes: codes as bytes, the rotary key as bf16 elements, the
             // scale field as fp32 elements
@@ -1475,7 +1499,12 @@ cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long lo
         }
         if (e != cudaSuccess) return e;
     }
-    {
+    if (folded) {
+        // merge of the pieces alone: o = o_lat (W_UV is inside the folded W_O)
+        ProfScope ps(s, "tc_merge");
+        e = Q > 1 ? launch_merge<true, true>(NV, uv, seqs, P, B, Q, ws, o, err_code, err_detail, s)
+                  : launch_merge<false, true>(NV, uv, seqs, P, B, Q, ws, o, err_code, err_detail, s);
+    } else {
         // merge of the pieces fused with o[v,h,:] = W_UV[h] o_lat[v,h,:]
         ProfScope ps(s, "tc_merge_w_uv");
         e = Q > 1 ? launch_merge<true>(NV, uv, seqs, P, B, Q, ws, o, err_code, err_detail, s)

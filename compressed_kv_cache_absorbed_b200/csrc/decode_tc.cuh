@@ -60,13 +60,17 @@ cudaError_t tile_weights_tc(const __nv_bfloat16* W_UKT, const __nv_bfloat16* W_U
 // pass false when other queries of the call read the same tiles.  1 <= Q <= the cluster
 // count; the workspace is that of B * Q queries.
 // fp8: the cache holds FP8 rows (kF8RowBytes each) instead of bf16 rows.
+// folded: q_lat is already in ws.q_lat (the absorbed query projection wrote it; qn and ukt
+// are not read) and the output is o_lat itself, o [B * Q, H, 512] in fp16 (saturated),
+// without W_UV (uv is not read); o may be ws.q_lat.
 cudaError_t decode_absorbed_tc(const __nv_bfloat16* qn, long long sQn_b, long long sQn_h,
                                const __nv_bfloat16* qr, long long sQr_b, long long sQr_h,
                                const __nv_bfloat16* ukt, const __nv_bfloat16* uv,
                                const void* cache, bool fp8, long long cache_rows, const int32_t* offsets,
                                const int32_t* seq_lens, const int32_t* block_table, int bt_stride,
                                int B, int Q, bool stream_once, float scale, __nv_bfloat16* o, const DecodeWs& ws,
-                               int num_sms, int* err_code, long long* err_detail, cudaStream_t s);
+                               int num_sms, int* err_code, long long* err_detail, cudaStream_t s,
+                               bool folded = false);
 
 // Clusters of the decode kernel on this device (sibling groups are formed from these).
 int decode_clusters(int num_sms);

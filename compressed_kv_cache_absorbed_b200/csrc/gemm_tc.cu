@@ -196,7 +196,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
         }
     } else if (warp == 1) {
         if (lane == 0) {
-            constexpr uint32_t idesc = ptx::idesc_bf16_f32(kBM, BN, 0, 0);
+            const uint32_t idesc = out.in_f16 ? ptx::idesc_f16_f32(kBM, BN, 0, 0) : ptx::idesc_bf16_f32(kBM, BN, 0, 0);
             int it = 0, lt = 0;
             bool ok = true;
             for (int t = blockIdx.x; ok && t < tiles; t += gridDim.x, ++lt) {
@@ -442,8 +442,9 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     const uint64_t sb[2] = {(uint64_t)sBn * 2, (uint64_t)sBz * 2};
     const uint32_t bx[3] = {(uint32_t)kBK, (uint32_t)kBM, 1};   // the 128-row operand
     const uint32_t by[3] = {(uint32_t)kBK, (uint32_t)BN, 1};    // the BN-row operand
-    if (!make_tmap_bf16(&ma, A, a_bcast ? 2 : 3, da, sa, swap ? by : bx) ||
-        !make_tmap_bf16(&mb, B, b_bcast ? 2 : 3, db, sb, swap ? bx : by))
+    const CUtensorMapDataType dt = out.in_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    if (!make_tmap(&ma, dt, 2, A, a_bcast ? 2 : 3, da, sa, swap ? by : bx, 128) ||
+        !make_tmap(&mb, dt, 2, B, b_bcast ? 2 : 3, db, sb, swap ? bx : by, 128))
         return cudaErrorInvalidValue;
     const CUtensorMap& mx = swap ? mb : ma;
     const CUtensorMap& my = swap ? ma : mb;

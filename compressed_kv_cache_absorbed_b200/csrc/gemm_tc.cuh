@@ -17,7 +17,7 @@ namespace tc {
 // Rotation is done in double precision and the result rounded once.
 // f16 (with f32 == 0) stores fp16 instead of bf16: every column, or with period > 0 only the
 // columns m with (m % period) < rope_start (the rotary columns stay bf16).  fp16 stores
-// saturate at +-65504.
+// saturate at +-65504.  in_f16: the operands A and B hold fp16, not bf16 (both the same).
 struct GemmOut {
     void* C;
     long long sz, sm, sn;
@@ -30,6 +30,7 @@ struct GemmOut {
     int pos_mod = 1;
     float theta = 10000.f;
     const double2* rope_tab = nullptr;
+    int in_f16 = 0;
 };
 
 // rope_tab[n * d_rope / 2 + i] = (cos, sin)(pos(n) * theta^(-2i/d_rope)), computed in double.

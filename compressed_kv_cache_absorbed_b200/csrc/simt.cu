@@ -383,11 +383,12 @@ prefill_attn_simt_kernel(const T* __restrict__ q, const T* __restrict__ k_nope,
 }
 
 template <typename T>
-__global__ void transpose_heads_kernel(const T* __restrict__ src, T* __restrict__ dst, int R, int C) {
+__global__ void transpose_heads_kernel(const T* __restrict__ src, T* __restrict__ dst, int R, int C,
+                                       long long src_head_stride) {
     __shared__ T tile[32][33];
     const int h = blockIdx.z;
     const int c0 = blockIdx.x * 32, r0 = blockIdx.y * 32;
-    const T* s = src + (long long)h * R * C;
+    const T* s = src + (long long)h * src_head_stride;
     T* d = dst + (long long)h * R * C;
     for (int i = threadIdx.y; i < 32; i += blockDim.y) {
         const int r = r0 + i, c = c0 + threadIdx.x;
@@ -471,9 +472,11 @@ cudaError_t launch_prefill_attn_simt(const T* q, const T* k_nope, const T* cache
 }
 
 template <typename T>
-cudaError_t launch_transpose_heads(const T* src, T* dst, int Hn, int R, int C, cudaStream_t s) {
+cudaError_t launch_transpose_heads(const T* src, T* dst, int Hn, int R, int C, cudaStream_t s,
+                                   long long src_head_stride) {
     dim3 grid(ceil_div(C, 32), ceil_div(R, 32), Hn);
-    transpose_heads_kernel<T><<<grid, dim3(32, 8), 0, s>>>(src, dst, R, C);
+    transpose_heads_kernel<T><<<grid, dim3(32, 8), 0, s>>>(src, dst, R, C,
+                                                           src_head_stride < 0 ? (long long)R * C : src_head_stride);
     return cudaGetLastError();
 }
 
@@ -491,7 +494,7 @@ using bf16 = __nv_bfloat16;
     template cudaError_t launch_prefill_attn_simt<T>(const T*, const T*, const T*, const T*,    \
                                                      int, int, int, int, int, int, int, float,  \
                                                      T*, cudaStream_t);                         \
-    template cudaError_t launch_transpose_heads<T>(const T*, T*, int, int, int, cudaStream_t);
+    template cudaError_t launch_transpose_heads<T>(const T*, T*, int, int, int, cudaStream_t, long long);
 MLA_INST_T(float)
 MLA_INST_T(bf16)
 

@@ -105,9 +105,22 @@ int32_t mla_decode_path(const mla_dims* dims);
  * W_Q rows are head-major, the qk_nope content rows of a head before its d_hR rotary rows.
  * Borrowed tensors must stay valid until mla_weights_destroy.  The handle owns device
  * memory allocated here (the only allocation the library makes).  Stream-ordered: the
- * packing kernels run on `stream`. */
+ * packing kernels run on `stream`.
+ *
+ * fold = 1 also precomputes the matrix products the up-projections can be folded into
+ * [L1 "Coste de computo": precomputed products], per head h (fp32 sums, one rounding; W_QUK
+ * in bf16, W_OUV in fp16 as it meets the merged latent output kept in fp16):
+ *   W_QUK [H*d_c, d_model]:  W_QUK[h*d_c + c, :] = sum_j W_UK[h, j, c] W_Q[h*(qk_nope+d_hR) + j, :]
+ *   W_OUV [d_model, H*d_c]:  W_OUV[:, h*d_c + c] = sum_v W_O[:, h*v_head + v] W_UV[h, v, c]
+ * and a copy of W_Q's rotary rows.  mla_decode_absorbed from hidden states then computes
+ * q_lat = W_QUK h directly (no q_nope, no absorption kernel) and out = W_OUV o_lat (no W_UV
+ * product): the same attention, with different rounding points.  At V2/V3 sizes the two
+ * products take ~0.94 GB each, and a decode step reads them all, ~3x the projection bytes
+ * and flops of fold = 0.  Requires W_Q and W_O (else MLA_ERR_INVALID_ARG) and the bf16
+ * tensor-core shape (else MLA_ERR_UNSUPPORTED); temporary device memory is allocated and
+ * freed stream-ordered.  Other entry points ignore the folded products. */
 mla_status mla_absorb_weights(const mla_dims* dims, const void* W_UK, const void* W_UV,
-                              const void* W_Q, const void* W_O, mla_weights* out,
+                              const void* W_Q, const void* W_O, int32_t fold, mla_weights* out,
                               mla_stream_t stream);
 
 /* Free a handle (synchronises the device first).  NULL is accepted. */

@@ -93,7 +93,11 @@ def test_argument_errors_return_before_any_launch():
     bad = v3(d_hR=7)
     assert lib.mla_append_cache(ctypes.byref(bad), None, None, None, None, None, 1, None, 1, None) == mla.MLA_ERR_UNSUPPORTED
     h = ctypes.c_void_p()
-    assert lib.mla_absorb_weights(ctypes.byref(d), None, None, None, None, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_absorb_weights(ctypes.byref(d), None, None, None, None, 0, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
+    # fold needs W_Q and W_O; fold outside {0, 1} is rejected (both before any device work)
+    dummy = ctypes.c_void_p(16)
+    assert lib.mla_absorb_weights(ctypes.byref(d), dummy, dummy, None, None, 1, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
+    assert lib.mla_absorb_weights(ctypes.byref(d), dummy, dummy, None, None, 2, ctypes.byref(h), None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_absorbed(ctypes.byref(d), None, None, None, None, None, None, 0, None, 1, None, None, 0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_prefill_causal(ctypes.byref(d), None, None, None, None, None, None, 1, 1, None, 0, None) == mla.MLA_ERR_INVALID_ARG
     assert lib.mla_decode_absorbed_paged(ctypes.byref(d), None, None, None, None, 1, None, 1, None, 1, None, None,

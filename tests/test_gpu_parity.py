@@ -209,7 +209,7 @@ def test_decode_attn_full_size_sampled(name):
 
 # --------------------------------------------------------------- decode layer
 
-def run_decode_layer(w, inp):
+def run_decode_layer(w, inp, fold=False):
     dims = dims_of(w)
     g = to_dev(inp)
     B = w.B
@@ -227,7 +227,7 @@ def run_decode_layer(w, inp):
     q_pos = torch.from_numpy(L.astype(np.int32)).to(DEV)
     slot = torch.from_numpy(offs[:-1] + L).to(DEV)
     mla.mla_append_cache(dims, g["h_new"], g["W_DKV"], g["W_KR"], q_pos, slot, cache)
-    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"])
+    weights = mla.mla_absorb_weights(dims, g["W_UK"], g["W_UV"], g["W_Q"], g["W_O"], fold=fold)
     out = torch.empty(B, w.d_model, dtype=g["h_new"].dtype, device=DEV)
     ws = mla.workspace(mla.mla_decode_workspace_size(dims, B))
     mla.mla_decode_absorbed(dims, weights, cache, g["offsets"], out, ws, h=g["h_new"], q_pos=q_pos)
@@ -284,6 +284,33 @@ def test_decode_layer_v3_full_size_sampled():
     frac = check_rows(got, allnew, "bf16", "v3 appended rows")
     assert frac >= CACHE_EXACT_FRAC
     assert torch.equal(cache[:8192].cpu(), inp["cache"][:8192])
+
+
+def test_decode_layer_folded_weights():
+    """fold = 1: W_UK folded into W_Q and W_UV into W_O ("Coste de computo", precomputed
+    products).  The layer output is the same attention, so it is held to the oracle's layer
+    at the same bound: every sequence of a reduced V3-shaped layer (ragged, several tiles), on
+    the folded kernels (no q absorption, no W_UV product), and sampled sequences at full size."""
+    w = workloads.shrink(workloads.WORKLOADS["v3_layer_b128_ctx8192"], B=5, ctx=300, seed=95)
+    inp = workloads.make_inputs(w)
+    mla.mla_profile_report(reset=True)
+    mla.mla_profile_enable(True)
+    try:
+        out, _ = run_decode_layer(w, inp, fold=True)
+    finally:
+        mla.mla_profile_enable(False)
+    names = set(mla.mla_profile_report(reset=True))
+    assert {"tc_q_lat_folded", "tc_q_rope_folded", "tc_flash_decode", "tc_merge", "tc_w_o_folded"} <= names, names
+    assert not names & {"tc_q_absorb", "tc_merge_w_uv", "tc_q_proj_rope", "tc_w_o"}, names
+    want, _ = oracle_decode_layer(w, inp, list(range(w.B)), absorbed=True)
+    assert_close(out, want, "bf16", "folded layer (reduced)")
+
+    w = workloads.WORKLOADS["v3_layer_b128_ctx8192"]
+    inp = workloads.make_inputs(w)
+    out, _ = run_decode_layer(w, inp, fold=True)
+    bs = [0, 57, w.B - 1]
+    want, _ = oracle_decode_layer(w, inp, bs, absorbed=True)
+    assert_close(out[bs], want, "bf16", "folded v3 layer out")
 
 
 # ---------------------------------------------------------------------- prefill

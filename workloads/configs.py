@@ -43,6 +43,7 @@ class Workload:
     rope_theta: float = 10000.0
     cache_std: float = 0.5    # synthetic cache rows ~ cache_std * N(0, 1)
     q_len: int = 1            # decode_multi: new tokens per sequence (appended after the ctx rows)
+    fold: bool = False        # decode_layer: weights with W_UK folded into W_Q and W_UV into W_O
 
     @property
     def row(self) -> int:
@@ -75,6 +76,11 @@ WORKLOADS: Dict[str, Workload] = {
     "v3_layer_b128_ctx8192": Workload("v3_layer_b128_ctx8192", "decode_layer", B=128, H=128,
                                       d_model=7168, d_c=512, d_hR=64, qk_nope=128, v_head=128,
                                       dtype="bf16", seed=_seed(4), ctx=8192, history="synthetic"),
+    # the same layer (same inputs) on folded weights: q_lat = (W_UK^T W_Q) h, out = (W_O W_UV) o_lat
+    "v3_layer_folded_b128_ctx8192": Workload("v3_layer_folded_b128_ctx8192", "decode_layer", B=128, H=128,
+                                             d_model=7168, d_c=512, d_hR=64, qk_nope=128, v_head=128,
+                                             dtype="bf16", seed=_seed(4), ctx=8192, history="synthetic",
+                                             fold=True),
     # causal prefill at V2 sizes with materialised K/V
     "v2_prefill_b4_s4096": Workload("v2_prefill_b4_s4096", "prefill", B=4, H=128, d_model=5120,
                                     d_c=512, d_hR=64, qk_nope=128, v_head=128, dtype="bf16",
@@ -99,7 +105,7 @@ WORKLOADS: Dict[str, Workload] = {
 # the order the workloads are listed in (smallest first)
 ORDER = ["tiny_fp32_layer", "v3_decode_b32_ctx4096", "v3_decode_fp8_b32_ctx4096", "v3_mtp_b32_ctx4096_q2",
          "v3_ragged_b64", "v3_chunk_b4_ctx4096_c1024",
-         "v3_layer_b128_ctx8192", "v2_prefill_b4_s4096"]
+         "v3_layer_b128_ctx8192", "v3_layer_folded_b128_ctx8192", "v2_prefill_b4_s4096"]
 
 
 def shrink(w: Workload, **over) -> Workload:
