@@ -26,11 +26,17 @@ namespace tc {
 
 namespace {
 
-constexpr int kBM = 128, kBK = 64, kGroupRows = 16;
+// A k-block is kSub TMA boxes of 64 columns (one 128-byte swizzle atom) per operand, so each
+// operand row is read in kSub * 128 contiguous bytes per stage: 2 boxes up to BN = 128 (the
+// weight-streaming shapes, where longer runs per row read DRAM better), 1 box for BN = 256
+// (whose stages would otherwise drop to two).
+constexpr int kBM = 128, kBox = 64, kGroupRows = 16;
 constexpr int kSwapMinTokens = 1024;   // token-major from this many tokens on
 
 template <int BN>
 struct GemmCfg {
+    static constexpr int kSub = BN >= 256 ? 1 : 2;
+    static constexpr int kBK = kBox * kSub;
     static constexpr int X_BYTES = kBM * kBK * 2;
     static constexpr int Y_BYTES = BN * kBK * 2;
     static constexpr int STAGE = X_BYTES + Y_BYTES;
@@ -89,6 +95,7 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     int Ny, int K, int Z, GemmOut out, int chain_head, int x_2d, int y_2d, int swap,
                     int* err_code, long long* err_detail) {
     using C = GemmCfg<BN>;
+    constexpr int kSub = C::kSub, kBK = C::kBK;
     constexpr int stages = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = (uint8_t*)(((uintptr_t)smem_raw + 1023) & ~(uintptr_t)1023);
@@ -139,16 +146,22 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
             ptx::tma_prefetch(&tmX);
             ptx::tma_prefetch(&tmY);
             auto load_x = [&](uint8_t* st, uint64_t* bar, int kb, const Tile& tl) {
-                if (x_2d)
-                    ptx::tma_load_2d(st, &tmX, bar, kb * kBK, tl.i0);
-                else
-                    ptx::tma_load_3d(st, &tmX, bar, kb * kBK, tl.i0, tl.z);
+#pragma unroll
+                for (int b = 0; b < kSub; ++b) {
+                    if (x_2d)
+                        ptx::tma_load_2d(st + b * kBM * 128, &tmX, bar, kb * kBK + b * kBox, tl.i0);
+                    else
+                        ptx::tma_load_3d(st + b * kBM * 128, &tmX, bar, kb * kBK + b * kBox, tl.i0, tl.z);
+                }
             };
             auto load_y = [&](uint8_t* st, uint64_t* bar, int kb, const Tile& tl) {
-                if (y_2d)
-                    ptx::tma_load_2d(st + C::X_BYTES, &tmY, bar, kb * kBK, tl.j0);
-                else
-                    ptx::tma_load_3d(st + C::X_BYTES, &tmY, bar, kb * kBK, tl.j0, tl.z);
+#pragma unroll
+                for (int b = 0; b < kSub; ++b) {
+                    if (y_2d)
+                        ptx::tma_load_2d(st + C::X_BYTES + b * BN * 128, &tmY, bar, kb * kBK + b * kBox, tl.j0);
+                    else
+                        ptx::tma_load_3d(st + C::X_BYTES + b * BN * 128, &tmY, bar, kb * kBK + b * kBox, tl.j0, tl.z);
+                }
             };
             // The weights (X weights-major, Y token-major) of the first stages do not depend
             // on earlier kernels: start them before waiting for those; the activations do.
@@ -217,8 +230,9 @@ gemm_bf16_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_consta
                     const uint32_t a = ptx::smem_u32(smem + s * C::STAGE);
                     const uint32_t b = a + C::X_BYTES;
 #pragma unroll
-                    for (int k = 0; k < kBK / 16; ++k)
-                        ptx::mma_ss(d, ptx::desc_kmajor_sw128(a + 32 * k), ptx::desc_kmajor_sw128(b + 32 * k), idesc,
+                    for (int k = 0; k < kBK / 16; ++k)   // box k / 4, K-step k % 4 within it
+                        ptx::mma_ss(d, ptx::desc_kmajor_sw128(a + (k >> 2) * kBM * 128 + 32 * (k & 3)),
+                                    ptx::desc_kmajor_sw128(b + (k >> 2) * BN * 128 + 32 * (k & 3)), idesc,
                                     (kb | k) != 0);
                     ptx::mma_commit(&empty[s]);
                 }
@@ -440,8 +454,8 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
     const uint64_t sa[2] = {(uint64_t)sAm * 2, (uint64_t)sAz * 2};
     const uint64_t db[3] = {(uint64_t)K, (uint64_t)N, (uint64_t)Z};
     const uint64_t sb[2] = {(uint64_t)sBn * 2, (uint64_t)sBz * 2};
-    const uint32_t bx[3] = {(uint32_t)kBK, (uint32_t)kBM, 1};   // the 128-row operand
-    const uint32_t by[3] = {(uint32_t)kBK, (uint32_t)BN, 1};    // the BN-row operand
+    const uint32_t bx[3] = {(uint32_t)kBox, (uint32_t)kBM, 1};   // the 128-row operand
+    const uint32_t by[3] = {(uint32_t)kBox, (uint32_t)BN, 1};    // the BN-row operand
     const CUtensorMapDataType dt = out.in_f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     if (!make_tmap(&ma, dt, 2, A, a_bcast ? 2 : 3, da, sa, swap ? by : bx, 128) ||
         !make_tmap(&mb, dt, 2, B, b_bcast ? 2 : 3, db, sb, swap ? bx : by, 128))
