@@ -437,11 +437,12 @@ cudaError_t gemm_bf16_tc(int Z, int M, int N, int K, const __nv_bfloat16* A, lon
                       (out.period == 0 || (out.period % 2 == 0 && out.rope_start % 2 == 0)) &&
                       (!out.f16 || out.period == 0 || (out.period % 32 == 0 && out.rope_start % 32 == 0));
     const int Mx = swap ? N : M, Ny = swap ? M : N;   // MMA rows (128-tiles) and columns (BN-tiles)
-    // the narrowest tile that covers Ny, narrowed further while there are fewer tiles than a
-    // quarter of the SMs (very skinny weight-streaming GEMMs: the weights are then re-read
-    // from L2)
+    // the narrowest tile that covers Ny, narrowed to 64 while there are fewer tiles than two
+    // waves of CTAs, and further to 32 while fewer than a quarter of the SMs (skinny
+    // weight-streaming GEMMs: more CTAs stream the weights, the operand re-reads come from L2)
     int BN = Ny <= 32 ? 32 : Ny <= 64 ? 64 : Ny <= 128 ? 128 : 256;
     const long long xtiles = (long long)Z * ((Mx + 127) / 128);
+    while (BN > 64 && xtiles * ((Ny + BN - 1) / BN) < 2 * sms) BN >>= 1;
     while (BN > 32 && xtiles * ((Ny + BN - 1) / BN) < sms / 4) BN >>= 1;
     const bool b_bcast = sBz == 0;   // one B for every z: a 2-D map
     const bool a_bcast = sAz == 0 && Z > 1;
