@@ -75,13 +75,18 @@ static_assert(kF8TileBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment
 // dequantisation warps turn it in place into an fp16 tile (code x scale) of the same layout;
 // the latent MMAs then run on fp16 operands (q_lat and P in fp16 too).
 template <bool kF8> struct DecCfg;
+// kSplitIssue: the score MMAs and the P c MMAs are issued by two threads in different warps
+// (warp 1 and warp 14), each waiting only for its own operands, so a ready P is not held up
+// behind the issue of the next score batch.  Otherwise one thread issues both (warp 1).
 template <> struct DecCfg<false> {
     static constexpr int kStages = 4, kStageBytes = kTileBytes, kXBufs = 2;
-    static constexpr int kThreads = 448;   // producer, MMA, 4 sender and 8 softmax warps
+    static constexpr int kThreads = 480;   // producer, S issuer, 4 sender, 8 softmax warps, P c issuer
+    static constexpr bool kSplitIssue = true;
 };
 template <> struct DecCfg<true> {
     static constexpr int kStages = 4, kStageBytes = kF8TileBytes, kXBufs = 2;
-    static constexpr int kThreads = 512;   // + 2 dequantisation warps
+    static constexpr int kThreads = 512;   // producer, MMA, 4 sender, 8 softmax, 2 dequantisation warps
+    static constexpr bool kSplitIssue = false;
 };
 // Shared memory: the ring of kStages tiles, kXBufs receive buffers for the peer's partial
 // scores and kXBufs staging buffers for this CTA's own (each kXBytes).  The
@@ -318,7 +323,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         ptx::mbar_init(&o_done[0], 1);
         ptx::mbar_init(&o_done[1], 1);
         ptx::mbar_init(q_ready, 128);
-        ptx::mbar_init(drain, 1);
+        ptx::mbar_init(drain, DecCfg<kF8>::kSplitIssue ? 2 : 1);
         for (int i = 0; i < 2; ++i) {
             ptx::mbar_init(&x_full[i], 1);
             ptx::mbar_init(&x_empty[i], 8);
@@ -535,6 +540,64 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
             }
         }
         if (!ok) fail(err_code, err_detail, abort_flag, 6);
+    } else if (DecCfg<kF8>::kSplitIssue && (warp == 1 || warp == 14)) {
+        // ------------------------------------------- MMA issuers: S (warp 1), P c (warp 14)
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, kT, 0, 0);
+            constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, 256, 0, 1);
+            uint32_t g = 0, sidx = 0;
+            bool ok = true;
+            Seg sq;
+            SegIter<kSib> iq = it;
+            while (ok && !*abort_flag && iq.next(sq)) {
+                for (int j = sq.j0; j < sq.j1; ++j, ++g) {
+                    const int st = g % kStages;
+                    if (warp == 1) {
+                        // S of tile g: its tile has landed, S(g - 1) has been read, and at a piece's
+                        // first tile the piece's query is in TMEM
+                        if (j == sq.j0) {
+                            if (!ptx::mbar_wait(q_ready, sidx & 1, abort_flag)) { ok = false; break; }
+                            ++sidx;
+                        }
+                        if (!ptx::mbar_wait(&tile_full[st], (g / kStages) & 1, abort_flag) ||
+                            (g > 0 && !ptx::mbar_wait(s_free, (g - 1) & 1, abort_flag))) {
+                            ok = false;
+                            break;
+                        }
+                        ptx::tc_fence_after();
+                        const uint32_t t = ptx::smem_u32(tiles + st * kStride);
+#pragma unroll
+                        for (int ks = 0; ks < 16; ++ks)   // latent columns: 4 chunks x 4 K-steps
+                            ptx::mma_ts(tmem + kColS, tmem + kColQ + 8 * ks,
+                                        ptx::desc_kmajor_sw128(t + (ks >> 2) * kChunkBytes + (ks & 3) * 32), idesc_s,
+                                        ks != 0);
+#pragma unroll
+                        for (int ks = 0; ks < 2; ++ks)    // this CTA's half of the rotary columns
+                            ptx::mma_ss(tmem + kColS, ptx::desc_kmajor_sw64(ptx::smem_u32(qrope) + 32 * ks),
+                                        ptx::desc_kmajor_sw64(t + 4 * kChunkBytes + 32 * ks), idesc_s, 1);
+                        ptx::mma_commit(s_full);
+                    } else {
+                        // O += P c of tile g once its P is in TMEM (the softmax writes a piece's
+                        // first P only after reading the previous piece's O)
+                        if (!ptx::mbar_wait(&p_ready[g & 1], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+                        ptx::tc_fence_after();
+                        const uint32_t v = ptx::smem_u32(tiles + st * kStride);
+                        const bool first = (j == sq.j0);
+#pragma unroll
+                        for (int k = 0; k < kT / 16; ++k)
+                            ptx::mma_ts(tmem + kColO, tmem + kColP + 32 * (g & 1) + 8 * k,
+                                        ptx::desc_mnmajor_sw128(v + 2048 * k, kChunkBytes), idesc_o,
+                                        !(first && k == 0));
+                        ptx::mma_commit(&o_done[g & 1]);
+                        ptx::mma_commit(&tile_empty[st]);
+                    }
+                }
+            }
+            if (!ok) fail(err_code, err_detail, abort_flag, 2);
+            // drain: wait (bounded) until the MMAs of both issuers have completed
+            ptx::mma_commit(drain);
+            if (!ptx::mbar_wait(drain, 0, nullptr)) fail(err_code, err_detail, abort_flag, 4);
+        }
     } else if (warp == 1) {
         // ------------------------------------------------------------- MMA issuer
         if (lane == 0) {
