@@ -25,9 +25,10 @@
 // softmax of tile g + 1 does not wait for the O MMAs of tile g.  The latent score MMAs and
 // the O MMAs read A from TMEM and only the tile from shared memory.
 //
-// Warp roles (448 threads): warp 0 issues TMA loads of 64-token tiles (4 latent boxes of
+// Warp roles (480 threads): warp 0 issues TMA loads of 64-token tiles (4 latent boxes of
 // 64 columns with 128-byte swizzle + this CTA's 32 rotary columns with 64-byte swizzle,
-// 36 KB) into a 4-stage ring; warp 1 owns TMEM and issues the MMAs; warps 2-5 (thread = head
+// 36 KB) into a 5-stage ring; warp 1 owns TMEM and issues the score MMAs, warp 14 the
+// P c MMAs (FP8 rows: warp 1 issues both, warps 14-15 dequantise); warps 2-5 (thread = head
 // = TMEM lane) load Q and send partial scores to the peer; warps 6-13 (two per TMEM
 // subpartition, one per half tile) run the online softmax (base-2, lazy rescale: the running
 // max moves only when a tile exceeds it by more than 8, so p <= 256), write P, and read O
@@ -78,8 +79,11 @@ template <bool kF8> struct DecCfg;
 // kSplitIssue: the score MMAs and the P c MMAs are issued by two threads in different warps
 // (warp 1 and warp 14), each waiting only for its own operands, so a ready P is not held up
 // behind the issue of the next score batch.  Otherwise one thread issues both (warp 1).
+// bf16 rows: 5 stages and one partial-score exchange buffer per direction; the stage a TMA
+// load waits for is then freed one tile earlier, and the ring, not the exchange, was what
+// held the score MMAs back.  FP8 rows keep 4 stages (a fifth does not fit) and two buffers.
 template <> struct DecCfg<false> {
-    static constexpr int kStages = 4, kStageBytes = kTileBytes, kXBufs = 2;
+    static constexpr int kStages = 5, kStageBytes = kTileBytes, kXBufs = 1;
     static constexpr int kThreads = 480;   // producer, S issuer, 4 sender, 8 softmax warps, P c issuer
     static constexpr bool kSplitIssue = true;
 };
