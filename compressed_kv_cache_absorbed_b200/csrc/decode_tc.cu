@@ -60,14 +60,14 @@ constexpr int kXBytes = 128 * kXRowBytes;     // one exchange buffer: 128 heads 
 constexpr int kBarBytes = 256 + 2048 + 256;
 // FP8 cache rows (see decode_tc.cuh): per tile and CTA, this CTA's 256 codes (two 128-byte
 // boxes, 128-byte swizzle), its 32 rotary columns (bf16, 64-byte swizzle) and the 64 rows'
-// 16-byte scale fields (the fp32 scale first).  They land in place in a stage one KB larger
-// than a bf16 tile: the codes in the upper half of the latent area (fp16 boxes 2 and 3), the
-// rotary box where the tile keeps it, the scales after it; the dequantisation warps then
-// expand the codes into the four fp16 latent boxes.
+// 16-byte scale fields (the fp32 scale first).  They land in place in a stage the size of a
+// bf16 tile: the codes in the upper half of the latent area (fp16 boxes 2 and 3), the rotary
+// box where the tile keeps it, the scales at the start of fp16 box 0 (read before box 0 is
+// written); the dequantisation warps then expand the codes into the four fp16 latent boxes.
 constexpr int kF8CodeBytes = kT * 128;
 constexpr int kF8CodeOffset = 2 * kChunkBytes;        // code boxes at fp16 boxes 2, 3
-constexpr int kF8StageScaleOffset = kTileBytes;        // after the rotary box
-constexpr int kF8TileBytes = kTileBytes + kT * 16;     // 37 KB
+constexpr int kF8StageScaleOffset = 0;                 // in fp16 box 0, written last
+constexpr int kF8TileBytes = kTileBytes;               // 36 KB
 constexpr int kF8LoadBytes = 2 * kF8CodeBytes + kRopeBytes + kT * 16;
 static_assert(kF8TileBytes % 1024 == 0, "FP8 stages keep the 1024-byte alignment of the swizzled boxes");
 
@@ -88,7 +88,7 @@ template <> struct DecCfg<false> {
     static constexpr bool kSplitIssue = true;
 };
 template <> struct DecCfg<true> {
-    static constexpr int kStages = 4, kStageBytes = kF8TileBytes, kXBufs = 2;
+    static constexpr int kStages = 5, kStageBytes = kF8TileBytes, kXBufs = 1;
     static constexpr int kThreads = 512;   // producer, MMA, 4 sender, 8 softmax, 2 dequantisation warps
     static constexpr bool kSplitIssue = false;
 };
@@ -102,6 +102,13 @@ constexpr int dec_smem() {
            kBarBytes;
 }
 static_assert(dec_smem<false>() <= 232448, "decode kernel shared memory over the 227 KB limit");
+// The barrier area: tile_full and tile_empty [kStages], 20 single barriers from s_full on,
+// f8_full [kStages], the pair's 2 x 2 x 128 floats, then the TMEM slot, the abort flag and
+// the planning's 16 + 2 ints.
+template <bool kF8>
+constexpr int dec_bar_bytes() { return (3 * DecCfg<kF8>::kStages + 20) * 8 + 512 * 4 + (2 + 16 + 2) * 4; }
+static_assert(dec_bar_bytes<false>() <= kBarBytes && dec_bar_bytes<true>() <= kBarBytes,
+              "decode kernel barrier area over its reserved bytes");
 static_assert(dec_smem<true>() <= 232448, "FP8 decode kernel shared memory over the 227 KB limit");
 constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
@@ -301,8 +308,8 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
     uint64_t* xs_ready = s_full + 12;  // [kXB] all 128 rows of xstage[g % kXB] written
     uint64_t* xs_free = s_full + 14;   // [kXB] the local softmax has read xstage[g % kXB]
     uint64_t* pair_bar = s_full + 16;  // [4] the two softmax warps of a subpartition
-    uint64_t* f8_full = s_full + 20;   // [4] a stage's FP8 data landed (FP8 rows)
-    float* pair_val = (float*)(s_full + 24);   // [2][2][128] values the two warps swap
+    uint64_t* f8_full = s_full + 20;   // [kStages] a stage's FP8 data landed (FP8 rows)
+    float* pair_val = (float*)(f8_full + kStages);   // [2][2][128] values the two warps swap
     uint32_t* tmem_slot = (uint32_t*)(pair_val + 512);
     volatile int* abort_flag = (volatile int*)(tmem_slot + 1);
     int* plan_wsum = (int*)(tmem_slot + 2);   // [16] per-warp sums of the planning scans
@@ -506,10 +513,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
         uint32_t g = 0;
         bool ok = true;
         Seg cur;
-        auto expand = [&](uint8_t* tl, int k, uint4 c, int box) {   // unit e = dt + 64 k of code box `box`
+        // unit e = dt + 64 k of code box `box`, row r = e / 8, whose scale is sc
+        auto expand = [&](uint8_t* tl, int k, uint4 c, int box, float sc) {
             const int e = dt + 64 * k;
             const int r = e >> 3, u = e & 7, sw = r & 7;       // row, unit within the code box
-            const float sc = *(const float*)(tl + kF8StageScaleOffset + r * 16);
             uint4 lo, hi;
             dequant16(c, __float2half2_rn(sc), lo, hi);
             // latent columns 128 box + 16 u .. + 15: fp16 box 2 box + (u >> 2), units 2 (u & 3), + 1
@@ -531,14 +538,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tm_cache, const __grid_cons
                     break;
                 }
                 uint8_t* tl = tiles + s * kStride;
-#pragma unroll 4
-                for (int k = 0; k < 8; ++k) expand(tl, k, code_unit(tl, k, 0), 0);
+                float sc[8];   // the scales of this thread's rows (dt / 8 + 8 k), both code boxes
+#pragma unroll
+                for (int k = 0; k < 8; ++k) sc[k] = *(const float*)(tl + kF8StageScaleOffset + ((dt + 64 * k) >> 3) * 16);
+                ptx::named_barrier_sync(8, 64);   // every scale is read before fp16 box 0 covers them
+#pragma unroll
+                for (int k = 0; k < 8; ++k) expand(tl, k, code_unit(tl, k, 0), 0, sc[k]);
                 uint4 c1[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) c1[k] = code_unit(tl, k, 1);
                 ptx::named_barrier_sync(8, 64);   // every code of the stage is read
 #pragma unroll
-                for (int k = 0; k < 8; ++k) expand(tl, k, c1[k], 1);
+                for (int k = 0; k < 8; ++k) expand(tl, k, c1[k], 1, sc[k]);
                 ptx::fence_proxy_async_smem();   // read by the tensor cores
                 ptx::mbar_arrive(&tile_full[s]);
             }
