@@ -79,9 +79,9 @@ template <bool kF8> struct DecCfg;
 // kSplitIssue: the score MMAs and the P c MMAs are issued by two threads in different warps
 // (warp 1 and warp 14), each waiting only for its own operands, so a ready P is not held up
 // behind the issue of the next score batch.  Otherwise one thread issues both (warp 1).
-// bf16 rows: 5 stages and one partial-score exchange buffer per direction; the stage a TMA
-// load waits for is then freed one tile earlier, and the ring, not the exchange, was what
-// held the score MMAs back.  FP8 rows keep 4 stages (a fifth does not fit) and two buffers.
+// Both variants: 5 stages and one partial-score exchange buffer per direction (a fifth stage
+// fits only beside one buffer).  With 4 stages the next score batch often waited for its
+// tile to land; the ring, not the exchange, held the score MMAs back.
 template <> struct DecCfg<false> {
     static constexpr int kStages = 5, kStageBytes = kTileBytes, kXBufs = 1;
     static constexpr int kThreads = 480;   // producer, S issuer, 4 sender, 8 softmax warps, P c issuer
