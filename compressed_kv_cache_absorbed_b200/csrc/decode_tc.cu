@@ -114,11 +114,11 @@ constexpr uint32_t kColQ = 0, kColS = 128, kColP = 192, kColO = 256, kTmemCols =
 constexpr float kRescaleThreshold = 8.0f;     // log2 units
 
 // The work split counts cost units: one per tile plus kPieceCost for every sequence start
-// (a new piece costs its partial's epilogue and a query reload, measured at about three
-// tiles), so clusters whose range starts sequences get fewer tiles.  Tile j of sequence b
-// sits at cost position first[b] + j, with first[b] = (cost of all earlier sequences) +
-// kPieceCost.
-constexpr int kPieceCost = 3;
+// (a new piece costs its partial's epilogue and a query reload: a switch stalls the score
+// MMAs ~4.5 us, about five 64-token tiles), so clusters whose range starts sequences get
+// fewer tiles.  Tile j of sequence b sits at cost position first[b] + j, with first[b] =
+// (cost of all earlier sequences) + kPieceCost.
+constexpr int kPieceCost = 5;
 
 // The merge kernel recomputes this split from the offsets (it needs each sequence's first
 // and last cost positions and the cost units per cluster).
